@@ -1,0 +1,428 @@
+"""Benchmark of the paged-KV decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--block-size B] [--cache-dtype bf16|f16|fp8_e4m3]
+                    [--impl ours|reference] [--no-cpu-baseline]
+
+One step = the whole hot path over one batch: reshape_and_cache of the step's
+new tokens (one per sequence), then paged_attn_decode (decode kernel + merge
+kernel) over every sequence, all through the C ABI. Default workload: the
+Llama-3-8B-shaped decode (64 sequences, lens ~ U[512, 4096], 32 q / 8 kv
+heads, D = 128, B = 16, bf16; about 604 MB of K/V, larger than the 126 MB L2,
+so no flush is needed between steps).
+
+metric / value: K+V bytes the decode reads per step (sum of L_s * 2 * Hk * D *
+elem) divided by the device time of a step, in GB/s, summed over ranks. With
+N > 1 each rank runs its own replica (the path has no exchange step), so
+scaling is weak. Rank 0 prints one JSON line.
+
+--impl reference times the fp64 CPU oracle on bounded samples of the same
+workload on the host cores (the only other place this file runs oracle/).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads as W  # noqa: E402
+
+METRIC = "paged decode attention HBM GB/s (KV bytes read/s) and % of B200 peak; seqs/s"
+UNIT = "GB/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--workload", default="llama3_8b")
+    ap.add_argument("--block-size", type=int, default=None)
+    ap.add_argument("--cache-dtype", default=None)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=None)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+def workload_spec(a) -> W.Spec:
+    over = {}
+    if a.block_size:
+        over["block_size"] = a.block_size
+    if a.cache_dtype:
+        over["cache_dtype"] = a.cache_dtype
+        if a.cache_dtype in ("f16", "bf16"):
+            over["q_dtype"] = a.cache_dtype
+    s = W.spec(a.workload, **over)
+    if s.lens[0] == "prefix":
+        raise SystemExit("bench.py times the layouts drawn by workloads.make_layout")
+    return s.replace(append=True)
+
+
+def config_of(s: W.Spec, lay, kv_bytes: int) -> dict:
+    return {"workload": W.describe(s), "num_seqs": s.num_seqs,
+            "num_q_heads": s.num_q_heads, "num_kv_heads": s.num_kv_heads, "head_dim": s.head_dim,
+            "block_size": s.block_size, "cache_dtype": s.cache_dtype,
+            "tokens": int(lay.lens.sum()), "kv_bytes_per_step": kv_bytes,
+            "l2": "inputs larger than L2 (K/V pool > 126 MB), no flush",
+            "step": "reshape_and_cache(new token per seq) + paged_attn_decode"}
+
+
+def kv_bytes_of(s: W.Spec, lens) -> int:
+    return int(sum(int(L) for L in lens)) * 2 * s.num_kv_heads * s.head_dim * s.cache_elem_bytes
+
+
+def decode_alg_bytes(s: W.Spec, lens) -> int:
+    """Algorithmic bytes of one decode: K+V of every stored token, q and out,
+    the used block-table entries and the lengths (plus fp8 scales)."""
+    B = s.block_size
+    kv = kv_bytes_of(s, lens)
+    qo = 2 * s.num_seqs * s.num_q_heads * s.head_dim * 2
+    tab = sum(-(-int(L) // B) for L in lens) * 4 + 4 * s.num_seqs
+    sc = 2 * s.num_kv_heads * 4 if s.cache_dtype == "fp8_e4m3" else 0
+    return kv + qo + tab + sc
+
+
+# ---------------------------------------------------------------------------
+# clocks
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, device: int):
+        self.lines = []
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            ident = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", ident], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=5)
+        sms, maxs, reasons = [], [], set()
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sms.append(float(parts[0]))
+                maxs.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(self.NAMES, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sms:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxs), "reasons": sorted(reasons),
+                "samples": len(sms)}
+
+
+# ---------------------------------------------------------------------------
+# roofline helpers
+# ---------------------------------------------------------------------------
+
+def measured_peak_hbm():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for f in ("decode.cuh", "ptx.cuh"):
+        with open(os.path.join(ROOT, "paged_kv_cache_453_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(s: W.Spec):
+    """DRAM bytes per decode launch from the committed ncu summary, if it was
+    taken on the current kernel source and this workload."""
+    p = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    key = f"{s.name}/{s.cache_dtype}/B{s.block_size}"
+    e = d.get(key)
+    if not e or e.get("kernel_sha") != kernel_source_sha():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline leg and the reference arm)
+# ---------------------------------------------------------------------------
+
+def _blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d["num_threads"] for d in threadpool_info() if d.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return 1
+
+
+def _host_inputs(s: W.Spec, lay, t):
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from oracle_io import raw
+    ks = None if t.k_scale is None else t.k_scale.cpu().numpy()
+    vs = None if t.v_scale is None else t.v_scale.cpu().numpy()
+    return raw(t.q), raw(t.k_cache), raw(t.v_cache), lay.tables.numpy(), lay.lens.numpy(), ks, vs
+
+
+def oracle_rate(s: W.Spec, host, seqs) -> tuple:
+    """(seconds, KV bytes) of the oracle over the given sequences."""
+    from oracle.attention import paged_decode
+    q, kp, vp, tab, lens, ks, vs = host
+    t0 = time.perf_counter()
+    paged_decode(q, kp, vp, tab, lens, s.scale, s.block_size, s.q_dtype, s.cache_dtype, k_scale=ks,
+                 v_scale=vs, seqs=seqs)
+    dt = time.perf_counter() - t0
+    return dt, kv_bytes_of(s, [lens[i] for i in seqs])
+
+
+def cpu_baseline(s: W.Spec, host, budget_s: float) -> dict:
+    S = s.num_seqs
+    dt1, _ = oracle_rate(s, host, [0])
+    n = max(1, min(S, int(budget_s / max(dt1, 1e-3))))
+    seqs = list(range(n))
+    dt, nbytes = oracle_rate(s, host, seqs)
+    return {"value": nbytes / dt / 1e9, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"fp64 numpy oracle on the first {n} of {S} sequences ({nbytes} K/V bytes), "
+                      f"{dt:.1f} s", "seqs_per_s": n / dt}
+
+
+# ---------------------------------------------------------------------------
+
+def dist_setup(a):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    pg = None
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        pg = dist
+    return ws, rank, local, pg
+
+
+def run_reference(a, s: W.Spec, ws: int, rank: int):
+    if rank != 0:
+        return
+    lay = W.make_layout(s)
+    t = W.make_tensors(s, lay.num_blocks, lay.fill_tables, lay.fill_lens, device="cpu")
+    host = _host_inputs(s, lay, t)
+    # Size each step's sample so that warm-up + steps take about 2 minutes.
+    dt1, _ = oracle_rate(s, host, [0])
+    per_step = 120.0 / max(1, a.steps + a.warmup)
+    frac = min(1.0, per_step / max(dt1, 1e-6))
+    S = s.num_seqs
+    order = list(range(S))
+
+    def step(i):
+        seq = order[i % S]
+        if frac >= 1.0:
+            return oracle_rate(s, host, [seq])
+        # part of one sequence: its first ceil(frac * L) tokens
+        L = int(host[4][seq])
+        n = max(1, int(math.ceil(frac * L)))
+        lens = host[4].copy()
+        lens[seq] = n
+        h2 = host[:4] + (lens,) + host[5:]
+        return oracle_rate(s, h2, [seq])
+
+    for i in range(a.warmup):
+        step(i)
+    tot_t, tot_b = 0.0, 0
+    for i in range(a.steps):
+        dt, nb = step(a.warmup + i)
+        tot_t += dt
+        tot_b += nb
+    value = tot_b / tot_t / 1e9
+    sample = (f"each step: fp64 numpy oracle on one sequence of the workload"
+              + ("" if frac >= 1.0 else f", its first {frac:.3%} of tokens"))
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * tot_t / max(1, a.steps),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_of(s, lay, kv_bytes_of(s, lay.lens.tolist())),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }))
+
+
+def main():
+    a = parse()
+    s = workload_spec(a)
+    ws, rank, local, dist = dist_setup(a)
+    if a.impl == "reference":
+        run_reference(a, s, ws, rank)
+        if dist:
+            dist.destroy_process_group()
+        return
+
+    import paged_kv_cache_453_b200 as P
+    from paged_kv_cache_453_b200.build import build
+    if rank == 0:
+        build()
+    if dist:
+        dist.barrier()
+    dev = local
+    torch.cuda.set_device(dev)
+    lay = W.make_layout(s)
+    t = W.make_tensors(s, lay.num_blocks, lay.fill_tables, lay.fill_lens, device=f"cuda:{dev}")
+    tables, lens = lay.tables.cuda(), lay.lens.cuda()
+    slots = lay.slot_mapping.cuda()
+    out = torch.empty_like(t.q)
+    fp8 = s.cache_dtype == "fp8_e4m3"
+    reshape = P.prepare_reshape(t.k_new, t.v_new, t.k_cache, t.v_cache, slots, t.k_scale, t.v_scale)
+    decode = P.prepare_decode(t.q, t.k_cache, t.v_cache, tables, lens, s.num_kv_heads, s.scale,
+                              s.block_size, out, t.k_scale, t.v_scale)
+    lens_l = lay.lens.tolist()
+    kv_bytes = kv_bytes_of(s, lens_l)
+    alg = decode_alg_bytes(s, lens_l)
+
+    for _ in range(max(3, a.warmup)):
+        reshape()
+        decode()
+    torch.cuda.synchronize()
+    st = P.device_error(dev)
+    if st != P.PKV_OK:
+        raise SystemExit(f"device check failed during warm-up: {P.status_string(st)}")
+
+    K = a.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(dev)
+    time.sleep(0.3 if clocks.proc else 0)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start.record()
+    for i in range(K):
+        reshape()
+        ev[i][0].record()
+        decode()
+        ev[i][1].record()
+    stop.record()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clk = clocks.stop()
+    elapsed_ms = start.elapsed_time(stop)
+    dec_ms = sum(e0.elapsed_time(e1) for e0, e1 in ev) / K
+    if dist:
+        tt = torch.tensor([elapsed_ms, dec_ms], device=f"cuda:{dev}", dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        elapsed_ms, dec_ms = float(tt[0]), float(tt[1])
+    st = P.device_error(dev)
+    if st != P.PKV_OK:
+        raise SystemExit(f"device check failed: {P.status_string(st)}")
+    step_s = elapsed_ms / 1e3 / K
+    value = ws * kv_bytes / step_s / 1e9
+    launches_per_step = 3  # reshape_and_cache, decode_kernel, decode_merge_kernel
+
+    # ---- end to end through the public API: pinned host in, result out ----
+    Ke = a.e2e_steps or max(3, min(K, 2000))
+    pin = lambda x: x.cpu().pin_memory()  # noqa: E731
+    h_in = {"q": pin(t.q), "k_new": pin(t.k_new), "v_new": pin(t.v_new), "slots": pin(lay.slot_mapping),
+            "tables": pin(lay.tables), "lens": pin(lay.lens)}
+    h_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    d_in = {"q": t.q, "k_new": t.k_new, "v_new": t.v_new, "slots": slots, "tables": tables, "lens": lens}
+    h2d = sum(x.numel() * x.element_size() for x in h_in.values())
+    d2h = h_out.numel() * h_out.element_size()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(Ke):
+        for k_, x in h_in.items():
+            d_in[k_].copy_(x, non_blocking=True)
+        reshape()
+        decode()
+        h_out.copy_(out, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if dist:
+        tt = torch.tensor([e2e_ms], device=f"cuda:{dev}", dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt[0])
+    e2e_value = ws * kv_bytes / (e2e_ms / 1e3 / Ke) / 1e9
+
+    if rank != 0:
+        if dist:
+            dist.destroy_process_group()
+        return
+    peak, peak_src = measured_peak_hbm()
+    achieved = alg / (dec_ms / 1e3) / 1e9
+    cpu = None
+    if ws == 1 and not a.no_cpu_baseline:
+        cpu = cpu_baseline(s, _host_inputs(s, lay, t), a.cpu_seconds)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": K, "warmup": a.warmup,
+        "ms_per_step": elapsed_ms / K, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp8_e4m3" if fp8 else s.cache_dtype, "data": "synthetic",
+        "config": config_of(s, lay, kv_bytes) | {"parallelism": f"replicas x{ws}"},
+        "seqs_per_s": ws * s.num_seqs / step_s,
+        "pct_of_hbm_peak": 100.0 * value / ws / peak,
+        "roofline": {"kernel": "paged_attn_decode (decode_kernel + decode_merge_kernel)", "bound": "hbm",
+                     "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": profiled_traffic(s), "peak_source": peak_src,
+                     "alg_bytes_per_launch": alg, "us_per_launch": dec_ms * 1e3},
+        "cpu_baseline": cpu,
+        "clocks": clk,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": Ke, "ms_per_step": e2e_ms / Ke},
+        "gpu_launches": launches_per_step * K,
+    }
+    print(json.dumps(line))
+    if dist:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,288 @@
+/*
+ * pagedkv.h - C ABI of libpagedkv.so: paged-KV decode attention for B200
+ * (sm_100a) and the host block allocator that builds its block tables.
+ *
+ * The method ("PagedAttention: treat the cache like virtual memory",
+ * "KV-Cache Management and PagedAttention"; "PagedAttention: OS Virtual Memory
+ * Architecture for GPUs" and "Under the Hood: The PagedAttention CUDA Kernel",
+ * "PagedAttention and KV Cache Management"): each sequence's KV cache is cut
+ * into fixed-size blocks of B tokens that live anywhere in a shared pool; a
+ * per-sequence block table maps logical block i (tokens iB .. iB+B-1) to its
+ * physical block, and the attention kernel takes that table as an argument and
+ * gathers K and V through it.
+ *
+ * Conventions shared by every device call
+ *   - Tensors are described by pkv_tensor: a DEVICE pointer, an element type,
+ *     up to 4 dims, and strides in ELEMENTS. The innermost dim must be
+ *     contiguous (stride 1). The caller owns every buffer; the library never
+ *     frees or keeps a pointer past the call.
+ *   - Pool layout ("HND" per block): k_cache and v_cache are
+ *     [num_blocks, num_kv_heads, block_size, head_dim], head_dim contiguous,
+ *     strides non-decreasing outward with every byte stride a multiple of 16
+ *     and the base 16-byte aligned. One (block, kv head) is one contiguous
+ *     block_size * head_dim run.
+ *   - Calls are asynchronous: the work is enqueued on `stream`
+ *     (a cudaStream_t passed as void*; NULL = the legacy default stream) and
+ *     nothing synchronises it. Arguments are checked on the host before any
+ *     launch; a bad argument returns PKV_ERR_INVALID_ARG (or
+ *     PKV_ERR_UNSUPPORTED for a valid but unimplemented shape) and launches
+ *     nothing. A failed launch returns PKV_ERR_CUDA.
+ *   - Device-side checks (a block id outside the pool, a context length
+ *     beyond the table row, a bounded wait that ran out) never fault: the
+ *     kernel records the problem in a per-device flag and carries on with
+ *     safe values. pkv_device_error() reads and clears that flag.
+ *   - Supported shapes: head_dim 64 or 128 (128 for fp8), block_size 16 or
+ *     32, num_q_heads = g * num_kv_heads with 1 <= g <= 8.
+ *
+ * The host allocator calls touch no device memory and are not thread-safe
+ * per handle (one handle per scheduler thread).
+ */
+#ifndef PAGEDKV_H_
+#define PAGEDKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PKV_F16 = 0,       /* IEEE binary16 */
+  PKV_BF16 = 1,      /* bfloat16 */
+  PKV_FP8_E4M3 = 2,  /* OCP fp8 E4M3 codes, stored as bytes */
+  PKV_I32 = 3,
+  PKV_I64 = 4,
+  PKV_F32 = 5
+} pkv_dtype;
+
+typedef struct {
+  void* data;        /* device pointer */
+  int32_t dtype;     /* pkv_dtype */
+  int32_t ndim;      /* 1..4 */
+  int64_t shape[4];
+  int64_t stride[4]; /* elements */
+} pkv_tensor;
+
+typedef enum {
+  PKV_OK = 0,
+  PKV_ERR_INVALID_ARG = -1,
+  PKV_ERR_UNSUPPORTED = -2,
+  PKV_ERR_OOM = -3,          /* allocator: not enough free blocks */
+  PKV_ERR_UNKNOWN_SEQ = -4,  /* allocator: no such sequence */
+  PKV_ERR_EXISTS = -5,       /* allocator: sequence id already in use */
+  PKV_ERR_DOUBLE_FREE = -6,  /* allocator: reference count would drop below 0 */
+  PKV_ERR_CUDA = -7,         /* a CUDA runtime call failed */
+  PKV_ERR_DEVICE_CHECK = -8, /* a kernel recorded a bad index or a wait that ran out */
+  PKV_ERR_WORKSPACE = -9     /* caller-provided workspace too small */
+} pkv_status;
+
+/* Text for a status code (static storage, never NULL). */
+const char* pkv_status_string(int status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int pkv_version(void);
+
+/* ------------------------------------------------------------------------ */
+/* Decode attention                                                         */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * paged_attn_decode - one decode step of attention over a paged KV cache.
+ *
+ * Defined by "Under the Hood: The PagedAttention CUDA Kernel" ("PagedAttention
+ * and KV Cache Management") and the block-table diagram of "PagedAttention:
+ * treat the cache like virtual memory" ("KV-Cache Management and
+ * PagedAttention"). For every sequence s and query head i, with kv head
+ * h = i / g and L = context_lens[s]:
+ *     K_s[t] = k_cache[block_tables[s][t / B], h, t % B, :]   (same for V)
+ *     out[s, i, :] = softmax_t(scale * <q[s, i, :], K_s[t]>) . V_s
+ * over t = 0 .. L-1. L = 0 gives out = 0. Slots past L in the last block and
+ * table entries past ceil(L/B) are never read into the result (they may hold
+ * anything, NaN included).
+ *
+ *   q            [S, Hq, D] f16 | bf16, read only
+ *   k_cache      [NB, Hk, B, D], same dtype as q
+ *   v_cache      [NB, Hk, B, D], same dtype as q
+ *   block_tables [S, MB] int32 physical block ids; entries >= ceil(L/B) ignored
+ *   context_lens [S] int32, 0 <= L <= MB * B (the new token included)
+ *   num_kv_heads Hk (must equal k_cache.shape[1])
+ *   scale        softmax scale (usually 1/sqrt(D))
+ *   block_size   B (must equal k_cache.shape[2])
+ *   out          [S, Hq, D], same dtype as q, written
+ *
+ * Uses a per-device workspace owned by the library: the first call on a
+ * device (or one needing more) allocates it with cudaMalloc, which
+ * synchronises; later calls reuse it. Calls that share a device and overlap
+ * on the GPU must use paged_attn_decode_ex with separate workspaces.
+ */
+int paged_attn_decode(const pkv_tensor* q, const pkv_tensor* k_cache, const pkv_tensor* v_cache,
+                      const pkv_tensor* block_tables, const pkv_tensor* context_lens,
+                      int num_kv_heads, float scale, int block_size, pkv_tensor* out,
+                      void* stream);
+
+/*
+ * paged_attn_decode_fp8 - as paged_attn_decode with an fp8-e4m3 cache.
+ * An fp8 cache halves the bytes per element ("Planning capacity when context
+ * gets long", "KV-Cache Management and PagedAttention"; "The KV Cache Size
+ * Equation", "PagedAttention and KV Cache Management").
+ *
+ *   k_cache, v_cache  [NB, Hk, B, D] PKV_FP8_E4M3 codes
+ *   k_scale, v_scale  [Hk] f32 device: element value = decode(code) * scale[h]
+ *   q, out            f16 | bf16 (q is rounded to f16 for the dot products)
+ */
+int paged_attn_decode_fp8(const pkv_tensor* q, const pkv_tensor* k_cache,
+                          const pkv_tensor* v_cache, const pkv_tensor* k_scale,
+                          const pkv_tensor* v_scale, const pkv_tensor* block_tables,
+                          const pkv_tensor* context_lens, int num_kv_heads, float scale,
+                          int block_size, pkv_tensor* out, void* stream);
+
+/*
+ * Bytes of workspace a decode with these sizes needs on `device`
+ * (split-KV partial results, one small header). Depends on the device's SM
+ * count, not on the context lengths.
+ */
+size_t paged_attn_decode_workspace_bytes(int num_q_heads, int num_kv_heads, int head_dim,
+                                         int block_size, int cache_dtype, int device);
+
+/*
+ * paged_attn_decode_ex - the general form: k_scale / v_scale are NULL for a
+ * 16-bit cache and required for fp8; `workspace` is a caller-owned device
+ * buffer of at least paged_attn_decode_workspace_bytes() bytes (16-byte
+ * aligned), else PKV_ERR_WORKSPACE. The workspace must not be used by
+ * another call until this one has finished on the GPU.
+ */
+int paged_attn_decode_ex(const pkv_tensor* q, const pkv_tensor* k_cache,
+                         const pkv_tensor* v_cache, const pkv_tensor* k_scale,
+                         const pkv_tensor* v_scale, const pkv_tensor* block_tables,
+                         const pkv_tensor* context_lens, int num_kv_heads, float scale,
+                         int block_size, pkv_tensor* out, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Cache writes and block copies                                            */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * reshape_and_cache - store each new token's K and V rows in its slot.
+ * During generation a token is written into its sequence's current block
+ * ("How Block Paging Operates During Generation", "PagedAttention and KV
+ * Cache Management"). Slot = physical_block * B + offset:
+ *     k_cache[slot / B, h, slot % B, :] = k[t, h, :]   (same for v)
+ * for every t with slot_mapping[t] >= 0 (negative = padding, skipped).
+ *
+ *   k, v          [T, Hk, D] same dtype as the caches (f16 | bf16)
+ *   k_cache, v_cache [NB, Hk, B, D], written
+ *   slot_mapping  [T] int64; slots must be distinct and < NB * B
+ * Bit-exact copy. A slot >= NB * B is skipped and flagged as a device check.
+ */
+int reshape_and_cache(const pkv_tensor* k, const pkv_tensor* v, pkv_tensor* k_cache,
+                      pkv_tensor* v_cache, const pkv_tensor* slot_mapping, void* stream);
+
+/*
+ * reshape_and_cache_fp8 - as reshape_and_cache into an fp8-e4m3 pool: stores
+ * the e4m3 code of the fp32 quotient x / scale[h], rounded to nearest even
+ * and saturated to +-448 (NaN stays NaN).
+ *
+ *   k, v          [T, Hk, D] f16 | bf16
+ *   k_cache, v_cache [NB, Hk, B, D] PKV_FP8_E4M3
+ *   k_scale, v_scale [Hk] f32 device
+ */
+int reshape_and_cache_fp8(const pkv_tensor* k, const pkv_tensor* v, pkv_tensor* k_cache,
+                          pkv_tensor* v_cache, const pkv_tensor* slot_mapping,
+                          const pkv_tensor* k_scale, const pkv_tensor* v_scale, void* stream);
+
+/*
+ * copy_blocks - device half of copy-on-write ("Parallel Sampling & Beam Search
+ * via Copy-on-Write", "PagedAttention and KV Cache Management"): for each
+ * (src, dst) row of `pairs`, block dst of both caches becomes a bit-exact copy
+ * of block src (all heads, all B slots).
+ *
+ *   k_cache, v_cache [NB, Hk, B, D] any element type (same for both)
+ *   pairs         [n, 2] int32 device; every dst distinct and no dst also a
+ *                 src in the same call (the allocator's copy-on-write pairs
+ *                 satisfy this); ids outside the pool are skipped and flagged.
+ */
+int copy_blocks(pkv_tensor* k_cache, pkv_tensor* v_cache, const pkv_tensor* pairs,
+                void* stream);
+
+/*
+ * pkv_device_error - synchronises `device` and returns PKV_ERR_DEVICE_CHECK
+ * if any kernel of this library flagged a device-side check since the last
+ * call (then clears the flag), else PKV_OK. Returns PKV_ERR_CUDA if the
+ * synchronisation itself fails.
+ */
+int pkv_device_error(int device);
+
+/* ------------------------------------------------------------------------ */
+/* Host block allocator                                                     */
+/* ------------------------------------------------------------------------ */
+/*
+ * Semantics of "Hands-On Implementation: Building a PagedAttention Block
+ * Allocator in Python" ("PagedAttention and KV Cache Management"): a pool of
+ * num_blocks blocks of block_size slots; new blocks come from the HEAD of the
+ * free list and released blocks go to its TAIL; a sequence of n tokens holds
+ * ceil(n / B) blocks; forking shares every block (reference count + 1);
+ * freeing drops one reference per block; a block is copied on write when a
+ * sequence must write into a block another sequence still references. Each
+ * call either succeeds or returns an error and changes nothing.
+ *
+ * Sequence ids are caller-chosen int64 values.
+ */
+
+/* Create a pool. initial_free_order: NULL for 0..num_blocks-1, else a
+ * permutation of the block ids giving the initial free-list order (host). */
+int pkv_alloc_create(int32_t num_blocks, int32_t block_size, const int32_t* initial_free_order,
+                     void** handle);
+void pkv_alloc_destroy(void* handle);
+
+/* New sequence holding num_tokens tokens in ceil(num_tokens / B) fresh
+ * blocks. PKV_ERR_EXISTS, PKV_ERR_OOM. */
+int pkv_seq_allocate(void* handle, int64_t seq, int32_t num_tokens);
+
+/* Reserve the slot of the sequence's next token. *slot gets the flat slot
+ * (block * B + offset). If the token must go into a block shared with
+ * another sequence, a fresh block replaces it in this sequence's table and
+ * *cow_src / *cow_dst name the block copy the device must do first (see
+ * copy_blocks); otherwise both are -1. A full last block (shared or not)
+ * gets a new block after it. PKV_ERR_UNKNOWN_SEQ, PKV_ERR_OOM. */
+int pkv_seq_append_slot(void* handle, int64_t seq, int64_t* slot, int32_t* cow_src,
+                        int32_t* cow_dst);
+
+/* dst shares every block of src (zero-copy fork). PKV_ERR_UNKNOWN_SEQ,
+ * PKV_ERR_EXISTS. */
+int pkv_seq_fork(void* handle, int64_t src, int64_t dst);
+
+/* Drop the sequence and one reference on each of its blocks, in table order;
+ * a block reaching 0 returns to the tail of the free list. Unknown seq:
+ * PKV_OK, nothing done. */
+int pkv_seq_free(void* handle, int64_t seq);
+
+/* Tokens held by seq (>= 0), or PKV_ERR_UNKNOWN_SEQ. */
+int64_t pkv_seq_num_tokens(void* handle, int64_t seq);
+
+/* Copy seq's block table into table[0 .. cap) (host); returns the number of
+ * blocks (which may exceed cap: only cap entries are written), or an error. */
+int pkv_seq_block_table(void* handle, int64_t seq, int32_t* table, int32_t cap);
+
+/* Build the decode inputs for n sequences, on the host: row i of `table`
+ * (n x max_blocks, row-major) gets seqs[i]'s block ids padded with -1, and
+ * lens[i] its token count. PKV_ERR_UNKNOWN_SEQ; PKV_ERR_INVALID_ARG if a
+ * table does not fit in max_blocks. */
+int pkv_build_block_tables(void* handle, const int64_t* seqs, int32_t n, int32_t* table,
+                           int32_t max_blocks, int32_t* lens);
+
+/* Pool statistics: free blocks, used blocks (refcount > 0), shared blocks
+ * (refcount > 1), tokens stored (each physical slot counted once). Any
+ * output pointer may be NULL. */
+int pkv_alloc_stats(void* handle, int32_t* free_blocks, int32_t* used_blocks,
+                    int32_t* shared_blocks, int64_t* tokens);
+
+/* Reference count of one block (>= 0) or PKV_ERR_INVALID_ARG. */
+int pkv_block_refcount(void* handle, int32_t block);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDKV_H_ */

@@ -1,0 +1,570 @@
+// C ABI of libpagedkv.so (declared in include/pagedkv.h): argument checks,
+// TMA tensor-map encoding, workspace management and kernel dispatch for the
+// decode, cache-write and block-copy kernels. The host allocator lives in
+// allocator.cpp.
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/pagedkv.h"
+#include "cache_ops.cuh"
+#include "decode.cuh"
+
+namespace pkv {
+
+// Per-device error word the kernels OR their device-check bits into.
+__device__ int g_pkv_err;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  bool init = false;
+  int sms = 0;
+  int* err = nullptr;  // device address of g_pkv_err
+  void* ws = nullptr;  // library-owned decode workspace
+  size_t ws_bytes = 0;
+};
+DeviceState g_dev[kMaxDevices];
+std::mutex g_mu;
+
+int current_device(int* dev) {
+  if (cudaGetDevice(dev) != cudaSuccess) return PKV_ERR_CUDA;
+  if (*dev < 0 || *dev >= kMaxDevices) return PKV_ERR_UNSUPPORTED;
+  return PKV_OK;
+}
+
+// Device properties and the error word's address, once per device (with
+// that device current).
+int device_state(int dev, DeviceState** out) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState& d = g_dev[dev];
+  if (!d.init) {
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return PKV_ERR_CUDA;
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_pkv_err) != cudaSuccess) return PKV_ERR_CUDA;
+    d.err = static_cast<int*>(p);
+    d.init = true;
+  }
+  *out = &d;
+  return PKV_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+int elem_bytes(int dt) {
+  switch (dt) {
+    case PKV_F16:
+    case PKV_BF16: return 2;
+    case PKV_FP8_E4M3: return 1;
+    case PKV_I32:
+    case PKV_F32: return 4;
+    case PKV_I64: return 8;
+    default: return 0;
+  }
+}
+
+bool well_formed(const pkv_tensor* t, int ndim, int dtype) {
+  if (!t || t->ndim != ndim || t->dtype != dtype) return false;
+  for (int i = 0; i < ndim; ++i)
+    if (t->shape[i] < 0) return false;
+  if (ndim > 0 && t->shape[ndim - 1] > 1 && t->stride[ndim - 1] != 1) return false;
+  for (int i = 0; i < ndim; ++i)
+    if (t->stride[i] < 0) return false;
+  bool empty = false;
+  for (int i = 0; i < ndim; ++i) empty |= t->shape[i] == 0;
+  return empty || t->data != nullptr;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Pool [NB, Hk, B, D]: innermost contiguous, strides non-decreasing outward,
+// byte strides multiples of 16, base 16-byte aligned.
+bool pool_ok(const pkv_tensor* t, int dtype) {
+  if (!well_formed(t, 4, dtype)) return false;
+  const int64_t eb = elem_bytes(dtype);
+  const int64_t* sh = t->shape;
+  const int64_t* st = t->stride;
+  if (st[3] != 1) return false;
+  if (st[2] < sh[3] || st[1] < sh[2] * st[2] || st[0] < sh[1] * st[1]) return false;
+  for (int i = 0; i < 3; ++i)
+    if ((st[i] * eb) % 16 != 0) return false;
+  return aligned(t->data, 16);
+}
+
+bool same_shape(const pkv_tensor* a, const pkv_tensor* b) {
+  if (a->ndim != b->ndim) return false;
+  for (int i = 0; i < a->ndim; ++i)
+    if (a->shape[i] != b->shape[i]) return false;
+  return true;
+}
+
+int encode_pool_map(CUtensorMap* map, const pkv_tensor* pool, int dtype) {
+  auto fn = encode_fn();
+  if (!fn) return PKV_ERR_CUDA;
+  const int eb = elem_bytes(dtype);
+  const int D = static_cast<int>(pool->shape[3]);
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(pool->shape[2]),
+                        static_cast<cuuint64_t>(pool->shape[1]),
+                        static_cast<cuuint64_t>(pool->shape[0])};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(pool->stride[2] * eb),
+                           static_cast<cuuint64_t>(pool->stride[1] * eb),
+                           static_cast<cuuint64_t>(pool->stride[0] * eb)};
+  const int epr = 128 / eb;
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(D < epr ? D : epr),
+                       static_cast<cuuint32_t>(pool->shape[2]), 1, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  CUtensorMapDataType ty = dtype == PKV_F16    ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                           : dtype == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                               : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  CUresult r = fn(map, ty, 4, pool->data, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? PKV_OK : PKV_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// Decode kernel registry
+// ---------------------------------------------------------------------------
+
+struct DecodeLaunch {
+  void (*kernel)(DecodeParams);
+  void (*merge)(DecodeParams);
+  int threads;
+  int smem;
+  int nc;
+  int occ[kMaxDevices];  // resident CTAs per SM, 0 = not queried yet
+};
+
+template <int CK, bool QBF, int D, int BS, int NC, int NS>
+DecodeLaunch* decode_entry() {
+  static DecodeLaunch e = {&decode_kernel<CK, QBF, D, BS, NC, NS>,
+                           &decode_merge_kernel<QBF, D>,
+                           NC * 32,
+                           DecodeCfg<CK, QBF, D, BS, NC, NS>::SMEM,
+                           NC,
+                           {0}};
+  return &e;
+}
+
+// Stage counts: about 96 KB of ring per 4-warp CTA (two CTAs per SM) where
+// a stage is 8 KB or less; 32-token 16-bit blocks use three 16 KB stages
+// per warp (one CTA per SM).
+DecodeLaunch* pick_decode(int ck, bool qbf, int D, int BS) {
+  constexpr int NC = 4;
+  if (ck == kCacheBF16) {
+    if (D == 128 && BS == 16) return decode_entry<kCacheBF16, true, 128, 16, NC, 3>();
+    if (D == 128 && BS == 32) return decode_entry<kCacheBF16, true, 128, 32, NC, 3>();
+    if (D == 64 && BS == 16) return decode_entry<kCacheBF16, true, 64, 16, NC, 6>();
+    if (D == 64 && BS == 32) return decode_entry<kCacheBF16, true, 64, 32, NC, 3>();
+  } else if (ck == kCacheF16) {
+    if (D == 128 && BS == 16) return decode_entry<kCacheF16, false, 128, 16, NC, 3>();
+    if (D == 128 && BS == 32) return decode_entry<kCacheF16, false, 128, 32, NC, 3>();
+    if (D == 64 && BS == 16) return decode_entry<kCacheF16, false, 64, 16, NC, 6>();
+    if (D == 64 && BS == 32) return decode_entry<kCacheF16, false, 64, 32, NC, 3>();
+  } else if (ck == kCacheE4M3 && D == 128) {
+    if (qbf) {
+      if (BS == 16) return decode_entry<kCacheE4M3, true, 128, 16, NC, 6>();
+      if (BS == 32) return decode_entry<kCacheE4M3, true, 128, 32, NC, 3>();
+    } else {
+      if (BS == 16) return decode_entry<kCacheE4M3, false, 128, 16, NC, 6>();
+      if (BS == 32) return decode_entry<kCacheE4M3, false, 128, 32, NC, 3>();
+    }
+  }
+  return nullptr;
+}
+
+int decode_grid(DecodeLaunch* e, int dev, int sms, int* grid) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (e->occ[dev] == 0) {
+    if (cudaFuncSetAttribute(e->kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, e->smem) !=
+        cudaSuccess)
+      return PKV_ERR_CUDA;
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, e->kernel, e->threads, e->smem) !=
+            cudaSuccess ||
+        occ < 1)
+      return PKV_ERR_CUDA;
+    e->occ[dev] = occ;
+  }
+  *grid = e->occ[dev] * sms;
+  return PKV_OK;
+}
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct WsLayout {
+  size_t hdr, desc, part_o, part_ml, total;
+};
+
+WsLayout ws_layout(int nwt, int g, int D) {
+  WsLayout l;
+  l.hdr = 0;
+  l.desc = 256;
+  l.part_o = round_up(l.desc + static_cast<size_t>(nwt) * 16, 256);
+  l.part_ml = round_up(l.part_o + static_cast<size_t>(nwt) * 2 * g * D * 4, 256);
+  l.total = round_up(l.part_ml + static_cast<size_t>(nwt) * 2 * g * 2 * 4, 256);
+  return l;
+}
+
+struct DecodeArgs {
+  const pkv_tensor *q, *kc, *vc, *ks, *vs, *bt, *cl;
+  int Hk;
+  float scale;
+  int BS;
+  pkv_tensor* out;
+};
+
+// Checks shapes/types and resolves the kernel. On PKV_OK, *entry is set, or
+// left NULL when there is nothing to compute (S == 0).
+int check_decode(const DecodeArgs& a, bool fp8, int* ck_out, DecodeLaunch** entry) {
+  *entry = nullptr;
+  if (!a.q || !a.kc || !a.vc || !a.bt || !a.cl || !a.out) return PKV_ERR_INVALID_ARG;
+  const int qdt = a.q->dtype;
+  if (qdt != PKV_F16 && qdt != PKV_BF16) return PKV_ERR_INVALID_ARG;
+  if (!well_formed(a.q, 3, qdt) || !well_formed(a.out, 3, qdt) || !same_shape(a.q, a.out))
+    return PKV_ERR_INVALID_ARG;
+  const int cdt = fp8 ? PKV_FP8_E4M3 : qdt;
+  if (!pool_ok(a.kc, cdt) || !pool_ok(a.vc, cdt) || !same_shape(a.kc, a.vc))
+    return PKV_ERR_INVALID_ARG;
+  const int64_t S = a.q->shape[0], Hq = a.q->shape[1], D = a.q->shape[2];
+  const int64_t NB = a.kc->shape[0], Hk = a.kc->shape[1], BS = a.kc->shape[2];
+  if (a.kc->shape[3] != D || Hk != a.Hk || BS != a.BS || Hk <= 0 || Hq % Hk != 0)
+    return PKV_ERR_INVALID_ARG;
+  if (!well_formed(a.bt, 2, PKV_I32) || a.bt->shape[0] != S) return PKV_ERR_INVALID_ARG;
+  if (!well_formed(a.cl, 1, PKV_I32) || a.cl->shape[0] != S) return PKV_ERR_INVALID_ARG;
+  if (S > 0 && a.cl->stride[0] != 1) return PKV_ERR_INVALID_ARG;
+  if (!std::isfinite(a.scale)) return PKV_ERR_INVALID_ARG;
+  if (fp8) {
+    if (!a.ks || !a.vs || !well_formed(a.ks, 1, PKV_F32) || !well_formed(a.vs, 1, PKV_F32) ||
+        a.ks->shape[0] != Hk || a.vs->shape[0] != Hk || a.ks->stride[0] != 1 ||
+        a.vs->stride[0] != 1)
+      return PKV_ERR_INVALID_ARG;
+  }
+  // q rows are read as 4- (16-bit cache) or 8-byte (fp8 cache) words
+  const int qa = fp8 ? 4 : 2;
+  if (S > 0 && (a.q->stride[0] % qa || a.q->stride[1] % qa || !aligned(a.q->data, 2 * qa)))
+    return PKV_ERR_INVALID_ARG;
+  const int64_t g = Hq / Hk;
+  if (g > 8 || (D != 64 && D != 128) || (BS != 16 && BS != 32) || (fp8 && D != 128))
+    return PKV_ERR_UNSUPPORTED;
+  if (NB > INT32_MAX || S > INT32_MAX || a.bt->shape[1] > INT32_MAX / 32)
+    return PKV_ERR_UNSUPPORTED;
+  if (S == 0) return PKV_OK;
+  if (a.bt->shape[1] < 1 || NB < 1) return PKV_ERR_INVALID_ARG;
+  const int ck = fp8 ? kCacheE4M3 : (qdt == PKV_BF16 ? kCacheBF16 : kCacheF16);
+  *ck_out = ck;
+  *entry = pick_decode(ck, qdt == PKV_BF16, static_cast<int>(D), static_cast<int>(BS));
+  return *entry ? PKV_OK : PKV_ERR_UNSUPPORTED;
+}
+
+int launch_decode(const DecodeArgs& a, bool fp8, void* ws, size_t ws_bytes, bool lib_ws,
+                  cudaStream_t stream) {
+  int ck = 0;
+  DecodeLaunch* e = nullptr;
+  int st = check_decode(a, fp8, &ck, &e);
+  if (st != PKV_OK || !e) return st;
+  int dev;
+  if ((st = current_device(&dev)) != PKV_OK) return st;
+  DeviceState* ds;
+  if ((st = device_state(dev, &ds)) != PKV_OK) return st;
+  int grid;
+  if ((st = decode_grid(e, dev, ds->sms, &grid)) != PKV_OK) return st;
+  const int nwt = grid * e->nc;
+  const int g = static_cast<int>(a.q->shape[1] / a.Hk);
+  const int D = static_cast<int>(a.q->shape[2]);
+  const WsLayout L = ws_layout(nwt, g, D);
+  if (lib_ws) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (ds->ws_bytes < L.total) {
+      if (ds->ws) cudaFree(ds->ws);
+      ds->ws = nullptr;
+      ds->ws_bytes = 0;
+      if (cudaMalloc(&ds->ws, L.total) != cudaSuccess) return PKV_ERR_CUDA;
+      ds->ws_bytes = L.total;
+    }
+    ws = ds->ws;
+    ws_bytes = ds->ws_bytes;
+  }
+  if (!ws || ws_bytes < L.total || !aligned(ws, 16)) return PKV_ERR_WORKSPACE;
+
+  DecodeParams p;
+  std::memset(&p, 0, sizeof(p));
+  const int cdt = fp8 ? PKV_FP8_E4M3 : a.q->dtype;
+  if ((st = encode_pool_map(&p.tmk, a.kc, cdt)) != PKV_OK) return st;
+  if ((st = encode_pool_map(&p.tmv, a.vc, cdt)) != PKV_OK) return st;
+  p.q = a.q->data;
+  p.q_s = a.q->stride[0];
+  p.q_h = a.q->stride[1];
+  p.out = a.out->data;
+  p.o_s = a.out->stride[0];
+  p.o_h = a.out->stride[1];
+  p.tables = static_cast<const int*>(a.bt->data);
+  p.t_s = a.bt->stride[0];
+  p.lens = static_cast<const int*>(a.cl->data);
+  p.k_scale = fp8 ? static_cast<const float*>(a.ks->data) : nullptr;
+  p.v_scale = fp8 ? static_cast<const float*>(a.vs->data) : nullptr;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+  p.S = static_cast<int>(a.q->shape[0]);
+  p.Hk = a.Hk;
+  p.g = g;
+  p.MB = static_cast<int>(a.bt->shape[1]);
+  p.NB = static_cast<int>(a.kc->shape[0]);
+  p.nwt = nwt;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  p.hdr = reinterpret_cast<long long*>(w + L.hdr);
+  p.err = ds->err;
+  p.part_o = reinterpret_cast<float*>(w + L.part_o);
+  p.part_ml = reinterpret_cast<float*>(w + L.part_ml);
+  p.desc = reinterpret_cast<int4*>(w + L.desc);
+
+  e->kernel<<<grid, e->threads, e->smem, stream>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return PKV_ERR_CUDA;
+  e->merge<<<nwt, 128, 0, stream>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return PKV_ERR_CUDA;
+  return PKV_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Cache writes and block copies
+// ---------------------------------------------------------------------------
+
+int launch_reshape(const pkv_tensor* k, const pkv_tensor* v, pkv_tensor* kc, pkv_tensor* vc,
+                   const pkv_tensor* slots, const pkv_tensor* ks, const pkv_tensor* vs, bool fp8,
+                   cudaStream_t stream) {
+  if (!k || !v || !kc || !vc || !slots) return PKV_ERR_INVALID_ARG;
+  const int xdt = k->dtype;
+  if (xdt != PKV_F16 && xdt != PKV_BF16) return PKV_ERR_INVALID_ARG;
+  const int cdt = fp8 ? PKV_FP8_E4M3 : xdt;
+  if (!well_formed(k, 3, xdt) || !well_formed(v, 3, xdt) || !same_shape(k, v))
+    return PKV_ERR_INVALID_ARG;
+  if (!pool_ok(kc, cdt) || !pool_ok(vc, cdt) || !same_shape(kc, vc)) return PKV_ERR_INVALID_ARG;
+  if (kc->stride[0] != vc->stride[0] || kc->stride[1] != vc->stride[1] ||
+      kc->stride[2] != vc->stride[2])
+    return PKV_ERR_INVALID_ARG;
+  const int64_t T = k->shape[0], Hk = k->shape[1], D = k->shape[2];
+  if (kc->shape[1] != Hk || kc->shape[3] != D) return PKV_ERR_INVALID_ARG;
+  if (!well_formed(slots, 1, PKV_I64) || slots->shape[0] != T) return PKV_ERR_INVALID_ARG;
+  if (T > 0 && slots->stride[0] != 1) return PKV_ERR_INVALID_ARG;
+  if (fp8 && (!ks || !vs || !well_formed(ks, 1, PKV_F32) || !well_formed(vs, 1, PKV_F32) ||
+              ks->shape[0] != Hk || vs->shape[0] != Hk || ks->stride[0] != 1 ||
+              vs->stride[0] != 1))
+    return PKV_ERR_INVALID_ARG;
+  const int eb = elem_bytes(cdt);
+  if ((D * eb) % 16 != 0) return PKV_ERR_UNSUPPORTED;
+  // 16-byte vector reads of the inputs
+  if (T > 0 && ((k->stride[0] * 2) % 16 || (k->stride[1] * 2) % 16 || (v->stride[0] * 2) % 16 ||
+                (v->stride[1] * 2) % 16 || !aligned(k->data, 16) || !aligned(v->data, 16)))
+    return PKV_ERR_INVALID_ARG;
+  if (T == 0 || Hk == 0) return PKV_OK;
+  if (kc->shape[0] > INT32_MAX) return PKV_ERR_UNSUPPORTED;
+  int dev, st;
+  if ((st = current_device(&dev)) != PKV_OK) return st;
+  DeviceState* ds;
+  if ((st = device_state(dev, &ds)) != PKV_OK) return st;
+  CacheParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.k = static_cast<const uint8_t*>(k->data);
+  p.v = static_cast<const uint8_t*>(v->data);
+  p.x_s0 = k->stride[0] * 2;
+  p.x_s1 = k->stride[1] * 2;
+  p.v_s0 = v->stride[0] * 2;
+  p.v_s1 = v->stride[1] * 2;
+  p.kc = static_cast<uint8_t*>(kc->data);
+  p.vc = static_cast<uint8_t*>(vc->data);
+  p.c_s0 = kc->stride[0] * eb;
+  p.c_s1 = kc->stride[1] * eb;
+  p.c_s2 = kc->stride[2] * eb;
+  p.slots = static_cast<const long long*>(slots->data);
+  p.k_scale = fp8 ? static_cast<const float*>(ks->data) : nullptr;
+  p.v_scale = fp8 ? static_cast<const float*>(vs->data) : nullptr;
+  p.T = static_cast<int>(T);
+  p.Hk = static_cast<int>(Hk);
+  p.B = static_cast<int>(kc->shape[2]);
+  p.NB = static_cast<int>(kc->shape[0]);
+  p.row_vecs = static_cast<int>(D * eb / 16);
+  p.in_bytes = static_cast<int>(D * 2);
+  const long long threads = T * Hk * p.row_vecs;
+  const int tpb = 128;
+  const long long blocks = (threads + tpb - 1) / tpb;
+  if (blocks > INT32_MAX) return PKV_ERR_UNSUPPORTED;
+  if (!fp8) reshape_and_cache_kernel<<<static_cast<int>(blocks), tpb, 0, stream>>>(p, ds->err);
+  else if (xdt == PKV_BF16)
+    reshape_and_cache_fp8_kernel<true><<<static_cast<int>(blocks), tpb, 0, stream>>>(p, ds->err);
+  else
+    reshape_and_cache_fp8_kernel<false><<<static_cast<int>(blocks), tpb, 0, stream>>>(p, ds->err);
+  return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace pkv
+
+using namespace pkv;
+
+extern "C" {
+
+const char* pkv_status_string(int s) {
+  switch (s) {
+    case PKV_OK: return "ok";
+    case PKV_ERR_INVALID_ARG: return "invalid argument";
+    case PKV_ERR_UNSUPPORTED: return "unsupported shape or type";
+    case PKV_ERR_OOM: return "out of free blocks";
+    case PKV_ERR_UNKNOWN_SEQ: return "unknown sequence";
+    case PKV_ERR_EXISTS: return "sequence exists";
+    case PKV_ERR_DOUBLE_FREE: return "double free";
+    case PKV_ERR_CUDA: return "CUDA error";
+    case PKV_ERR_DEVICE_CHECK: return "device-side check failed";
+    case PKV_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+int pkv_version(void) { return 100; }
+
+int paged_attn_decode(const pkv_tensor* q, const pkv_tensor* k_cache, const pkv_tensor* v_cache,
+                      const pkv_tensor* block_tables, const pkv_tensor* context_lens,
+                      int num_kv_heads, float scale, int block_size, pkv_tensor* out,
+                      void* stream) {
+  DecodeArgs a{q, k_cache, v_cache, nullptr, nullptr, block_tables, context_lens,
+               num_kv_heads, scale, block_size, out};
+  return launch_decode(a, false, nullptr, 0, true, static_cast<cudaStream_t>(stream));
+}
+
+int paged_attn_decode_fp8(const pkv_tensor* q, const pkv_tensor* k_cache,
+                          const pkv_tensor* v_cache, const pkv_tensor* k_scale,
+                          const pkv_tensor* v_scale, const pkv_tensor* block_tables,
+                          const pkv_tensor* context_lens, int num_kv_heads, float scale,
+                          int block_size, pkv_tensor* out, void* stream) {
+  DecodeArgs a{q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
+               num_kv_heads, scale, block_size, out};
+  return launch_decode(a, true, nullptr, 0, true, static_cast<cudaStream_t>(stream));
+}
+
+size_t paged_attn_decode_workspace_bytes(int num_q_heads, int num_kv_heads, int head_dim,
+                                         int block_size, int cache_dtype, int device) {
+  if (num_kv_heads <= 0 || num_q_heads % num_kv_heads || device < 0 || device >= kMaxDevices)
+    return 0;
+  const bool fp8 = cache_dtype == PKV_FP8_E4M3;
+  const int ck = fp8 ? kCacheE4M3 : (cache_dtype == PKV_BF16 ? kCacheBF16 : kCacheF16);
+  DecodeLaunch* e = pick_decode(ck, cache_dtype == PKV_BF16 || fp8, head_dim, block_size);
+  if (!e) return 0;
+  int prev;
+  if (cudaGetDevice(&prev) != cudaSuccess) return 0;
+  if (prev != device && cudaSetDevice(device) != cudaSuccess) return 0;
+  DeviceState* ds;
+  int grid = 0;
+  size_t bytes = 0;
+  if (device_state(device, &ds) == PKV_OK && decode_grid(e, device, ds->sms, &grid) == PKV_OK)
+    bytes = ws_layout(grid * e->nc, num_q_heads / num_kv_heads, head_dim).total;
+  if (prev != device) cudaSetDevice(prev);
+  return bytes;
+}
+
+int paged_attn_decode_ex(const pkv_tensor* q, const pkv_tensor* k_cache,
+                         const pkv_tensor* v_cache, const pkv_tensor* k_scale,
+                         const pkv_tensor* v_scale, const pkv_tensor* block_tables,
+                         const pkv_tensor* context_lens, int num_kv_heads, float scale,
+                         int block_size, pkv_tensor* out, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  const bool fp8 = k_cache && k_cache->dtype == PKV_FP8_E4M3;
+  DecodeArgs a{q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
+               num_kv_heads, scale, block_size, out};
+  return launch_decode(a, fp8, workspace, workspace_bytes, false,
+                       static_cast<cudaStream_t>(stream));
+}
+
+int reshape_and_cache(const pkv_tensor* k, const pkv_tensor* v, pkv_tensor* k_cache,
+                      pkv_tensor* v_cache, const pkv_tensor* slot_mapping, void* stream) {
+  return launch_reshape(k, v, k_cache, v_cache, slot_mapping, nullptr, nullptr, false,
+                        static_cast<cudaStream_t>(stream));
+}
+
+int reshape_and_cache_fp8(const pkv_tensor* k, const pkv_tensor* v, pkv_tensor* k_cache,
+                          pkv_tensor* v_cache, const pkv_tensor* slot_mapping,
+                          const pkv_tensor* k_scale, const pkv_tensor* v_scale, void* stream) {
+  return launch_reshape(k, v, k_cache, v_cache, slot_mapping, k_scale, v_scale, true,
+                        static_cast<cudaStream_t>(stream));
+}
+
+int copy_blocks(pkv_tensor* k_cache, pkv_tensor* v_cache, const pkv_tensor* pairs,
+                void* stream) {
+  if (!k_cache || !v_cache || !pairs) return PKV_ERR_INVALID_ARG;
+  const int dt = k_cache->dtype;
+  const int eb = elem_bytes(dt);
+  if (eb == 0 || eb > 2 || !pool_ok(k_cache, dt) || !pool_ok(v_cache, dt) ||
+      !same_shape(k_cache, v_cache))
+    return PKV_ERR_INVALID_ARG;
+  for (int i = 0; i < 3; ++i)
+    if (k_cache->stride[i] != v_cache->stride[i]) return PKV_ERR_INVALID_ARG;
+  if (!well_formed(pairs, 2, PKV_I32) || pairs->shape[1] != 2) return PKV_ERR_INVALID_ARG;
+  const int64_t n = pairs->shape[0];
+  if (n == 0) return PKV_OK;
+  if ((k_cache->shape[3] * eb) % 16 != 0) return PKV_ERR_UNSUPPORTED;
+  if (n > INT32_MAX || k_cache->shape[0] > INT32_MAX) return PKV_ERR_UNSUPPORTED;
+  int dev, st;
+  if ((st = current_device(&dev)) != PKV_OK) return st;
+  DeviceState* ds;
+  if ((st = device_state(dev, &ds)) != PKV_OK) return st;
+  CopyParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.kc = static_cast<uint8_t*>(k_cache->data);
+  p.vc = static_cast<uint8_t*>(v_cache->data);
+  p.c_s0 = k_cache->stride[0] * eb;
+  p.c_s1 = k_cache->stride[1] * eb;
+  p.c_s2 = k_cache->stride[2] * eb;
+  p.pairs = static_cast<const int*>(pairs->data);
+  p.pr_s = pairs->stride[0];
+  p.n = static_cast<int>(n);
+  p.Hk = static_cast<int>(k_cache->shape[1]);
+  p.B = static_cast<int>(k_cache->shape[2]);
+  p.NB = static_cast<int>(k_cache->shape[0]);
+  p.row_vecs = static_cast<int>(k_cache->shape[3] * eb / 16);
+  const int total = p.Hk * p.B * p.row_vecs;
+  const int tpb = 256;
+  int chunks = (total + tpb - 1) / tpb;
+  if (chunks > 65535) chunks = 65535;
+  dim3 grid(static_cast<unsigned>(n), static_cast<unsigned>(chunks));
+  copy_blocks_kernel<<<grid, tpb, 0, static_cast<cudaStream_t>(stream)>>>(p, ds->err);
+  return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+int pkv_device_error(int device) {
+  if (device < 0 || device >= kMaxDevices) return PKV_ERR_INVALID_ARG;
+  int prev;
+  if (cudaGetDevice(&prev) != cudaSuccess) return PKV_ERR_CUDA;
+  if (prev != device && cudaSetDevice(device) != cudaSuccess) return PKV_ERR_CUDA;
+  int st = PKV_OK;
+  int v = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess ||
+      cudaMemcpyFromSymbol(&v, g_pkv_err, sizeof(int)) != cudaSuccess) {
+    st = PKV_ERR_CUDA;
+  } else if (v != 0) {
+    const int zero = 0;
+    st = cudaMemcpyToSymbol(g_pkv_err, &zero, sizeof(int)) == cudaSuccess ? PKV_ERR_DEVICE_CHECK
+                                                                           : PKV_ERR_CUDA;
+  }
+  if (prev != device) cudaSetDevice(prev);
+  return st;
+}
+
+}  // extern "C"

@@ -1,0 +1,115 @@
+"""The C++ block allocator (through the C ABI) against the pages' demo run and
+against the oracle allocator on random operation sequences (bit-exact)."""
+import random
+
+import pytest
+
+import paged_kv_cache_453_b200 as P
+import workloads as W
+from oracle.allocator import BlockAllocator as OracleAlloc, AllocError
+from test_oracle_allocator import run_demo
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from paged_kv_cache_453_b200.build import build
+    build()
+
+
+def test_demo_run_matches_pages():
+    run_demo(lambda n, B: P.BlockAllocator(n, B), lambda a, s: a.table(s), lambda a: a.num_free(),
+             lambda a, s, n: a.allocate(s, n), lambda a, s, d: a.fork(s, d),
+             lambda a, s: a.append_slot(s), lambda a, s: a.free(s))
+
+
+def _same(a: P.BlockAllocator, o: OracleAlloc, seqs):
+    for s in seqs:
+        assert a.table(s) == o.table(s)
+        assert a.num_tokens(s) == o.num_tokens[s]
+    assert [a.refcount(b) for b in range(o.num_blocks)] == o.refcount
+    st = a.stats()
+    ost = o.stats()
+    assert (st["free"], st["used"], st["shared"], st["tokens"]) == (
+        ost["free"], ost["used"], ost["shared"], ost["tokens"])
+
+
+@pytest.mark.parametrize("seed", [1, 2, 3])
+def test_random_ops_match_oracle(seed):
+    rng = random.Random(seed)
+    N, B = 48, rng.choice([2, 4, 16])
+    order = rng.sample(range(N), N)
+    a = P.BlockAllocator(N, B, order)
+    o = OracleAlloc(N, B, order)
+    live, nxt = [], 0
+    for step in range(2000):
+        op = rng.random()
+        if op < 0.2 or not live:
+            args, name = (nxt, rng.randint(0, 3 * B)), "allocate"
+        elif op < 0.3:
+            args, name = (rng.choice(live), nxt), "fork"
+        elif op < 0.42:
+            args, name = (rng.choice(live),), "free"
+        elif op < 0.45:
+            args, name = (10_000 + rng.randint(0, 5),), "append_slot"   # unknown sequence
+        else:
+            args, name = (rng.choice(live),), "append_slot"
+        err_o = err_a = None
+        try:
+            ro = getattr(o, name)(*args)
+        except AllocError as e:
+            err_o = e.code
+        try:
+            ra = getattr(a, name)(*args)
+        except P.PkvError as e:
+            err_a = e.status
+        assert err_o == err_a, (step, name, args, err_o, err_a)
+        if err_o is None:
+            if name == "append_slot":
+                assert ra == ro
+            if name in ("allocate", "fork"):
+                live.append(nxt)
+                nxt += 1
+            if name == "free":
+                live.remove(args[0])
+        _same(a, o, live)
+
+
+def test_build_block_tables_pads_and_checks():
+    a = P.BlockAllocator(16, 4)
+    a.allocate(7, 9)
+    a.allocate(8, 0)
+    table, lens = a.build_block_tables([8, 7], 4)
+    assert table.tolist() == [[-1, -1, -1, -1], [0, 1, 2, -1]]
+    assert lens.tolist() == [0, 9]
+    with pytest.raises(P.PkvError) as e:
+        a.build_block_tables([7], 2)           # 3 blocks do not fit in 2
+    assert e.value.status == P.PKV_ERR_INVALID_ARG
+    with pytest.raises(P.PkvError) as e:
+        a.build_block_tables([9], 4)
+    assert e.value.status == P.PKV_ERR_UNKNOWN_SEQ
+
+
+def test_prefix_script_same_as_oracle():
+    s = W.spec("prefix_13b")
+    sc = W.prefix_script(s)
+    a = P.BlockAllocator(sc.num_blocks, s.block_size, sc.free_order)
+    o = OracleAlloc(sc.num_blocks, s.block_size, sc.free_order)
+    a.run(sc.setup)
+    o.run(sc.setup)
+    steps_a = [a.append_slot(r) for r in sc.step_appends]
+    steps_o = [o.append_slot(r) for r in sc.step_appends]
+    assert steps_a == steps_o
+    _same(a, o, sc.seqs)
+
+
+def test_errors_are_atomic():
+    a = P.BlockAllocator(2, 4)
+    a.allocate(1, 6)
+    a.fork(1, 2)
+    with pytest.raises(P.PkvError) as e:
+        a.append_slot(1)          # copy-on-write needs a free block
+    assert e.value.status == P.PKV_ERR_OOM
+    assert a.table(1) == [0, 1] and a.num_tokens(1) == 6 and a.refcount(1) == 2
+    with pytest.raises(P.PkvError) as e:
+        P.BlockAllocator(3, 4, [0, 0, 1])
+    assert e.value.status == P.PKV_ERR_INVALID_ARG

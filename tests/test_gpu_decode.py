@@ -1,0 +1,170 @@
+"""Decode attention on the GPU against the fp64 oracle (through the C ABI).
+
+Small cases compare every output element; the full-size workloads compare
+sampled sequences. Tolerances (max abs error vs the oracle on the stored,
+dequantised cache): fp16 2e-3, bf16 1e-2, fp8-e4m3 3e-2.
+"""
+import numpy as np
+import pytest
+import torch
+
+import paged_kv_cache_453_b200 as P
+import workloads as W
+from gpu_cases import TOL, decode_case, run_decode, oracle_decode, max_err, check_no_device_error
+from oracle.numerics import decode_e4m3
+from oracle_io import raw
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def setup():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from paged_kv_cache_453_b200.build import build
+    build()
+    torch.cuda.init()
+
+
+def _small(name, **kw):
+    base = W.spec(name)
+    return base.replace(**kw)
+
+
+SMALL = {
+    "tiny": W.spec("tiny"),
+    "8b_small": W.scaled_down(W.spec("llama3_8b"), 8, 700),
+    "70b_small": W.scaled_down(W.spec("llama3_70b"), 4, 900).replace(lens=("uniform", 300, 900)),
+    "mha_f16": W.spec("llama3_8b").replace(num_seqs=5, num_q_heads=6, num_kv_heads=6, cache_dtype="f16",
+                                           q_dtype="f16", lens=("uniform", 1, 400), table_width=None),
+    "skewed_b16": W.scaled_down(W.spec("long_skewed"), 16, 3000),
+    "skewed_b32": W.scaled_down(W.spec("long_skewed"), 16, 3000, block_size=32),
+    "skewed_fp8_b16": W.scaled_down(W.spec("long_skewed"), 16, 3000, cache_dtype="fp8_e4m3"),
+    "skewed_fp8_b32": W.scaled_down(W.spec("long_skewed"), 16, 3000, cache_dtype="fp8_e4m3",
+                                    block_size=32),
+    "fp8_f16q": W.scaled_down(W.spec("long_skewed"), 6, 500, cache_dtype="fp8_e4m3", q_dtype="f16"),
+    "d64_bf16_b32": W.spec("tiny").replace(cache_dtype="bf16", q_dtype="bf16", block_size=32,
+                                           pool_blocks=None, lens=("fixed", [5, 33, 64, 70])),
+    "d64_f16_b16_g1": W.spec("tiny").replace(num_q_heads=2, lens=("fixed", [3, 16, 31, 48])),
+    "f16_b32_g8": W.spec("llama3_70b").replace(num_seqs=3, cache_dtype="f16", q_dtype="f16",
+                                               block_size=32, lens=("fixed", [33, 100, 257]),
+                                               table_width=None),
+    "g3": W.spec("llama3_8b").replace(num_seqs=3, num_q_heads=6, num_kv_heads=2,
+                                      lens=("fixed", [40, 1, 77]), table_width=None),
+    "g6": W.spec("llama3_8b").replace(num_seqs=3, num_q_heads=12, num_kv_heads=2,
+                                      lens=("fixed", [140, 16, 17]), table_width=None),
+    "edge_lens": W.spec("llama3_8b").replace(num_seqs=9, lens=("fixed", [0, 1, 15, 16, 17, 31, 32, 33, 0]),
+                                             table_width=None),
+    "many_short": W.spec("llama3_8b").replace(num_seqs=300, num_q_heads=8, num_kv_heads=2,
+                                              lens=("uniform", 0, 40), table_width=None),
+    "one_long": W.spec("llama3_8b").replace(num_seqs=1, lens=("fixed", [6000]), table_width=None),
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_decode_matches_oracle_small(name):
+    s, lay, t = decode_case(SMALL[name], seed=SMALL[name].seed + 99)
+    out = run_decode(s, lay, t)
+    torch.cuda.synchronize()
+    check_no_device_error()
+    ref = oracle_decode(s, lay, t)
+    err = max_err(out, ref)
+    assert err <= TOL[s.cache_dtype], (name, err)
+
+
+def test_one_token_context_returns_v0_exactly():
+    for cd in ("f16", "bf16"):
+        s = W.spec("llama3_70b").replace(num_seqs=3, cache_dtype=cd, q_dtype=cd, lens=("fixed", [1, 1, 1]),
+                                         table_width=None)
+        s, lay, t = decode_case(s)
+        out = run_decode(s, lay, t)
+        for i in range(3):
+            blk = int(lay.tables[i, 0])
+            for h in range(s.num_q_heads):
+                v0 = t.v_cache[blk, h // s.group, 0]
+                assert torch.equal(out[i, h], v0), (cd, i, h)
+    check_no_device_error()
+
+
+def test_deterministic_and_explicit_workspace():
+    s, lay, t = decode_case(W.scaled_down(W.spec("long_skewed"), 16, 3000))
+    a = run_decode(s, lay, t)
+    b = run_decode(s, lay, t)
+    nbytes = P.workspace_bytes(s.num_q_heads, s.num_kv_heads, s.head_dim, s.block_size, P.PKV_BF16,
+                               torch.cuda.current_device())
+    assert nbytes > 0
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    c = run_decode(s, lay, t, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b) and torch.equal(a, c)
+    with pytest.raises(P.PkvError) as e:
+        run_decode(s, lay, t, workspace=ws[: nbytes // 2])
+    assert e.value.status == P.PKV_ERR_WORKSPACE
+    check_no_device_error()
+
+
+def test_fp8_widening_of_every_code():
+    # One token whose V row holds 128 codes: out = decode(code) * v_scale exactly
+    # (every e4m3 value is exact in bf16), for both halves of the code space.
+    for half in range(2):
+        s = W.spec("long_skewed").replace(num_seqs=1, num_q_heads=1, num_kv_heads=1, cache_dtype="fp8_e4m3",
+                                          lens=("fixed", [1]), table_width=None, pool_blocks=4)
+        s, lay, t = decode_case(s)
+        codes = torch.arange(128 * half, 128 * half + 128, dtype=torch.int64)
+        codes[codes == 0x7F] = 0x7E
+        codes[codes == 0xFF] = 0xFE
+        blk = int(lay.tables[0, 0])
+        t.v_cache[blk, 0, 0] = codes.to(torch.uint8).cuda()
+        t.v_scale.fill_(1.0)
+        out = run_decode(s, lay, t)
+        expect = torch.tensor(decode_e4m3(codes.numpy()), dtype=torch.float64)
+        assert torch.equal(out[0, 0].double().cpu(), expect), half
+    check_no_device_error()
+
+
+def test_bad_inputs_are_flagged_not_faulted():
+    s, lay, t = decode_case(W.spec("tiny"))
+    tables = lay.tables.clone()
+    tables[1, 0] = 10 ** 6                       # block id outside the pool
+    out = torch.empty_like(t.q)
+    P.paged_attn_decode(t.q, t.k_cache, t.v_cache, tables.cuda(), lay.lens.cuda(), s.num_kv_heads, s.scale,
+                        s.block_size, out)
+    assert P.device_error(torch.cuda.current_device()) == P.PKV_ERR_DEVICE_CHECK
+    lens = lay.lens.clone()
+    lens[2] = lay.tables.shape[1] * s.block_size + 5   # longer than the table row
+    P.paged_attn_decode(t.q, t.k_cache, t.v_cache, lay.tables.cuda(), lens.cuda(), s.num_kv_heads, s.scale,
+                        s.block_size, out)
+    assert P.device_error(torch.cuda.current_device()) == P.PKV_ERR_DEVICE_CHECK
+    check_no_device_error()                       # the flag was cleared
+    with pytest.raises(P.PkvError) as e:         # host-side shape check
+        P.paged_attn_decode(t.q, t.k_cache, t.v_cache, lay.tables.cuda(), lay.lens.cuda(), 3, s.scale,
+                            s.block_size, out)
+    assert e.value.status == P.PKV_ERR_INVALID_ARG
+
+
+def _sample(lens, k, rng):
+    order = np.argsort(lens)
+    pick = set(int(i) for i in order[-2:]) | set(int(i) for i in order[:2])
+    pick |= set(int(i) for i in rng.choice(len(lens), size=min(k, len(lens)), replace=False))
+    return sorted(pick)
+
+
+@pytest.mark.parametrize("name,over", [
+    ("llama3_8b", {}),
+    ("llama3_70b", {}),
+    ("long_skewed", {}),
+    ("long_skewed", {"block_size": 32}),
+    ("long_skewed", {"cache_dtype": "fp8_e4m3"}),
+    ("long_skewed", {"cache_dtype": "fp8_e4m3", "block_size": 32}),
+])
+def test_decode_full_size_sampled(name, over):
+    spec = W.spec(name, **over)
+    s, lay, t = decode_case(spec)
+    out = run_decode(s, lay, t)
+    torch.cuda.synchronize()
+    check_no_device_error()
+    seqs = _sample(lay.lens.numpy(), 4, np.random.default_rng(0))
+    ref = oracle_decode(s, lay, t, seqs=seqs)
+    err = max_err(out, ref, seqs)
+    assert err <= TOL[s.cache_dtype], (name, over, err)
+    # every other row is finite and bounded by the largest |v| of the pool
+    assert torch.isfinite(out).all()
