@@ -74,7 +74,8 @@ typedef enum {
   PKV_ERR_DOUBLE_FREE = -6,  /* allocator: reference count would drop below 0 */
   PKV_ERR_CUDA = -7,         /* a CUDA runtime call failed */
   PKV_ERR_DEVICE_CHECK = -8, /* a kernel recorded a bad index or a wait that ran out */
-  PKV_ERR_WORKSPACE = -9     /* caller-provided workspace too small */
+  PKV_ERR_WORKSPACE = -9,    /* caller-provided workspace too small */
+  PKV_ERR_SCRATCH_LIMIT = -10 /* needs more than the library's static scratch */
 } pkv_status;
 
 /* Text for a status code (static storage, never NULL). */
@@ -158,6 +159,41 @@ int paged_attn_decode_ex(const pkv_tensor* q, const pkv_tensor* k_cache,
                          const pkv_tensor* context_lens, int num_kv_heads, float scale,
                          int block_size, pkv_tensor* out, void* workspace,
                          size_t workspace_bytes, void* stream);
+
+/*
+ * paged_attn_decode_noalloc - paged_attn_decode / paged_attn_decode_fp8 for
+ * callers that cannot allocate device memory when they call: for example an
+ * engine that hands almost all of HBM to its own KV-block pool at start-up
+ * (a late cudaMalloc would fail or fragment that pool), or a caller whose
+ * latency budget cannot absorb the device synchronisation cudaMalloc
+ * implies. The pages have no counterpart of this call; it is a property of
+ * this library, not of the method.
+ *
+ * Same arguments and results as paged_attn_decode_ex without the workspace:
+ * k_scale / v_scale are NULL for a 16-bit cache and required for fp8. The
+ * split-KV scratch lives in a static device array of
+ * PKV_NOALLOC_SCRATCH_BYTES bytes that every GPU loading this library keeps
+ * until the process exits. The call allocates nothing: it calls no
+ * cudaMalloc / cudaFree and no allocating library routine.
+ *
+ *   - The first call on each device looks up that array's device address
+ *     (cudaGetSymbolAddress, with the device current); make that first call
+ *     before any stream capture on the device.
+ *   - A shape whose scratch would exceed the limit (it grows with the
+ *     device's SM count, the query-head group g and head_dim, not with the
+ *     context lengths) returns PKV_ERR_SCRATCH_LIMIT and launches nothing.
+ *   - All calls on a device share the one array and it keeps the last
+ *     call's contents; nothing in it needs to start at zero (the kernels
+ *     write every descriptor and partial before reading it). Calls that
+ *     overlap on the GPU (different streams, no ordering between them) race
+ *     on the array and give wrong results: serialise them.
+ */
+#define PKV_NOALLOC_SCRATCH_BYTES (16u << 20)
+int paged_attn_decode_noalloc(const pkv_tensor* q, const pkv_tensor* k_cache,
+                              const pkv_tensor* v_cache, const pkv_tensor* k_scale,
+                              const pkv_tensor* v_scale, const pkv_tensor* block_tables,
+                              const pkv_tensor* context_lens, int num_kv_heads, float scale,
+                              int block_size, pkv_tensor* out, void* stream);
 
 /* ------------------------------------------------------------------------ */
 /* Cache writes and block copies                                            */

@@ -38,12 +38,13 @@ PKV_ERR_DOUBLE_FREE = -6
 PKV_ERR_CUDA = -7
 PKV_ERR_DEVICE_CHECK = -8
 PKV_ERR_WORKSPACE = -9
+PKV_ERR_SCRATCH_LIMIT = -10
 
 # Every symbol include/pagedkv.h declares.
 EXPORTED = (
     "pkv_status_string", "pkv_version",
     "paged_attn_decode", "paged_attn_decode_fp8", "paged_attn_decode_workspace_bytes",
-    "paged_attn_decode_ex", "reshape_and_cache", "reshape_and_cache_fp8", "copy_blocks",
+    "paged_attn_decode_ex", "paged_attn_decode_noalloc", "reshape_and_cache", "reshape_and_cache_fp8", "copy_blocks",
     "pkv_device_error",
     "pkv_alloc_create", "pkv_alloc_destroy", "pkv_seq_allocate", "pkv_seq_append_slot",
     "pkv_seq_fork", "pkv_seq_free", "pkv_seq_num_tokens", "pkv_seq_block_table",
@@ -84,6 +85,8 @@ def lib() -> ctypes.CDLL:
             "paged_attn_decode_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int] * 6),
             "paged_attn_decode_ex": (ctypes.c_int, [P, P, P, P, P, P, P, ctypes.c_int, f32,
                                                     ctypes.c_int, P, vp, ctypes.c_size_t, vp]),
+            "paged_attn_decode_noalloc": (ctypes.c_int, [P, P, P, P, P, P, P, ctypes.c_int, f32,
+                                                         ctypes.c_int, P, vp]),
             "reshape_and_cache": (ctypes.c_int, [P, P, P, P, P, vp]),
             "reshape_and_cache_fp8": (ctypes.c_int, [P, P, P, P, P, P, P, vp]),
             "copy_blocks": (ctypes.c_int, [P, P, P, vp]),
@@ -205,6 +208,25 @@ def paged_attn_decode_ex(q, k_cache, v_cache, block_tables, context_lens, num_kv
                                       ctypes.c_void_p(workspace.data_ptr()),
                                       workspace.numel() * workspace.element_size(),
                                       _stream(stream)), "paged_attn_decode_ex")
+
+
+def paged_attn_decode_noalloc(q, k_cache, v_cache, block_tables, context_lens, num_kv_heads: int,
+                              scale: float, block_size: int, out, k_scale=None, v_scale=None,
+                              stream=None) -> None:
+    """Decode for callers that cannot allocate device memory at call time:
+    the split-KV scratch is a static device array of the library (see
+    paged_attn_decode_noalloc in include/pagedkv.h). Calls on one device
+    share that array, so calls that overlap on the GPU race."""
+    fp8 = k_scale is not None
+    ks = _desc(k_scale) if fp8 else None
+    vs = _desc(v_scale) if fp8 else None
+    ds = [_desc(q), _desc(k_cache, fp8), _desc(v_cache, fp8), _desc(block_tables),
+          _desc(context_lens), _desc(out)]
+    _check(lib().paged_attn_decode_noalloc(_ref(ds[0]), _ref(ds[1]), _ref(ds[2]),
+                                           _ref(ks) if fp8 else None, _ref(vs) if fp8 else None,
+                                           _ref(ds[3]), _ref(ds[4]), int(num_kv_heads), float(scale),
+                                           int(block_size), _ref(ds[5]), _stream(stream)),
+           "paged_attn_decode_noalloc")
 
 
 def reshape_and_cache(k, v, k_cache, v_cache, slot_mapping, stream=None) -> None:

@@ -419,6 +419,34 @@ int launch_reshape(const pkv_tensor* k, const pkv_tensor* v, pkv_tensor* kc, pkv
 }  // namespace
 }  // namespace pkv
 
+// Split-KV scratch of paged_attn_decode_noalloc: a fixed array in device
+// memory, created when the library's module is loaded on a device, so that
+// call needs no allocation. In host code this name is only a handle: its
+// device address comes from cudaGetSymbolAddress below.
+static __device__ __align__(256) unsigned char pkv_noalloc_scratch[PKV_NOALLOC_SCRATCH_BYTES];
+
+namespace pkv {
+namespace {
+
+void* g_noalloc_ptr[kMaxDevices];
+
+// Device address of pkv_noalloc_scratch on `dev` (which must be current),
+// looked up once per device.
+int noalloc_scratch(int dev, void** out) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, pkv_noalloc_scratch);
+    if (e != cudaSuccess || !p) return PKV_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return PKV_OK;
+}
+
+}  // namespace
+}  // namespace pkv
+
 using namespace pkv;
 
 extern "C" {
@@ -435,6 +463,7 @@ const char* pkv_status_string(int s) {
     case PKV_ERR_CUDA: return "CUDA error";
     case PKV_ERR_DEVICE_CHECK: return "device-side check failed";
     case PKV_ERR_WORKSPACE: return "workspace missing or too small";
+    case PKV_ERR_SCRATCH_LIMIT: return "request needs more than the static scratch limit";
     default: return "unknown status";
   }
 }
@@ -490,6 +519,35 @@ int paged_attn_decode_ex(const pkv_tensor* q, const pkv_tensor* k_cache,
   DecodeArgs a{q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
                num_kv_heads, scale, block_size, out};
   return launch_decode(a, fp8, workspace, workspace_bytes, false,
+                       static_cast<cudaStream_t>(stream));
+}
+
+// Decode for callers that cannot allocate: the scratch is the static
+// pkv_noalloc_scratch array of this file (see the declaration in pagedkv.h).
+int paged_attn_decode_noalloc(const pkv_tensor* q, const pkv_tensor* k_cache,
+                              const pkv_tensor* v_cache, const pkv_tensor* k_scale,
+                              const pkv_tensor* v_scale, const pkv_tensor* block_tables,
+                              const pkv_tensor* context_lens, int num_kv_heads, float scale,
+                              int block_size, pkv_tensor* out, void* stream) {
+  const bool fp8 = k_cache && k_cache->dtype == PKV_FP8_E4M3;
+  DecodeArgs a{q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
+               num_kv_heads, scale, block_size, out};
+  int ck = 0;
+  DecodeLaunch* e = nullptr;
+  int st = check_decode(a, fp8, &ck, &e);
+  if (st != PKV_OK || !e) return st;
+  int dev;
+  if ((st = current_device(&dev)) != PKV_OK) return st;
+  DeviceState* ds;
+  if ((st = device_state(dev, &ds)) != PKV_OK) return st;
+  int grid;
+  if ((st = decode_grid(e, dev, ds->sms, &grid)) != PKV_OK) return st;
+  const int g = static_cast<int>(q->shape[1] / num_kv_heads);
+  const size_t need = ws_layout(grid * e->nc, g, static_cast<int>(q->shape[2])).total;
+  if (need > PKV_NOALLOC_SCRATCH_BYTES) return PKV_ERR_SCRATCH_LIMIT;
+  void* scratch = nullptr;
+  if ((st = noalloc_scratch(dev, &scratch)) != PKV_OK) return st;
+  return launch_decode(a, fp8, scratch, PKV_NOALLOC_SCRATCH_BYTES, false,
                        static_cast<cudaStream_t>(stream));
 }
 
