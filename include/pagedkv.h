@@ -150,8 +150,11 @@ size_t paged_attn_decode_workspace_bytes(int num_q_heads, int num_kv_heads, int 
  * paged_attn_decode_ex - the general form: k_scale / v_scale are NULL for a
  * 16-bit cache and required for fp8; `workspace` is a caller-owned device
  * buffer of at least paged_attn_decode_workspace_bytes() bytes (16-byte
- * aligned), else PKV_ERR_WORKSPACE. The workspace must not be used by
- * another call until this one has finished on the GPU.
+ * aligned), else PKV_ERR_WORKSPACE. Zero-fill it once before its first use
+ * (e.g. cudaMemset): it holds the split-KV work-claiming state, which every
+ * call leaves zeroed again. The workspace must not be used by another call
+ * until this one has finished on the GPU; after a PKV_ERR_DEVICE_CHECK from
+ * a call that used it, zero it again.
  */
 int paged_attn_decode_ex(const pkv_tensor* q, const pkv_tensor* k_cache,
                          const pkv_tensor* v_cache, const pkv_tensor* k_scale,
@@ -179,14 +182,19 @@ int paged_attn_decode_ex(const pkv_tensor* q, const pkv_tensor* k_cache,
  *   - The first call on each device looks up that array's device address
  *     (cudaGetSymbolAddress, with the device current); make that first call
  *     before any stream capture on the device.
- *   - A shape whose scratch would exceed the limit (it grows with the
- *     device's SM count, the query-head group g and head_dim, not with the
- *     context lengths) returns PKV_ERR_SCRATCH_LIMIT and launches nothing.
+ *   - A shape whose minimum scratch would exceed the limit (it grows with
+ *     the device's SM count, the query-head group g and head_dim, not with
+ *     the context lengths) returns PKV_ERR_SCRATCH_LIMIT and launches
+ *     nothing.
  *   - All calls on a device share the one array and it keeps the last
- *     call's contents; nothing in it needs to start at zero (the kernels
- *     write every descriptor and partial before reading it). Calls that
- *     overlap on the GPU (different streams, no ordering between them) race
- *     on the array and give wrong results: serialise them.
+ *     call's contents; each call first zeroes the part that must start at
+ *     zero (the work-claiming state, a few KB, with cudaMemsetAsync on
+ *     `stream`). Calls that overlap on the GPU (different streams, no
+ *     ordering between them) race on the array and give wrong results:
+ *     serialise them.
+ *   - When the default split-KV scratch does not fit, the call keeps fewer
+ *     slots for rebalancing work between warps (same results, possibly a
+ *     little slower).
  */
 #define PKV_NOALLOC_SCRATCH_BYTES (16u << 20)
 int paged_attn_decode_noalloc(const pkv_tensor* q, const pkv_tensor* k_cache,

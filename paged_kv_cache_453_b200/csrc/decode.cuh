@@ -10,11 +10,17 @@
 // block b) triple; items are ordered s-major, then h, then b, and a unit
 // (s, h) owns max(ceil(L_s / B), 1) consecutive items (an empty sequence keeps
 // one item so that its output is written). The W items are cut into equal
-// contiguous ranges, one per warp of a grid sized to fill every SM once, so
-// every warp streams the same number of KV bytes whatever the length mix.
-// A warp writes the output of every unit that lies wholly inside its range;
-// a unit cut by a range boundary leaves fp32 partials (m, l, unnormalised O)
-// per piece, and decode_merge_kernel combines them.
+// contiguous ranges, one per warp of a grid that fills every SM once.
+// Equal bytes do not mean equal time: SMs in some GPCs get less DRAM
+// bandwidth than others. So a warp claims the items of its range one by one
+// from the front of an atomic range word, and a warp that runs out steals the
+// back half of the largest unclaimed remainder (a steal is one CAS on that
+// word). Every range, own or stolen, is a contiguous sub-range of items; a
+// warp writes the output of each unit that lies wholly inside a sub-range it
+// processed, and a unit cut by sub-range boundaries leaves fp32 partials
+// (m, l, unnormalised O) per piece, which decode_merge_kernel combines.
+// Range words and the steal-slot pool start at zero and the merge kernel
+// zeroes them again after use; steal records carry a 32-bit call tag.
 //
 // Per warp: a private ring of NS shared-memory stages. Lane 0 issues the TMA
 // tensor loads of one item (the K tile and the V tile of one (block, head):
@@ -36,11 +42,18 @@
 // folded into the logit scale and the output.
 #pragma once
 
+#include <type_traits>
+
 #include "ptx.cuh"
 
 namespace pkv {
 
 enum CacheKind : int { kCacheF16 = 0, kCacheBF16 = 1, kCacheE4M3 = 2 };
+
+constexpr int kMaxSteals = 6;     // steals from one warp's range per call
+constexpr int kMinStealable = 8;  // a remainder worth splitting (items)
+constexpr int kStealTries = 8;
+constexpr int kErrBadMerge = 16;  // a merge record out of range (skipped)
 
 struct DecodeParams {
   CUtensorMap tmk;  // K pool viewed as {D, B, Hk, NB}
@@ -56,12 +69,17 @@ struct DecodeParams {
   const float* v_scale;
   float scale_log2;  // softmax scale * log2(e)
   int S, Hk, g, MB, NB;
-  int nwt;            // consumer warps in the grid
-  long long* hdr;     // workspace header: [0] total items W
-  int* err;           // device-check flag (OR of error bits)
-  float* part_o;      // [nwt][2][g][D]
-  float* part_ml;     // [nwt][2][g][2]
-  int4* desc;         // [nwt] last-segment descriptor (s, h, U1 lo, U1 hi); s < 0: none
+  int nwt;                    // consumer warps in the grid
+  int tag;                    // per-call tag of steal records (never 0)
+  int pool_slots;             // partial slots available to steals
+  long long* hdr;             // workspace header: [0] total items W
+  int* err;                   // device-check flag (OR of error bits)
+  unsigned long long* words;  // [nwt] range word: front | back | steals; 0 between calls
+  unsigned* pool;             // steal-slot pool counter; 0 between calls
+  int4* steal_info;           // [nwt][kMaxSteals] (start lo, slot base, tag, start hi)
+  int4* desc;                 // [nwt][1 + kMaxSteals] last-piece descriptor per sub-range
+  float* part_o;              // [2 nwt + pool_slots][g][D]
+  float* part_ml;             // [2 nwt + pool_slots][g][2]
 };
 
 __device__ __forceinline__ uint64_t global_ns() {
@@ -82,10 +100,33 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, uint64_
   }
 }
 
+// ---- range words: front [0,24) | back [24,48) | steals [48,52)
+// front counts items the owner claimed, back items thieves took from the end.
+__device__ __forceinline__ unsigned rw_front(unsigned long long w) { return unsigned(w & 0xffffffu); }
+__device__ __forceinline__ unsigned rw_back(unsigned long long w) {
+  return unsigned((w >> 24) & 0xffffffu);
+}
+__device__ __forceinline__ unsigned rw_steals(unsigned long long w) {
+  return unsigned((w >> 48) & 0xfu);
+}
+__device__ __forceinline__ unsigned long long rw_make(unsigned front, unsigned back, unsigned steals) {
+  return static_cast<unsigned long long>(front) | (static_cast<unsigned long long>(back) << 24) |
+         (static_cast<unsigned long long>(steals) << 48);
+}
+__device__ __forceinline__ unsigned long long ld_relaxed(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
 template <int BS>
 __device__ __forceinline__ int items_of(int L) {
   int n = (L + BS - 1) / BS;
   return n > 0 ? n : 1;
+}
+
+__device__ __forceinline__ long long range_lo(long long w, long long W, int nwt) {
+  return (w * W) / nwt;
 }
 
 template <int BS>
@@ -129,6 +170,7 @@ struct DecodeCfg {
   static_assert((D * EB) % 128 == 0, "head_dim * elem bytes must be a multiple of 128");
   static_assert(BS % 16 == 0, "block_size must be a multiple of 16");
   static_assert(TILE % 1024 == 0, "tiles must keep 1 KiB swizzle alignment");
+  static_assert(NS >= 2, "the claim pipeline needs two stages");
 };
 
 // Byte offset of 16-byte chunk `bcol / 16` of token row `t` inside a tile
@@ -162,6 +204,9 @@ __global__ void __launch_bounds__(NC * 32) decode_kernel(const __grid_constant__
   const int c = lane & 3;   // thread in group
   const int max_len = p.MB * BS;
 
+  // The merge kernel may be scheduled now; it waits for this grid to finish.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
   if (lane == 0) {
     for (int i = 0; i < NS; ++i) mbar_init(bars + (warp * NS + i) * 8, 1);
   }
@@ -184,8 +229,7 @@ __global__ void __launch_bounds__(NC * 32) decode_kernel(const __grid_constant__
       }
       sum += static_cast<long long>(p.Hk) * items_of<BS>(len);
     }
-    // inclusive warp scan, then warp totals
-    long long v = sum;
+    long long v = sum;  // inclusive warp scan, then warp totals
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       long long u = __shfl_up_sync(0xffffffffu, v, o);
@@ -209,19 +253,21 @@ __global__ void __launch_bounds__(NC * 32) decode_kernel(const __grid_constant__
   if (blockIdx.x == 0 && tid == 0) p.hdr[0] = W;
 
   const int gw = blockIdx.x * NC + warp;
-  const long long lo = (static_cast<long long>(gw) * W) / p.nwt;
-  const long long hi = (static_cast<long long>(gw + 1) * W) / p.nwt;
-  if (lane == 0) p.desc[gw] = make_int4(-1, 0, 0, 0);
-  if (lo >= hi) return;
+  const long long my_lo = range_lo(gw, W, p.nwt);
+  const long long my_len = range_lo(gw + 1, W, p.nwt) - my_lo;
+  if (my_len >= (1ll << 23)) {  // range words hold 24-bit counts
+    if (lane == 0) atomicOr(p.err, kErrBadLen);
+    return;
+  }
 
-  // ---- locate the item `lo`: chunk by binary search, then a warp-wide walk ----
-  Cursor<BS> cur;
-  cur.k = -1;
-  {
+  if (lane == 0) p.desc[gw * (1 + kMaxSteals)] = make_int4(-1, 0, 0, 0);
+
+  // Position of global item x: chunk by binary search, then a warp-wide walk.
+  auto locate = [&](long long x, Cursor<BS>& out) -> bool {
     int a = 0, bnd = C::NT - 1;
-    while (a < bnd) {  // largest t with scan[t] <= lo
+    while (a < bnd) {  // largest t with scan[t] <= x
       int m = (a + bnd + 1) >> 1;
-      if (scan[m] <= lo) a = m;
+      if (scan[m] <= x) a = m;
       else bnd = m - 1;
     }
     const int s_lo = static_cast<int>((static_cast<long long>(a) * p.S) / C::NT);
@@ -242,28 +288,25 @@ __global__ void __launch_bounds__(NC * 32) decode_kernel(const __grid_constant__
         long long u = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += u;
       }
-      const unsigned hit = __ballot_sync(0xffffffffu, s < s_hi && base + incl > lo);
+      const unsigned hit = __ballot_sync(0xffffffffu, s < s_hi && base + incl > x);
       if (hit) {
         const int j = __ffs(hit) - 1;
         const long long start = __shfl_sync(0xffffffffu, base + incl - w, j);
         const int L = __shfl_sync(0xffffffffu, len, j);
         const int n = items_of<BS>(L);
-        const long long off = lo - start;
-        cur.k = lo;
-        cur.s = s0 + j;
-        cur.h = static_cast<int>(off / n);
-        cur.b = static_cast<int>(off % n);
-        cur.L = L;
-        cur.n = n;
-        break;
+        const long long off = x - start;
+        out.k = x;
+        out.s = s0 + j;
+        out.h = static_cast<int>(off / n);
+        out.b = static_cast<int>(off % n);
+        out.L = L;
+        out.n = n;
+        return true;
       }
       base += __shfl_sync(0xffffffffu, incl, 31);
     }
-  }
-  if (cur.k != lo) {  // unreachable when the scan is consistent; never index with garbage
-    if (lane == 0) atomicOr(p.err, kErrBadLen);
-    return;
-  }
+    return false;
+  };
 
   const uint64_t policy = l2_policy_evict_first();
   const uint32_t my_stages = stages + warp * NS * C::STAGE;
@@ -271,356 +314,658 @@ __global__ void __launch_bounds__(NC * 32) decode_kernel(const __grid_constant__
 
   // Table-entry window of the producer: lane j holds table[tw_s][tw_b0 + j].
   int tw_s = -1, tw_b0 = 0, tw_val = 0;
-  Cursor<BS> pc = cur;
+  long long it = 0;      // items consumed by this warp (ring position)
+  long long issued = 0;  // items issued into the ring
 
-  auto issue = [&](int stage) {
-    const uint32_t bar = my_bars + stage * 8;
-    if (pc.L == 0) {
-      if (lane == 0) mbar_arrive(bar);
-      return;
-    }
-    if (pc.s != tw_s || pc.b < tw_b0 || pc.b >= tw_b0 + 32) {
-      tw_s = pc.s;
-      tw_b0 = pc.b;
-      const int nb = (pc.L + BS - 1) / BS;
-      tw_val = (tw_b0 + lane < nb) ? __ldg(p.tables + pc.s * p.t_s + tw_b0 + lane) : 0;
-    }
-    int phys = __shfl_sync(0xffffffffu, tw_val, pc.b - tw_b0);
-    if (phys < 0 || phys >= p.NB) {
-      if (lane == 0) atomicOr(p.err, kErrBadBlock);
-      phys = 0;
-    }
-    if (lane == 0) {
-      const uint32_t dk = my_stages + stage * C::STAGE;
-      const uint32_t dv = dk + C::TILE;
-      mbar_arrive_expect_tx(bar, C::STAGE);
-#pragma unroll
-      for (int hh = 0; hh < C::NH; ++hh)
-        tma_load_4d(dk + hh * BS * 128, &p.tmk, bar, hh * C::EPR, 0, pc.h, phys, policy);
-#pragma unroll
-      for (int hh = 0; hh < C::NH; ++hh)
-        tma_load_4d(dv + hh * BS * 128, &p.tmv, bar, hh * C::EPR, 0, pc.h, phys, policy);
-    }
-  };
-
-  long long issued = 0;
-  for (int i = 0; i < NS && pc.k < hi; ++i) {
-    issue(i);
-    pc.advance(p, max_len);
-    ++issued;
-  }
-
-  // ---- per-unit state ----
   uint32_t qb[C::KS][2];
   float acc[C::MT][4];
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
   float sl = p.scale_log2;
-
   const bool h0_ok = (2 * c) < p.g;
   const bool h1_ok = (2 * c + 1) < p.g;
 
-  auto begin_unit = [&]() {
-#pragma unroll
-    for (int mt = 0; mt < C::MT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
-    m0 = m1 = -INFINITY;
-    l0 = l1 = 0.f;
-    sl = p.scale_log2;
-    if constexpr (FP8) sl *= __ldg(p.k_scale + cur.h);
-    const bool row_ok = r < p.g;
-    const long long qoff = cur.s * p.q_s + (static_cast<long long>(cur.h) * p.g + r) * p.q_h;
-    if constexpr (!FP8) {
-      const uint32_t* qp = reinterpret_cast<const uint32_t*>(
-          static_cast<const uint16_t*>(p.q) + qoff);
-#pragma unroll
-      for (int ks = 0; ks < C::KS; ++ks) {
-        qb[ks][0] = row_ok ? __ldg(qp + (ks * 16 + 2 * c) / 2) : 0u;
-        qb[ks][1] = row_ok ? __ldg(qp + (ks * 16 + 8 + 2 * c) / 2) : 0u;
-      }
-    } else {
-      // k-slot order of the widened fp8 tile: slots 2c, 2c+1 <- dims 4c, 4c+1
-      // and slots 2c+8, 2c+9 <- dims 4c+2, 4c+3 of each 16-dim step.
-      const uint2* qp = reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(p.q) + qoff);
-#pragma unroll
-      for (int ks = 0; ks < C::KS; ++ks) {
-        uint2 v = row_ok ? __ldg(qp + (ks * 16 + 4 * c) / 4) : make_uint2(0u, 0u);
-        float f0, f1, f2, f3;
-        if constexpr (QBF) {
-          f0 = __uint_as_float(v.x << 16);
-          f1 = __uint_as_float(v.x & 0xffff0000u);
-          f2 = __uint_as_float(v.y << 16);
-          f3 = __uint_as_float(v.y & 0xffff0000u);
-        } else {
-          __half2 a = *reinterpret_cast<__half2*>(&v.x);
-          __half2 b = *reinterpret_cast<__half2*>(&v.y);
-          f0 = __low2float(a);
-          f1 = __high2float(a);
-          f2 = __low2float(b);
-          f3 = __high2float(b);
-        }
-        qb[ks][0] = pack2<false>(f0, f1);
-        qb[ks][1] = pack2<false>(f2, f3);
-      }
+  // Process the sub-range [a, hi) of warp `owner`'s static range as its
+  // `sub`-th sub-range (0 = the owner's own front part, j + 1 = steal j).
+  // In claim mode the items are claimed one by one from the range word, and
+  // hi drops to where thieves took over. Partials go to slots slot_base (+1).
+  auto run_range = [&](long long a, long long hi, bool claim, int owner, int sub,
+                       long long slot_base) -> bool {
+    Cursor<BS> cur;
+    if (!locate(a, cur)) {
+      if (lane == 0) atomicOr(p.err, kErrBadLen);
+      return false;
     }
-  };
+    Cursor<BS> pc = cur;
+    const long long lo = a;
+    unsigned long long* wp = p.words + owner;
+    const unsigned own_len = static_cast<unsigned>(hi - a);
+    bool claiming = claim;
+    unsigned long long pend = 0;  // lane 0: pending claim of the item at pc
 
-  auto finish_unit = [&]() {
-    // full row sums per head: reduce the thread partials over the 8 row groups
-#pragma unroll
-    for (int o = 4; o < 32; o <<= 1) {
-      l0 += __shfl_xor_sync(0xffffffffu, l0, o);
-      l1 += __shfl_xor_sync(0xffffffffu, l1, o);
-    }
-    float vs = 1.f;
-    if constexpr (FP8) vs = __ldg(p.v_scale + cur.h);
-    const long long ub = cur.unit_begin(), ue = cur.unit_end();
-    const int hq0 = cur.h * p.g + 2 * c;
-    if (ub >= lo && ue <= hi) {  // whole unit in this warp: final output
-      const float i0 = l0 > 0.f ? vs / l0 : 0.f;
-      const float i1 = l1 > 0.f ? vs / l1 : 0.f;
-      uint16_t* o = static_cast<uint16_t*>(p.out) + cur.s * p.o_s;
-#pragma unroll
-      for (int mt = 0; mt < C::MT; ++mt) {
-        const int da = FP8 ? 16 * mt + 2 * r : 16 * mt + r;
-        const int db = FP8 ? da + 1 : da + 8;
-        if (h0_ok) {
-          uint16_t* oh = o + hq0 * p.o_h;
-          float x = acc[mt][0] * i0, y = acc[mt][2] * i0;
-          if constexpr (QBF) {
-            oh[da] = __bfloat16_as_ushort(__float2bfloat16_rn(x));
-            oh[db] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
-          } else {
-            oh[da] = __half_as_ushort(__float2half_rn(x));
-            oh[db] = __half_as_ushort(__float2half_rn(y));
-          }
-        }
-        if (h1_ok) {
-          uint16_t* oh = o + (hq0 + 1) * p.o_h;
-          float x = acc[mt][1] * i1, y = acc[mt][3] * i1;
-          if constexpr (QBF) {
-            oh[da] = __bfloat16_as_ushort(__float2bfloat16_rn(x));
-            oh[db] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
-          } else {
-            oh[da] = __half_as_ushort(__float2half_rn(x));
-            oh[db] = __half_as_ushort(__float2half_rn(y));
-          }
-        }
+    auto issue = [&](int stage) {
+      const uint32_t bar = my_bars + stage * 8;
+      if (pc.L == 0) {
+        if (lane == 0) mbar_arrive(bar);
+        return;
       }
-    } else {  // piece of a cut unit: fp32 partials for the merge kernel
-      const int slot = ub < lo ? 0 : 1;
-      const long long base = (static_cast<long long>(gw) * 2 + slot) * p.g;
-      float* po = p.part_o + base * D;
+      if (pc.s != tw_s || pc.b < tw_b0 || pc.b >= tw_b0 + 32) {
+        tw_s = pc.s;
+        tw_b0 = pc.b;
+        const int nb = (pc.L + BS - 1) / BS;
+        tw_val = (tw_b0 + lane < nb) ? __ldg(p.tables + pc.s * p.t_s + tw_b0 + lane) : 0;
+      }
+      int phys = __shfl_sync(0xffffffffu, tw_val, pc.b - tw_b0);
+      if (phys < 0 || phys >= p.NB) {
+        if (lane == 0) atomicOr(p.err, kErrBadBlock);
+        phys = 0;
+      }
+      if (lane == 0) {
+        const uint32_t dk = my_stages + stage * C::STAGE;
+        const uint32_t dv = dk + C::TILE;
+        mbar_arrive_expect_tx(bar, C::STAGE);
 #pragma unroll
-      for (int mt = 0; mt < C::MT; ++mt) {
-        const int da = FP8 ? 16 * mt + 2 * r : 16 * mt + r;
-        const int db = FP8 ? da + 1 : da + 8;
-        if (h0_ok) {
-          po[(2 * c) * D + da] = acc[mt][0] * vs;
-          po[(2 * c) * D + db] = acc[mt][2] * vs;
-        }
-        if (h1_ok) {
-          po[(2 * c + 1) * D + da] = acc[mt][1] * vs;
-          po[(2 * c + 1) * D + db] = acc[mt][3] * vs;
+        for (int hh = 0; hh < C::NH; ++hh)
+          tma_load_4d(dk + hh * BS * 128, &p.tmk, bar, hh * C::EPR, 0, pc.h, phys, policy);
+#pragma unroll
+        for (int hh = 0; hh < C::NH; ++hh)
+          tma_load_4d(dv + hh * BS * 128, &p.tmv, bar, hh * C::EPR, 0, pc.h, phys, policy);
+      }
+    };
+    // Issue the item at pc into the next ring stage if it is ours; false when
+    // the sub-range has ended.
+    auto try_issue = [&]() -> bool {
+      if (pc.k >= hi) return false;
+      if (claiming) {
+        const unsigned long long w = __shfl_sync(0xffffffffu, pend, 0);
+        if (rw_front(w) + rw_back(w) >= own_len) {
+          claiming = false;
+          hi = pc.k;  // everything from here on belongs to thieves
+          return false;
         }
       }
-      if (r == 0) {
-        float* pm = p.part_ml + base * 2;
-        if (h0_ok) {
-          pm[(2 * c) * 2 + 0] = m0;
-          pm[(2 * c) * 2 + 1] = l0;
-        }
-        if (h1_ok) {
-          pm[(2 * c + 1) * 2 + 0] = m1;
-          pm[(2 * c + 1) * 2 + 1] = l1;
-        }
-      }
-      if (slot == 1 && lane == 0)
-        p.desc[gw] = make_int4(cur.s, cur.h, static_cast<int>(ue & 0xffffffffll),
-                               static_cast<int>(ue >> 32));
-    }
-  };
-
-  // ---- main loop ----
-  long long it = 0;
-  while (cur.k < hi) {
-    if (cur.b == 0 || cur.k == lo) begin_unit();
-    const int stage = static_cast<int>(it % NS);
-    const uint32_t parity = static_cast<uint32_t>((it / NS) & 1);
-    if (!warp_wait(my_bars + stage * 8, parity, kWaitNs)) {
-      if (lane == 0) atomicOr(p.err, kErrWaitTimeout);
-      for (long long j = it + 1; j < issued; ++j)  // let copies in flight land
-        warp_wait(my_bars + static_cast<int>(j % NS) * 8, static_cast<uint32_t>((j / NS) & 1),
-                  100000000ull);
-      return;
-    }
-
-    if (cur.L > 0) {
-      const uint32_t tk = my_stages + stage * C::STAGE;
-      const uint32_t tv = tk + C::TILE;
-      const int nvalid = min(BS, cur.L - cur.b * BS);
-
-      // S^T = K Q^T
-      float sacc[C::TT][4];
-#pragma unroll
-      for (int tt = 0; tt < C::TT; ++tt) {
-        sacc[tt][0] = sacc[tt][1] = sacc[tt][2] = sacc[tt][3] = 0.f;
-        const int trow = tt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-        if constexpr (!FP8) {
-#pragma unroll
-          for (int ks = 0; ks < C::KS; ++ks) {
-            uint32_t a0, a1, a2, a3;
-            ldsm_x4(tk + swz<BS>(trow, ks * 32 + (lane >> 4) * 16), a0, a1, a2, a3);
-            mma16816<MBF>(sacc[tt], a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
-          }
-        } else {
-#pragma unroll
-          for (int kp = 0; kp < C::KS / 2; ++kp) {
-            uint32_t x0, x1, x2, x3;
-            ldsm_x4(tk + swz<BS>(trow, kp * 32 + (lane >> 4) * 16), x0, x1, x2, x3);
-            mma16816<false>(sacc[tt], e4m3x2_to_f16x2(x0 & 0xffff), e4m3x2_to_f16x2(x1 & 0xffff),
-                            e4m3x2_to_f16x2(x0 >> 16), e4m3x2_to_f16x2(x1 >> 16), qb[2 * kp][0],
-                            qb[2 * kp][1]);
-            mma16816<false>(sacc[tt], e4m3x2_to_f16x2(x2 & 0xffff), e4m3x2_to_f16x2(x3 & 0xffff),
-                            e4m3x2_to_f16x2(x2 >> 16), e4m3x2_to_f16x2(x3 >> 16),
-                            qb[2 * kp + 1][0], qb[2 * kp + 1][1]);
-          }
-        }
-      }
-
-      // online softmax over this block's tokens, per head column
-      float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-      for (int tt = 0; tt < C::TT; ++tt) {
-        const int t0 = tt * 16 + r, t1 = t0 + 8;
-        sacc[tt][0] = t0 < nvalid ? sacc[tt][0] * sl : -INFINITY;
-        sacc[tt][1] = t0 < nvalid ? sacc[tt][1] * sl : -INFINITY;
-        sacc[tt][2] = t1 < nvalid ? sacc[tt][2] * sl : -INFINITY;
-        sacc[tt][3] = t1 < nvalid ? sacc[tt][3] * sl : -INFINITY;
-        mx0 = fmaxf(mx0, fmaxf(sacc[tt][0], sacc[tt][2]));
-        mx1 = fmaxf(mx1, fmaxf(sacc[tt][1], sacc[tt][3]));
-      }
-#pragma unroll
-      for (int o = 4; o < 32; o <<= 1) {
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
-      }
-      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);  // finite: nvalid >= 1
-      const float al0 = exp2f(m0 - mn0), al1 = exp2f(m1 - mn1);
-      m0 = mn0;
-      m1 = mn1;
-      uint32_t pb[C::TT][2];
-      float ps0 = 0.f, ps1 = 0.f;
-#pragma unroll
-      for (int tt = 0; tt < C::TT; ++tt) {
-        const float p0 = exp2f(sacc[tt][0] - mn0), p1 = exp2f(sacc[tt][1] - mn1);
-        const float p2 = exp2f(sacc[tt][2] - mn0), p3 = exp2f(sacc[tt][3] - mn1);
-        ps0 += p0 + p2;
-        ps1 += p1 + p3;
-        pb[tt][0] = movmatrix_t(pack2<MBF>(p0, p1));
-        pb[tt][1] = movmatrix_t(pack2<MBF>(p2, p3));
-      }
-      l0 = l0 * al0 + ps0;
-      l1 = l1 * al1 + ps1;
-#pragma unroll
-      for (int mt = 0; mt < C::MT; ++mt) {
-        acc[mt][0] *= al0;
-        acc[mt][1] *= al1;
-        acc[mt][2] *= al0;
-        acc[mt][3] *= al1;
-      }
-
-      // O^T += V^T P^T
-#pragma unroll
-      for (int tt = 0; tt < C::TT; ++tt) {
-        // tokens of this thread's A-fragment halves: lo = 2c, hi = 2c+1 (+8 for a2/a3)
-        const int tb = tt * 16 + 2 * c;
-        const uint32_t keep01 = (tb < nvalid ? 0x0000ffffu : 0u) | (tb + 1 < nvalid ? 0xffff0000u : 0u);
-        const uint32_t keep23 =
-            (tb + 8 < nvalid ? 0x0000ffffu : 0u) | (tb + 9 < nvalid ? 0xffff0000u : 0u);
-        if constexpr (!FP8) {
-          const int vrow = tt * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
-#pragma unroll
-          for (int mt = 0; mt < C::MT; ++mt) {
-            uint32_t a0, a1, a2, a3;
-            ldsm_x4_t(tv + swz<BS>(vrow, mt * 32 + ((lane >> 3) & 1) * 16), a0, a1, a2, a3);
-            mma16816<MBF>(acc[mt], a0 & keep01, a1 & keep01, a2 & keep23, a3 & keep23, pb[tt][0],
-                          pb[tt][1]);
-          }
-        } else {
-          const int vrow = tt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-#pragma unroll
-          for (int mp = 0; mp < C::MT / 2; ++mp) {
-            uint32_t x0, x1, x2, x3;
-            ldsm_x4_t(tv + swz<BS>(vrow, mp * 32 + (lane >> 4) * 16), x0, x1, x2, x3);
-            const uint32_t e0 = prmt(x0, 0, 0x3120), e1 = prmt(x1, 0, 0x3120);
-            const uint32_t e2 = prmt(x2, 0, 0x3120), e3 = prmt(x3, 0, 0x3120);
-            mma16816<false>(acc[2 * mp], e4m3x2_to_f16x2(e0 & 0xffff) & keep01,
-                            e4m3x2_to_f16x2(e0 >> 16) & keep01,
-                            e4m3x2_to_f16x2(e1 & 0xffff) & keep23,
-                            e4m3x2_to_f16x2(e1 >> 16) & keep23, pb[tt][0], pb[tt][1]);
-            mma16816<false>(acc[2 * mp + 1], e4m3x2_to_f16x2(e2 & 0xffff) & keep01,
-                            e4m3x2_to_f16x2(e2 >> 16) & keep01,
-                            e4m3x2_to_f16x2(e3 & 0xffff) & keep23,
-                            e4m3x2_to_f16x2(e3 >> 16) & keep23, pb[tt][0], pb[tt][1]);
-          }
-        }
-      }
-    }
-
-    __syncwarp();
-    if (pc.k < hi) {  // refill this stage NS items ahead
-      issue(stage);
+      issue(static_cast<int>(issued % NS));
       pc.advance(p, max_len);
       ++issued;
+      if (claiming && lane == 0) pend = atomicAdd(wp, 1ull);  // claim the following item
+      return true;
+    };
+
+    if (lane == 0) p.desc[owner * (1 + kMaxSteals) + sub] = make_int4(-1, 0, 0, 0);
+    if (claiming && lane == 0) pend = atomicAdd(wp, 1ull);
+    for (int i = 0; i < NS; ++i)
+      if (!try_issue()) break;
+
+    auto begin_unit = [&]() {
+#pragma unroll
+      for (int mt = 0; mt < C::MT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+      m0 = m1 = -INFINITY;
+      l0 = l1 = 0.f;
+      sl = p.scale_log2;
+      if constexpr (FP8) sl *= __ldg(p.k_scale + cur.h);
+      const bool row_ok = r < p.g;
+      const long long qoff = cur.s * p.q_s + (static_cast<long long>(cur.h) * p.g + r) * p.q_h;
+      if constexpr (!FP8) {
+        const uint32_t* qp =
+            reinterpret_cast<const uint32_t*>(static_cast<const uint16_t*>(p.q) + qoff);
+#pragma unroll
+        for (int ks = 0; ks < C::KS; ++ks) {
+          qb[ks][0] = row_ok ? __ldg(qp + (ks * 16 + 2 * c) / 2) : 0u;
+          qb[ks][1] = row_ok ? __ldg(qp + (ks * 16 + 8 + 2 * c) / 2) : 0u;
+        }
+      } else {
+        // k-slot order of the widened fp8 tile: slots 2c, 2c+1 <- dims 4c, 4c+1
+        // and slots 2c+8, 2c+9 <- dims 4c+2, 4c+3 of each 16-dim step.
+        const uint2* qp =
+            reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(p.q) + qoff);
+#pragma unroll
+        for (int ks = 0; ks < C::KS; ++ks) {
+          uint2 v = row_ok ? __ldg(qp + (ks * 16 + 4 * c) / 4) : make_uint2(0u, 0u);
+          float f0, f1, f2, f3;
+          if constexpr (QBF) {
+            f0 = __uint_as_float(v.x << 16);
+            f1 = __uint_as_float(v.x & 0xffff0000u);
+            f2 = __uint_as_float(v.y << 16);
+            f3 = __uint_as_float(v.y & 0xffff0000u);
+          } else {
+            __half2 a2 = *reinterpret_cast<__half2*>(&v.x);
+            __half2 b2 = *reinterpret_cast<__half2*>(&v.y);
+            f0 = __low2float(a2);
+            f1 = __high2float(a2);
+            f2 = __low2float(b2);
+            f3 = __high2float(b2);
+          }
+          qb[ks][0] = pack2<false>(f0, f1);
+          qb[ks][1] = pack2<false>(f2, f3);
+        }
+      }
+    };
+
+    auto finish_unit = [&]() {
+      // full row sums per head: reduce the thread partials over the 8 row groups
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+      }
+      float vs = 1.f;
+      if constexpr (FP8) vs = __ldg(p.v_scale + cur.h);
+      const long long ub = cur.unit_begin(), ue = cur.unit_end();
+      const int hq0 = cur.h * p.g + 2 * c;
+      if (ub >= lo && ue <= hi) {  // whole unit in this sub-range: final output
+        const float i0 = l0 > 0.f ? vs / l0 : 0.f;
+        const float i1 = l1 > 0.f ? vs / l1 : 0.f;
+        uint16_t* o = static_cast<uint16_t*>(p.out) + cur.s * p.o_s;
+#pragma unroll
+        for (int mt = 0; mt < C::MT; ++mt) {
+          const int da = FP8 ? 16 * mt + 2 * r : 16 * mt + r;
+          const int db = FP8 ? da + 1 : da + 8;
+          if (h0_ok) {
+            uint16_t* oh = o + hq0 * p.o_h;
+            const float x = acc[mt][0] * i0, y = acc[mt][2] * i0;
+            if constexpr (QBF) {
+              oh[da] = __bfloat16_as_ushort(__float2bfloat16_rn(x));
+              oh[db] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
+            } else {
+              oh[da] = __half_as_ushort(__float2half_rn(x));
+              oh[db] = __half_as_ushort(__float2half_rn(y));
+            }
+          }
+          if (h1_ok) {
+            uint16_t* oh = o + (hq0 + 1) * p.o_h;
+            const float x = acc[mt][1] * i1, y = acc[mt][3] * i1;
+            if constexpr (QBF) {
+              oh[da] = __bfloat16_as_ushort(__float2bfloat16_rn(x));
+              oh[db] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
+            } else {
+              oh[da] = __half_as_ushort(__float2half_rn(x));
+              oh[db] = __half_as_ushort(__float2half_rn(y));
+            }
+          }
+        }
+      } else {  // piece of a cut unit: fp32 partials for the merge kernel
+        const int slot = ub < lo ? 0 : 1;
+        const long long base = (slot_base + slot) * p.g;
+        float* po = p.part_o + base * D;
+#pragma unroll
+        for (int mt = 0; mt < C::MT; ++mt) {
+          const int da = FP8 ? 16 * mt + 2 * r : 16 * mt + r;
+          const int db = FP8 ? da + 1 : da + 8;
+          if (h0_ok) {
+            po[(2 * c) * D + da] = acc[mt][0] * vs;
+            po[(2 * c) * D + db] = acc[mt][2] * vs;
+          }
+          if (h1_ok) {
+            po[(2 * c + 1) * D + da] = acc[mt][1] * vs;
+            po[(2 * c + 1) * D + db] = acc[mt][3] * vs;
+          }
+        }
+        if (r == 0) {
+          float* pm = p.part_ml + base * 2;
+          if (h0_ok) {
+            pm[(2 * c) * 2 + 0] = m0;
+            pm[(2 * c) * 2 + 1] = l0;
+          }
+          if (h1_ok) {
+            pm[(2 * c + 1) * 2 + 0] = m1;
+            pm[(2 * c + 1) * 2 + 1] = l1;
+          }
+        }
+        if (slot == 1 && lane == 0)
+          p.desc[owner * (1 + kMaxSteals) + sub] =
+              make_int4(cur.s, cur.h, static_cast<int>(ue & 0xffffffffll),
+                        static_cast<int>(ue >> 32));
+      }
+    };
+
+    // ---- main loop over the sub-range ----
+    while (cur.k < hi) {
+      if (cur.b == 0 || cur.k == lo) begin_unit();
+      const int stage = static_cast<int>(it % NS);
+      const uint32_t parity = static_cast<uint32_t>((it / NS) & 1);
+      if (!warp_wait(my_bars + stage * 8, parity, kWaitNs)) {
+        if (lane == 0) atomicOr(p.err, kErrWaitTimeout);
+        for (long long j = it + 1; j < issued; ++j)  // let copies in flight land
+          warp_wait(my_bars + static_cast<int>(j % NS) * 8, static_cast<uint32_t>((j / NS) & 1),
+                    100000000ull);
+        return false;
+      }
+
+      if (cur.L > 0) {
+        const uint32_t tk = my_stages + stage * C::STAGE;
+        const uint32_t tv = tk + C::TILE;
+        const int nvalid = min(BS, cur.L - cur.b * BS);
+
+        // S^T = K Q^T
+        float sacc[C::TT][4];
+#pragma unroll
+        for (int tt = 0; tt < C::TT; ++tt) {
+          sacc[tt][0] = sacc[tt][1] = sacc[tt][2] = sacc[tt][3] = 0.f;
+          const int trow = tt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+          if constexpr (!FP8) {
+#pragma unroll
+            for (int ks = 0; ks < C::KS; ++ks) {
+              uint32_t a0, a1, a2, a3;
+              ldsm_x4(tk + swz<BS>(trow, ks * 32 + (lane >> 4) * 16), a0, a1, a2, a3);
+              mma16816<MBF>(sacc[tt], a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
+            }
+          } else {
+#pragma unroll
+            for (int kp = 0; kp < C::KS / 2; ++kp) {
+              uint32_t x0, x1, x2, x3;
+              ldsm_x4(tk + swz<BS>(trow, kp * 32 + (lane >> 4) * 16), x0, x1, x2, x3);
+              mma16816<false>(sacc[tt], e4m3x2_to_f16x2(x0 & 0xffff),
+                              e4m3x2_to_f16x2(x1 & 0xffff), e4m3x2_to_f16x2(x0 >> 16),
+                              e4m3x2_to_f16x2(x1 >> 16), qb[2 * kp][0], qb[2 * kp][1]);
+              mma16816<false>(sacc[tt], e4m3x2_to_f16x2(x2 & 0xffff),
+                              e4m3x2_to_f16x2(x3 & 0xffff), e4m3x2_to_f16x2(x2 >> 16),
+                              e4m3x2_to_f16x2(x3 >> 16), qb[2 * kp + 1][0], qb[2 * kp + 1][1]);
+            }
+          }
+        }
+
+        // online softmax over this block's tokens, per head column
+        float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+        for (int tt = 0; tt < C::TT; ++tt) {
+          const int t0 = tt * 16 + r, t1 = t0 + 8;
+          sacc[tt][0] = t0 < nvalid ? sacc[tt][0] * sl : -INFINITY;
+          sacc[tt][1] = t0 < nvalid ? sacc[tt][1] * sl : -INFINITY;
+          sacc[tt][2] = t1 < nvalid ? sacc[tt][2] * sl : -INFINITY;
+          sacc[tt][3] = t1 < nvalid ? sacc[tt][3] * sl : -INFINITY;
+          mx0 = fmaxf(mx0, fmaxf(sacc[tt][0], sacc[tt][2]));
+          mx1 = fmaxf(mx1, fmaxf(sacc[tt][1], sacc[tt][3]));
+        }
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+        }
+        const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);  // finite: nvalid >= 1
+        if (__any_sync(0xffffffffu, mn0 != m0 || mn1 != m1)) {   // a running max moved
+          const float al0 = exp2f(m0 - mn0), al1 = exp2f(m1 - mn1);
+          l0 *= al0;
+          l1 *= al1;
+#pragma unroll
+          for (int mt = 0; mt < C::MT; ++mt) {
+            acc[mt][0] *= al0;
+            acc[mt][1] *= al1;
+            acc[mt][2] *= al0;
+            acc[mt][3] *= al1;
+          }
+          m0 = mn0;
+          m1 = mn1;
+        }
+        uint32_t pb[C::TT][2];
+#pragma unroll
+        for (int tt = 0; tt < C::TT; ++tt) {
+          const float p0 = exp2f(sacc[tt][0] - m0), p1 = exp2f(sacc[tt][1] - m1);
+          const float p2 = exp2f(sacc[tt][2] - m0), p3 = exp2f(sacc[tt][3] - m1);
+          l0 += p0 + p2;
+          l1 += p1 + p3;
+          pb[tt][0] = movmatrix_t(pack2<MBF>(p0, p1));
+          pb[tt][1] = movmatrix_t(pack2<MBF>(p2, p3));
+        }
+
+        // O^T += V^T P^T; V entries of tokens past the context are zeroed
+        // (a NaN there times p = 0 would still be NaN).
+        auto pv = [&](auto masked) {
+          constexpr bool MASK = decltype(masked)::value;
+#pragma unroll
+          for (int tt = 0; tt < C::TT; ++tt) {
+            uint32_t keep01 = 0xffffffffu, keep23 = 0xffffffffu;
+            if constexpr (MASK) {
+              const int tb = tt * 16 + 2 * c;  // tokens of this thread's A halves
+              keep01 = (tb < nvalid ? 0x0000ffffu : 0u) | (tb + 1 < nvalid ? 0xffff0000u : 0u);
+              keep23 = (tb + 8 < nvalid ? 0x0000ffffu : 0u) | (tb + 9 < nvalid ? 0xffff0000u : 0u);
+            }
+            if constexpr (!FP8) {
+              const int vrow = tt * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
+#pragma unroll
+              for (int mt = 0; mt < C::MT; ++mt) {
+                uint32_t a0, a1, a2, a3;
+                ldsm_x4_t(tv + swz<BS>(vrow, mt * 32 + ((lane >> 3) & 1) * 16), a0, a1, a2, a3);
+                if constexpr (MASK) {
+                  a0 &= keep01;
+                  a1 &= keep01;
+                  a2 &= keep23;
+                  a3 &= keep23;
+                }
+                mma16816<MBF>(acc[mt], a0, a1, a2, a3, pb[tt][0], pb[tt][1]);
+              }
+            } else {
+              const int vrow = tt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+              for (int mp = 0; mp < C::MT / 2; ++mp) {
+                uint32_t x0, x1, x2, x3;
+                ldsm_x4_t(tv + swz<BS>(vrow, mp * 32 + (lane >> 4) * 16), x0, x1, x2, x3);
+                const uint32_t e0 = prmt(x0, 0, 0x3120), e1 = prmt(x1, 0, 0x3120);
+                const uint32_t e2 = prmt(x2, 0, 0x3120), e3 = prmt(x3, 0, 0x3120);
+                uint32_t f[8] = {e4m3x2_to_f16x2(e0 & 0xffff), e4m3x2_to_f16x2(e0 >> 16),
+                                 e4m3x2_to_f16x2(e1 & 0xffff), e4m3x2_to_f16x2(e1 >> 16),
+                                 e4m3x2_to_f16x2(e2 & 0xffff), e4m3x2_to_f16x2(e2 >> 16),
+                                 e4m3x2_to_f16x2(e3 & 0xffff), e4m3x2_to_f16x2(e3 >> 16)};
+                if constexpr (MASK) {
+                  f[0] &= keep01;
+                  f[1] &= keep01;
+                  f[2] &= keep23;
+                  f[3] &= keep23;
+                  f[4] &= keep01;
+                  f[5] &= keep01;
+                  f[6] &= keep23;
+                  f[7] &= keep23;
+                }
+                mma16816<false>(acc[2 * mp], f[0], f[1], f[2], f[3], pb[tt][0], pb[tt][1]);
+                mma16816<false>(acc[2 * mp + 1], f[4], f[5], f[6], f[7], pb[tt][0], pb[tt][1]);
+              }
+            }
+          }
+        };
+        if (nvalid == BS) pv(std::false_type{});
+        else pv(std::true_type{});
+      }
+
+      __syncwarp();
+      try_issue();  // refill the freed stage NS items ahead
+      if (cur.b == cur.n - 1 || cur.k == hi - 1) finish_unit();
+      cur.advance(p, max_len);
+      ++it;
     }
-    if (cur.b == cur.n - 1 || cur.k == hi - 1) finish_unit();
-    cur.advance(p, max_len);
-    ++it;
+    return true;
+  };
+
+  // ---- own range, then steal until no remainder is worth splitting ----
+  if (my_len > 0 && !run_range(my_lo, my_lo + my_len, true, gw, 0, 2ll * gw)) return;
+
+  const long long nominal = W / p.nwt;  // every static range is nominal or nominal + 1 long
+  for (int attempt = 0; attempt < 4 * kStealTries; ++attempt) {
+    // reserve two partial slots from the pool
+    unsigned slot0 = 0;
+    if (lane == 0) slot0 = atomicAdd(p.pool, 2u);
+    slot0 = __shfl_sync(0xffffffffu, slot0, 0);
+    if (slot0 + 2 > static_cast<unsigned>(p.pool_slots)) break;
+
+    // find the victim with the largest unclaimed remainder, steal its back half
+    int stolen = 0;
+    long long sa = 0, sb = 0;
+    int victim = -1, sj = 0;
+    for (int tries = 0; tries < kStealTries && !stolen; ++tries) {
+      long long best = 0;
+      int bv = -1;
+      unsigned long long bw = 0;
+      for (int v = lane; v < p.nwt; v += 32) {
+        const unsigned long long w = ld_relaxed(p.words + v);
+        const long long rem = rw_steals(w) >= kMaxSteals
+                                  ? 0
+                                  : nominal - static_cast<long long>(rw_front(w)) - rw_back(w);
+        if (rem > best) {
+          best = rem;
+          bv = v;
+          bw = w;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const long long ob = __shfl_xor_sync(0xffffffffu, best, o);
+        const int ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const unsigned long long ow = __shfl_xor_sync(0xffffffffu, bw, o);
+        if (ob > best || (ob == best && ov > bv)) {
+          best = ob;
+          bv = ov;
+          bw = ow;
+        }
+      }
+      if (best < kMinStealable) break;
+      if (lane == 0) {
+        const long long vlo = range_lo(bv, W, p.nwt);
+        const long long vlen = range_lo(bv + 1, W, p.nwt) - vlo;
+        const unsigned f = rw_front(bw), b = rw_back(bw), ns = rw_steals(bw);
+        const long long rem = vlen - static_cast<long long>(f) - b;
+        if (rem >= kMinStealable && ns < kMaxSteals) {
+          const unsigned take = static_cast<unsigned>(rem / 2);
+          const unsigned long long want = rw_make(f, b + take, ns + 1);
+          if (atomicCAS(p.words + bv, bw, want) == bw) {
+            stolen = 1;
+            sb = vlo + vlen - b;
+            sa = sb - take;
+            victim = bv;
+            sj = static_cast<int>(ns);
+            p.steal_info[bv * kMaxSteals + sj] =
+                make_int4(static_cast<int>(sa & 0xffffffffll), 2 * p.nwt + static_cast<int>(slot0),
+                          p.tag, static_cast<int>(sa >> 32));
+          }
+        }
+      }
+      stolen = __shfl_sync(0xffffffffu, stolen, 0);
+    }
+    if (!stolen) break;
+    sa = __shfl_sync(0xffffffffu, sa, 0);
+    sb = __shfl_sync(0xffffffffu, sb, 0);
+    victim = __shfl_sync(0xffffffffu, victim, 0);
+    sj = __shfl_sync(0xffffffffu, sj, 0);
+    if (!run_range(sa, sb, false, victim, sj + 1, 2ll * p.nwt + static_cast<long long>(slot0)))
+      return;
   }
 }
 
-// Combine the pieces of every unit cut by warp-range boundaries. One CTA per
-// warp of the decode grid; the CTA whose warp holds the first piece of a cut
-// unit (its slot-1 partial) merges it with the slot-0 partials of the
-// following warps whose ranges intersect the unit.
+// Combine the pieces of every unit cut by sub-range boundaries. One CTA per
+// static warp range w0 (all resident at once: few registers, small shared
+// memory), organised as a fixed number of memory rounds whose loads are all
+// independent: (1) the range's descriptors, steal records and the item count
+// together; (2) for each of its sub-ranges whose last piece starts a cut
+// unit, the steal records of the following static ranges, one range per
+// thread (the next 128, and so on), listing the piece slots of every
+// sub-range that starts before the unit's end (order does not matter to the
+// merge); (3) the pieces' running maxima per head; (4) the rescaled sums.
 template <bool QBF, int D>
-__global__ void __launch_bounds__(128) decode_merge_kernel(const __grid_constant__ DecodeParams p) {
-  const int gw = blockIdx.x;
-  const int4 d = p.desc[gw];
-  if (d.x < 0) return;
-  const int s = d.x, h = d.y;
-  const long long U1 = static_cast<long long>(static_cast<unsigned>(d.z)) |
-                       (static_cast<long long>(d.w) << 32);
-  const long long W = p.hdr[0];
+__global__ void __launch_bounds__(128, 8) decode_merge_kernel(const __grid_constant__ DecodeParams p) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the decode grid has finished
+  constexpr int NT = 128;
+  constexpr int kCap = 2048;  // pieces of one cut unit
+  constexpr int ND = 1 + kMaxSteals;
+  __shared__ int s_slot[kCap];
+  __shared__ int4 s_desc[ND];
+  __shared__ int4 s_rec[kMaxSteals];
+  __shared__ long long s_own_start[kMaxSteals];
+  __shared__ int s_own_slot[kMaxSteals];
+  __shared__ long long s_W;
+  __shared__ int s_n, s_m_own;
+
+  const int tid = threadIdx.x;
+  const int w0 = blockIdx.x;
   const int g = p.g;
-  for (int e = threadIdx.x; e < g * D; e += blockDim.x) {
-    const int i = e / D, dd = e % D;
-    // pass 1: running max over pieces
-    float mstar = -INFINITY;
-    for (int w = gw;; ++w) {
-      const long long lo = (static_cast<long long>(w) * W) / p.nwt;
-      if (w > gw && lo >= U1) break;
-      const long long hi = (static_cast<long long>(w + 1) * W) / p.nwt;
-      if (hi <= lo) continue;
-      const int slot = (w == gw) ? 1 : 0;
-      mstar = fmaxf(mstar, p.part_ml[((static_cast<long long>(w) * 2 + slot) * g + i) * 2]);
+  const int E = g * D;
+
+  // round 1: descriptors, own steal records, item count
+  if (tid < ND) s_desc[tid] = p.desc[w0 * ND + tid];
+  else if (tid >= 32 && tid < 32 + kMaxSteals) s_rec[tid - 32] = p.steal_info[w0 * kMaxSteals + tid - 32];
+  else if (tid == 64) s_W = p.hdr[0];
+  else if (tid == 96) {
+    p.words[w0] = 0ull;  // leave the claim state zeroed for the next call
+    if (w0 == 0) *p.pool = 0u;
+  }
+  __syncthreads();
+  const long long W = s_W;
+
+  // Steal records j = 0, 1, ... of warp v's range that carry this call's tag,
+  // each starting inside v's range with its slots in the pool.
+  auto valid_steals = [&](int v, const int4* rec, long long* starts, int* slots) -> int {
+    const long long vlo = range_lo(v, W, p.nwt), vhi = range_lo(v + 1, W, p.nwt);
+    int m = 0;
+    for (int j = 0; j < kMaxSteals; ++j) {
+      if (rec[j].z != p.tag) break;
+      const long long st = static_cast<long long>(static_cast<unsigned>(rec[j].x)) |
+                           (static_cast<long long>(rec[j].w) << 32);
+      if (st <= vlo || st >= vhi || rec[j].y < 2 * p.nwt ||
+          rec[j].y + 2 > 2 * p.nwt + p.pool_slots) {
+        atomicOr(p.err, kErrBadMerge);
+        break;
+      }
+      starts[j] = st;
+      slots[j] = rec[j].y;
+      m = j + 1;
     }
-    float lsum = 0.f, osum = 0.f;
-    for (int w = gw;; ++w) {
-      const long long lo = (static_cast<long long>(w) * W) / p.nwt;
-      if (w > gw && lo >= U1) break;
-      const long long hi = (static_cast<long long>(w + 1) * W) / p.nwt;
-      if (hi <= lo) continue;
-      const int slot = (w == gw) ? 1 : 0;
-      const long long base = (static_cast<long long>(w) * 2 + slot) * g + i;
-      const float mp = p.part_ml[base * 2];
-      const float sc = (mp == -INFINITY) ? 0.f : exp2f(mp - mstar);
-      lsum += p.part_ml[base * 2 + 1] * sc;
-      osum += p.part_o[base * D + dd] * sc;
+    return m;
+  };
+
+  if (tid == 0) s_m_own = valid_steals(w0, s_rec, s_own_start, s_own_slot);
+  __syncthreads();
+  const int m_own = s_m_own;
+
+  for (int k = 0; k <= m_own; ++k) {
+    const int4 d = s_desc[k];
+    if (d.x < 0) continue;
+    const int s = d.x, h = d.y;
+    const long long U1 = static_cast<long long>(static_cast<unsigned>(d.z)) |
+                         (static_cast<long long>(d.w) << 32);
+    if (s >= p.S || h < 0 || h >= p.Hk || U1 <= 0 || U1 > W) {
+      if (tid == 0) atomicOr(p.err, kErrBadMerge);
+      continue;
     }
-    const float v = lsum > 0.f ? osum / lsum : 0.f;
-    uint16_t* o = static_cast<uint16_t*>(p.out) + s * p.o_s + (static_cast<long long>(h) * g + i) * p.o_h;
-    if constexpr (QBF) o[dd] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
-    else o[dd] = __half_as_ushort(__float2half_rn(v));
+    // item-order position of this sub-range in w0's list: 0 = owner part,
+    // i >= 1 = steal (m - i)
+    const int pos0 = (k == 0) ? 0 : m_own - (k - 1);
+    if (tid == 0) {
+      s_n = 1;
+      s_slot[0] = ((k == 0) ? 2 * w0 : s_own_slot[k - 1]) + 1;
+    }
+    __syncthreads();
+    // round 2: the pieces of the sub-ranges after this one that start before U1
+    for (int chunk = 0;; ++chunk) {
+      const int v = w0 + chunk * NT + tid;
+      if (v < p.nwt && range_lo(v, W, p.nwt) < U1) {
+        long long st_v[kMaxSteals];
+        int sl_v[kMaxSteals];
+        int m;
+        if (v == w0) {
+          m = m_own;
+          for (int j = 0; j < m; ++j) {
+            st_v[j] = s_own_start[j];
+            sl_v[j] = s_own_slot[j];
+          }
+        } else {
+          int4 rec[kMaxSteals];
+#pragma unroll
+          for (int j = 0; j < kMaxSteals; ++j) rec[j] = p.steal_info[v * kMaxSteals + j];
+          m = valid_steals(v, rec, st_v, sl_v);
+        }
+        const long long vlo = range_lo(v, W, p.nwt), vhi = range_lo(v + 1, W, p.nwt);
+        for (int pos = (v == w0) ? pos0 + 1 : 0; pos <= m; ++pos) {
+          const long long st = pos == 0 ? vlo : st_v[m - pos];
+          const long long en = pos < m ? st_v[m - pos - 1] : vhi;
+          if (st >= U1) break;
+          if (en > st) {
+            const int idx = atomicAdd(&s_n, 1);
+            if (idx < kCap) s_slot[idx] = pos == 0 ? 2 * v : sl_v[m - pos];
+          }
+        }
+      }
+      const long long next = w0 + static_cast<long long>(chunk + 1) * NT;
+      if (next >= p.nwt || range_lo(next, W, p.nwt) >= U1) break;
+    }
+    __syncthreads();
+    const int n = s_n;
+    if (n > kCap) {
+      if (tid == 0) atomicOr(p.err, kErrBadMerge);
+      __syncthreads();
+      continue;
+    }
+    // round 3: fold the pieces in. Thread t owns an 8-element chunk of one
+    // head (chunk t % NC8) and the pieces q = t / NC8 (mod PG); it loads four
+    // pieces at a time (m, l and two float4 of O each) before folding them
+    // with an online max / rescale, then the piece groups are combined.
+    const int NC8 = E / 8;                // chunks of 8 elements (D is a multiple of 8)
+    const int PG = NT / NC8;              // piece groups (1 at g = 8, D = 128)
+    const int c8 = tid % NC8, pg = tid / NC8;
+    const int hi8 = c8 / (D / 8), d8 = (c8 % (D / 8)) * 8;
+    float rm = -INFINITY, rl = 0.f, ra[8];
+#pragma unroll
+    for (int x = 0; x < 8; ++x) ra[x] = 0.f;
+    if (pg < PG) {
+      for (int q0 = pg; q0 < n; q0 += 4 * PG) {
+        float mv[4], lv[4];
+        float4 o0[4], o1[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int q = q0 + u * PG;
+          mv[u] = -INFINITY;
+          lv[u] = 0.f;
+          o0[u] = o1[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (q < n) {
+            const long long base = static_cast<long long>(s_slot[q]) * g + hi8;
+            mv[u] = p.part_ml[base * 2];
+            lv[u] = p.part_ml[base * 2 + 1];
+            const float4* op = reinterpret_cast<const float4*>(p.part_o + base * D + d8);
+            o0[u] = op[0];
+            o1[u] = op[1];
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (mv[u] == -INFINITY) continue;
+          const float mn = fmaxf(rm, mv[u]);
+          const float sa = (rm == -INFINITY) ? 0.f : exp2f(rm - mn), sb = exp2f(mv[u] - mn);
+          rl = rl * sa + lv[u] * sb;
+          ra[0] = ra[0] * sa + o0[u].x * sb;
+          ra[1] = ra[1] * sa + o0[u].y * sb;
+          ra[2] = ra[2] * sa + o0[u].z * sb;
+          ra[3] = ra[3] * sa + o0[u].w * sb;
+          ra[4] = ra[4] * sa + o1[u].x * sb;
+          ra[5] = ra[5] * sa + o1[u].y * sb;
+          ra[6] = ra[6] * sa + o1[u].z * sb;
+          ra[7] = ra[7] * sa + o1[u].w * sb;
+          rm = mn;
+        }
+      }
+    }
+    // combine the piece groups of each chunk (through the now unused list)
+    if (PG > 1) {
+      float* red = reinterpret_cast<float*>(s_slot);  // [NT][10]
+      __syncthreads();
+      red[tid * 10 + 0] = rm;
+      red[tid * 10 + 1] = rl;
+#pragma unroll
+      for (int x = 0; x < 8; ++x) red[tid * 10 + 2 + x] = ra[x];
+      __syncthreads();
+      if (pg == 0) {
+        for (int gq = 1; gq < PG; ++gq) {
+          const float* r2 = red + (gq * NC8 + c8) * 10;
+          const float m2 = r2[0];
+          if (m2 == -INFINITY) continue;
+          const float mn = fmaxf(rm, m2);
+          const float sa = (rm == -INFINITY) ? 0.f : exp2f(rm - mn), sb = exp2f(m2 - mn);
+          rl = rl * sa + r2[1] * sb;
+#pragma unroll
+          for (int x = 0; x < 8; ++x) ra[x] = ra[x] * sa + r2[2 + x] * sb;
+          rm = mn;
+        }
+      }
+    }
+    if (pg == 0) {
+      const float inv = rl > 0.f ? 1.f / rl : 0.f;
+      uint16_t* oh = static_cast<uint16_t*>(p.out) + s * p.o_s +
+                     (static_cast<long long>(h) * g + hi8) * p.o_h + d8;
+      uint32_t w4[4];
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        if constexpr (QBF) {
+          __nv_bfloat162 v2 = __floats2bfloat162_rn(ra[2 * x] * inv, ra[2 * x + 1] * inv);
+          w4[x] = *reinterpret_cast<uint32_t*>(&v2);
+        } else {
+          __half2 v2 = __floats2half2_rn(ra[2 * x] * inv, ra[2 * x + 1] * inv);
+          w4[x] = *reinterpret_cast<uint32_t*>(&v2);
+        }
+      }
+      if ((reinterpret_cast<uintptr_t>(oh) & 15) == 0) {
+        *reinterpret_cast<uint4*>(oh) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+      } else {
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+          oh[2 * x] = static_cast<uint16_t>(w4[x] & 0xffffu);
+          oh[2 * x + 1] = static_cast<uint16_t>(w4[x] >> 16);
+        }
+      }
+    }
+    __syncthreads();  // s_slot / s_n are reused by the next cut unit
   }
 }
 

@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -213,18 +214,65 @@ int decode_grid(DecodeLaunch* e, int dev, int sms, int* grid) {
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Decode workspace: header (total items, steal-slot pool counter), range
+// words, steal records, last-piece descriptors, and fp32 partial slots (two
+// per warp for its own range, `pool` more for steals). The range words and
+// the pool counter must be zero before a call (every call leaves them zero
+// again) and steal records are recognised by the call's tag, so these
+// regions sit at the same offsets, with the same sizes, for every kernel
+// configuration (sized for kWordsPerSM warps per SM, more than any
+// configuration has): no configuration's scratch ever lands in another's
+// claim state or steal records.
+constexpr int kWordsPerSM = 16;
+
 struct WsLayout {
-  size_t hdr, desc, part_o, part_ml, total;
+  size_t hdr, pool, words, steal, desc, part_o, part_ml, total;
+  int pool_slots;
 };
 
-WsLayout ws_layout(int nwt, int g, int D) {
+size_t slot_bytes(int g, int D) { return static_cast<size_t>(g) * (D + 2) * 4; }
+
+WsLayout ws_layout(int sms, int nwt, int g, int D, int pool_slots) {
   WsLayout l;
   l.hdr = 0;
-  l.desc = 256;
-  l.part_o = round_up(l.desc + static_cast<size_t>(nwt) * 16, 256);
-  l.part_ml = round_up(l.part_o + static_cast<size_t>(nwt) * 2 * g * D * 4, 256);
-  l.total = round_up(l.part_ml + static_cast<size_t>(nwt) * 2 * g * 2 * 4, 256);
+  l.pool = 64;
+  l.words = 256;
+  size_t cap = static_cast<size_t>(kWordsPerSM) * sms;
+  if (cap < static_cast<size_t>(nwt)) cap = nwt;
+  l.steal = round_up(l.words + cap * 8, 256);
+  l.desc = round_up(l.steal + cap * kMaxSteals * 16, 256);
+  l.part_o = round_up(l.desc + cap * (1 + kMaxSteals) * 16, 256);
+  const size_t slots = 2 * static_cast<size_t>(nwt) + pool_slots;
+  l.part_ml = round_up(l.part_o + slots * g * D * 4, 256);
+  l.total = round_up(l.part_ml + slots * g * 2 * 4, 256);
+  l.pool_slots = pool_slots;
   return l;
+}
+
+// Default: room for one steal per warp.
+WsLayout ws_default(int sms, int nwt, int g, int D) {
+  return ws_layout(sms, nwt, g, D, 2 * nwt);
+}
+
+// The largest layout that fits in `bytes` (fewer steal slots), or one whose
+// total exceeds `bytes` when even no steal slots fit.
+WsLayout ws_fit(int sms, int nwt, int g, int D, size_t bytes) {
+  const WsLayout full = ws_default(sms, nwt, g, D);
+  if (full.total <= bytes) return full;
+  const WsLayout base = ws_layout(sms, nwt, g, D, 0);
+  if (base.total > bytes) return base;
+  int pool = static_cast<int>((bytes - base.total) / slot_bytes(g, D)) & ~1;
+  while (pool > 0 && ws_layout(sms, nwt, g, D, pool).total > bytes) pool -= 2;
+  return ws_layout(sms, nwt, g, D, pool);
+}
+
+std::atomic<unsigned> g_call_tag{1};
+
+int next_tag() {
+  for (;;) {
+    const unsigned t = g_call_tag.fetch_add(1);
+    if (static_cast<int>(t) != 0) return static_cast<int>(t);
+  }
 }
 
 struct DecodeArgs {
@@ -278,8 +326,12 @@ int check_decode(const DecodeArgs& a, bool fp8, int* ck_out, DecodeLaunch** entr
   return *entry ? PKV_OK : PKV_ERR_UNSUPPORTED;
 }
 
+// Launch decode + merge. lib_ws: use (and grow) the library's workspace for
+// this device; otherwise `ws` is the caller's. fit: shrink the steal-slot pool
+// to fit ws_bytes; clear: zero the claim state first (callers that cannot
+// vouch for it).
 int launch_decode(const DecodeArgs& a, bool fp8, void* ws, size_t ws_bytes, bool lib_ws,
-                  cudaStream_t stream) {
+                  cudaStream_t stream, bool fit = false, bool clear = false) {
   int ck = 0;
   DecodeLaunch* e = nullptr;
   int st = check_decode(a, fp8, &ck, &e);
@@ -293,7 +345,8 @@ int launch_decode(const DecodeArgs& a, bool fp8, void* ws, size_t ws_bytes, bool
   const int nwt = grid * e->nc;
   const int g = static_cast<int>(a.q->shape[1] / a.Hk);
   const int D = static_cast<int>(a.q->shape[2]);
-  const WsLayout L = ws_layout(nwt, g, D);
+  if (nwt > kWordsPerSM * ds->sms) return PKV_ERR_UNSUPPORTED;
+  const WsLayout L = fit ? ws_fit(ds->sms, nwt, g, D, ws_bytes) : ws_default(ds->sms, nwt, g, D);
   if (lib_ws) {
     std::lock_guard<std::mutex> lk(g_mu);
     if (ds->ws_bytes < L.total) {
@@ -301,12 +354,14 @@ int launch_decode(const DecodeArgs& a, bool fp8, void* ws, size_t ws_bytes, bool
       ds->ws = nullptr;
       ds->ws_bytes = 0;
       if (cudaMalloc(&ds->ws, L.total) != cudaSuccess) return PKV_ERR_CUDA;
+      if (cudaMemset(ds->ws, 0, L.total) != cudaSuccess) return PKV_ERR_CUDA;
       ds->ws_bytes = L.total;
     }
     ws = ds->ws;
     ws_bytes = ds->ws_bytes;
   }
   if (!ws || ws_bytes < L.total || !aligned(ws, 16)) return PKV_ERR_WORKSPACE;
+  if (clear && cudaMemsetAsync(ws, 0, L.steal, stream) != cudaSuccess) return PKV_ERR_CUDA;
 
   DecodeParams p;
   std::memset(&p, 0, sizeof(p));
@@ -331,17 +386,34 @@ int launch_decode(const DecodeArgs& a, bool fp8, void* ws, size_t ws_bytes, bool
   p.MB = static_cast<int>(a.bt->shape[1]);
   p.NB = static_cast<int>(a.kc->shape[0]);
   p.nwt = nwt;
+  p.tag = next_tag();
+  p.pool_slots = L.pool_slots;
   uint8_t* w = static_cast<uint8_t*>(ws);
   p.hdr = reinterpret_cast<long long*>(w + L.hdr);
   p.err = ds->err;
+  p.words = reinterpret_cast<unsigned long long*>(w + L.words);
+  p.pool = reinterpret_cast<unsigned*>(w + L.pool);
+  p.steal_info = reinterpret_cast<int4*>(w + L.steal);
+  p.desc = reinterpret_cast<int4*>(w + L.desc);
   p.part_o = reinterpret_cast<float*>(w + L.part_o);
   p.part_ml = reinterpret_cast<float*>(w + L.part_ml);
-  p.desc = reinterpret_cast<int4*>(w + L.desc);
 
   e->kernel<<<grid, e->threads, e->smem, stream>>>(p);
   if (cudaGetLastError() != cudaSuccess) return PKV_ERR_CUDA;
-  e->merge<<<nwt, 128, 0, stream>>>(p);
-  if (cudaGetLastError() != cudaSuccess) return PKV_ERR_CUDA;
+  // The merge kernel is launched as a programmatic dependent of the decode
+  // kernel: its CTAs can be resident before the decode grid ends and start
+  // the moment it has (griddepcontrol.wait), hiding the launch gap.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(nwt));
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, e->merge, p) != cudaSuccess) return PKV_ERR_CUDA;
   return PKV_OK;
 }
 
@@ -504,7 +576,7 @@ size_t paged_attn_decode_workspace_bytes(int num_q_heads, int num_kv_heads, int 
   int grid = 0;
   size_t bytes = 0;
   if (device_state(device, &ds) == PKV_OK && decode_grid(e, device, ds->sms, &grid) == PKV_OK)
-    bytes = ws_layout(grid * e->nc, num_q_heads / num_kv_heads, head_dim).total;
+    bytes = ws_default(ds->sms, grid * e->nc, num_q_heads / num_kv_heads, head_dim).total;
   if (prev != device) cudaSetDevice(prev);
   return bytes;
 }
@@ -543,12 +615,15 @@ int paged_attn_decode_noalloc(const pkv_tensor* q, const pkv_tensor* k_cache,
   int grid;
   if ((st = decode_grid(e, dev, ds->sms, &grid)) != PKV_OK) return st;
   const int g = static_cast<int>(q->shape[1] / num_kv_heads);
-  const size_t need = ws_layout(grid * e->nc, g, static_cast<int>(q->shape[2])).total;
+  const size_t need =
+      ws_fit(ds->sms, grid * e->nc, g, static_cast<int>(q->shape[2]), PKV_NOALLOC_SCRATCH_BYTES)
+          .total;
   if (need > PKV_NOALLOC_SCRATCH_BYTES) return PKV_ERR_SCRATCH_LIMIT;
   void* scratch = nullptr;
   if ((st = noalloc_scratch(dev, &scratch)) != PKV_OK) return st;
+  // The scratch keeps the previous call's contents: clear the claim state.
   return launch_decode(a, fp8, scratch, PKV_NOALLOC_SCRATCH_BYTES, false,
-                       static_cast<cudaStream_t>(stream));
+                       static_cast<cudaStream_t>(stream), true, true);
 }
 
 int reshape_and_cache(const pkv_tensor* k, const pkv_tensor* v, pkv_tensor* k_cache,

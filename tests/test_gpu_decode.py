@@ -85,17 +85,19 @@ def test_one_token_context_returns_v0_exactly():
     check_no_device_error()
 
 
-def test_deterministic_and_explicit_workspace():
+def test_repeated_calls_and_explicit_workspace():
+    # Work is rebalanced between warps at run time, so repeated calls may cut
+    # units differently (last-bit differences); each result meets the tolerance.
     s, lay, t = decode_case(W.scaled_down(W.spec("long_skewed"), 16, 3000))
-    a = run_decode(s, lay, t)
-    b = run_decode(s, lay, t)
+    ref = oracle_decode(s, lay, t)
     nbytes = P.workspace_bytes(s.num_q_heads, s.num_kv_heads, s.head_dim, s.block_size, P.PKV_BF16,
                                torch.cuda.current_device())
     assert nbytes > 0
-    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
-    c = run_decode(s, lay, t, workspace=ws)
-    torch.cuda.synchronize()
-    assert torch.equal(a, b) and torch.equal(a, c)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    for i in range(6):
+        out = run_decode(s, lay, t, workspace=ws if i % 2 else None)
+        torch.cuda.synchronize()
+        assert max_err(out, ref) <= TOL[s.cache_dtype], i
     with pytest.raises(P.PkvError) as e:
         run_decode(s, lay, t, workspace=ws[: nbytes // 2])
     assert e.value.status == P.PKV_ERR_WORKSPACE
@@ -168,3 +170,22 @@ def test_decode_full_size_sampled(name, over):
     assert err <= TOL[s.cache_dtype], (name, over, err)
     # every other row is finite and bounded by the largest |v| of the pool
     assert torch.isfinite(out).all()
+
+
+def test_one_workspace_shared_by_configurations():
+    # Kernel configurations differ in grid size (one or two CTAs per SM); the
+    # work-claiming state of one must not be disturbed by another's scratch.
+    cases = [decode_case(SMALL[n], seed=SMALL[n].seed + 7)
+             for n in ("skewed_b32", "8b_small", "d64_f16_b16_g1", "skewed_fp8_b16", "tiny")]
+    dev = torch.cuda.current_device()
+    code = {"bf16": P.PKV_BF16, "f16": P.PKV_F16, "fp8_e4m3": P.PKV_FP8_E4M3}
+    nbytes = max(P.workspace_bytes(s.num_q_heads, s.num_kv_heads, s.head_dim, s.block_size,
+                                   code[s.cache_dtype], dev) for s, _, _ in cases)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    refs = [oracle_decode(*c) for c in cases]
+    for rnd in range(3):
+        for (s, lay, t), ref in zip(cases, refs):
+            out = run_decode(s, lay, t, workspace=ws)
+            torch.cuda.synchronize()
+            assert max_err(out, ref) <= TOL[s.cache_dtype], (rnd, s.name)
+    check_no_device_error()
