@@ -182,7 +182,7 @@ __device__ __forceinline__ uint32_t swz(int t, int bcol) {
 }
 
 template <int CK, bool QBF, int D, int BS, int NC, int NS>
-__global__ void __launch_bounds__(NC * 32) decode_kernel(const __grid_constant__ DecodeParams p) {
+__global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
   using C = DecodeCfg<CK, QBF, D, BS, NC, NS>;
   constexpr bool FP8 = C::kFp8;
   constexpr bool MBF = C::kMmaBF16;
@@ -530,10 +530,18 @@ __global__ void __launch_bounds__(NC * 32) decode_kernel(const __grid_constant__
         return false;
       }
 
+      bool refilled = false;
       if (cur.L > 0) {
         const uint32_t tk = my_stages + stage * C::STAGE;
         const uint32_t tv = tk + C::TILE;
         const int nvalid = min(BS, cur.L - cur.b * BS);
+        // 16-token blocks: the V fragments go to registers right after QK^T
+        // (the MMAs consume the K fragments, the context mask consumes the V
+        // fragments), so the stage is refilled before the softmax and PV and
+        // stays in flight for longer.
+        constexpr bool kEarly = (C::TT == 1);
+        constexpr int VF = FP8 ? C::MT / 2 : C::MT;  // ldmatrix.x4 of one V tile
+        uint32_t vf[kEarly ? VF : 1][FP8 ? 8 : 4];
 
         // S^T = K Q^T
         float sacc[C::TT][4];
@@ -561,6 +569,46 @@ __global__ void __launch_bounds__(NC * 32) decode_kernel(const __grid_constant__
                               e4m3x2_to_f16x2(x3 >> 16), qb[2 * kp + 1][0], qb[2 * kp + 1][1]);
             }
           }
+        }
+
+        // V fragments of tile tt (rows tt*16..), tokens past the context
+        // zeroed (a NaN there times p = 0 would still be NaN). Non-fp8: four
+        // A registers per m-tile; fp8: eight (two m-tiles), widened to f16.
+        auto load_v = [&](int tt, int i, uint32_t* f) {
+          const int tb = tt * 16 + 2 * c;  // tokens of this thread's A halves
+          const uint32_t keep01 =
+              (tb < nvalid ? 0x0000ffffu : 0u) | (tb + 1 < nvalid ? 0xffff0000u : 0u);
+          const uint32_t keep23 =
+              (tb + 8 < nvalid ? 0x0000ffffu : 0u) | (tb + 9 < nvalid ? 0xffff0000u : 0u);
+          if constexpr (!FP8) {
+            const int vrow = tt * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
+            ldsm_x4_t(tv + swz<BS>(vrow, i * 32 + ((lane >> 3) & 1) * 16), f[0], f[1], f[2], f[3]);
+            f[0] &= keep01;
+            f[1] &= keep01;
+            f[2] &= keep23;
+            f[3] &= keep23;
+          } else {
+            const int vrow = tt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+            uint32_t x0, x1, x2, x3;
+            ldsm_x4_t(tv + swz<BS>(vrow, i * 32 + (lane >> 4) * 16), x0, x1, x2, x3);
+            const uint32_t e0 = prmt(x0, 0, 0x3120), e1 = prmt(x1, 0, 0x3120);
+            const uint32_t e2 = prmt(x2, 0, 0x3120), e3 = prmt(x3, 0, 0x3120);
+            f[0] = e4m3x2_to_f16x2(e0 & 0xffff) & keep01;
+            f[1] = e4m3x2_to_f16x2(e0 >> 16) & keep01;
+            f[2] = e4m3x2_to_f16x2(e1 & 0xffff) & keep23;
+            f[3] = e4m3x2_to_f16x2(e1 >> 16) & keep23;
+            f[4] = e4m3x2_to_f16x2(e2 & 0xffff) & keep01;
+            f[5] = e4m3x2_to_f16x2(e2 >> 16) & keep01;
+            f[6] = e4m3x2_to_f16x2(e3 & 0xffff) & keep23;
+            f[7] = e4m3x2_to_f16x2(e3 >> 16) & keep23;
+          }
+        };
+        if constexpr (kEarly) {
+#pragma unroll
+          for (int i = 0; i < VF; ++i) load_v(0, i, vf[i]);
+          __syncwarp();
+          try_issue();  // every read of this stage has completed: refill it
+          refilled = true;
         }
 
         // online softmax over this block's tokens, per head column
@@ -606,66 +654,29 @@ __global__ void __launch_bounds__(NC * 32) decode_kernel(const __grid_constant__
           pb[tt][1] = movmatrix_t(pack2<MBF>(p2, p3));
         }
 
-        // O^T += V^T P^T; V entries of tokens past the context are zeroed
-        // (a NaN there times p = 0 would still be NaN).
-        auto pv = [&](auto masked) {
-          constexpr bool MASK = decltype(masked)::value;
+        // O^T += V^T P^T
 #pragma unroll
-          for (int tt = 0; tt < C::TT; ++tt) {
-            uint32_t keep01 = 0xffffffffu, keep23 = 0xffffffffu;
-            if constexpr (MASK) {
-              const int tb = tt * 16 + 2 * c;  // tokens of this thread's A halves
-              keep01 = (tb < nvalid ? 0x0000ffffu : 0u) | (tb + 1 < nvalid ? 0xffff0000u : 0u);
-              keep23 = (tb + 8 < nvalid ? 0x0000ffffu : 0u) | (tb + 9 < nvalid ? 0xffff0000u : 0u);
-            }
+        for (int tt = 0; tt < C::TT; ++tt) {
+#pragma unroll
+          for (int i = 0; i < VF; ++i) {
+            uint32_t fl[FP8 ? 8 : 4];
+            const uint32_t* f = fl;
+            if constexpr (kEarly) f = vf[i];
+            else load_v(tt, i, fl);
             if constexpr (!FP8) {
-              const int vrow = tt * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
-#pragma unroll
-              for (int mt = 0; mt < C::MT; ++mt) {
-                uint32_t a0, a1, a2, a3;
-                ldsm_x4_t(tv + swz<BS>(vrow, mt * 32 + ((lane >> 3) & 1) * 16), a0, a1, a2, a3);
-                if constexpr (MASK) {
-                  a0 &= keep01;
-                  a1 &= keep01;
-                  a2 &= keep23;
-                  a3 &= keep23;
-                }
-                mma16816<MBF>(acc[mt], a0, a1, a2, a3, pb[tt][0], pb[tt][1]);
-              }
+              mma16816<MBF>(acc[i], f[0], f[1], f[2], f[3], pb[tt][0], pb[tt][1]);
             } else {
-              const int vrow = tt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-#pragma unroll
-              for (int mp = 0; mp < C::MT / 2; ++mp) {
-                uint32_t x0, x1, x2, x3;
-                ldsm_x4_t(tv + swz<BS>(vrow, mp * 32 + (lane >> 4) * 16), x0, x1, x2, x3);
-                const uint32_t e0 = prmt(x0, 0, 0x3120), e1 = prmt(x1, 0, 0x3120);
-                const uint32_t e2 = prmt(x2, 0, 0x3120), e3 = prmt(x3, 0, 0x3120);
-                uint32_t f[8] = {e4m3x2_to_f16x2(e0 & 0xffff), e4m3x2_to_f16x2(e0 >> 16),
-                                 e4m3x2_to_f16x2(e1 & 0xffff), e4m3x2_to_f16x2(e1 >> 16),
-                                 e4m3x2_to_f16x2(e2 & 0xffff), e4m3x2_to_f16x2(e2 >> 16),
-                                 e4m3x2_to_f16x2(e3 & 0xffff), e4m3x2_to_f16x2(e3 >> 16)};
-                if constexpr (MASK) {
-                  f[0] &= keep01;
-                  f[1] &= keep01;
-                  f[2] &= keep23;
-                  f[3] &= keep23;
-                  f[4] &= keep01;
-                  f[5] &= keep01;
-                  f[6] &= keep23;
-                  f[7] &= keep23;
-                }
-                mma16816<false>(acc[2 * mp], f[0], f[1], f[2], f[3], pb[tt][0], pb[tt][1]);
-                mma16816<false>(acc[2 * mp + 1], f[4], f[5], f[6], f[7], pb[tt][0], pb[tt][1]);
-              }
+              mma16816<false>(acc[2 * i], f[0], f[1], f[2], f[3], pb[tt][0], pb[tt][1]);
+              mma16816<false>(acc[2 * i + 1], f[4], f[5], f[6], f[7], pb[tt][0], pb[tt][1]);
             }
           }
-        };
-        if (nvalid == BS) pv(std::false_type{});
-        else pv(std::true_type{});
+        }
       }
 
-      __syncwarp();
-      try_issue();  // refill the freed stage NS items ahead
+      if (!refilled) {
+        __syncwarp();
+        try_issue();  // refill the freed stage NS items ahead
+      }
       if (cur.b == cur.n - 1 || cur.k == hi - 1) finish_unit();
       cur.advance(p, max_len);
       ++it;
