@@ -36,6 +36,7 @@ struct CacheParams {
 
 // 16-bit pools: a plain 16-byte copy per thread.
 __global__ void reshape_and_cache_kernel(const __grid_constant__ CacheParams p, int* err) {
+  pdl_launch_dependents();  // a decode launched after this may start its prologue
   const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const long long per_tok = static_cast<long long>(p.Hk) * p.row_vecs;
   if (i >= per_tok * p.T) return;
@@ -104,6 +105,7 @@ __device__ __forceinline__ uint4 quantise16(const int4& a, const int4& b, float 
 
 template <bool BF16>
 __global__ void reshape_and_cache_fp8_kernel(const __grid_constant__ CacheParams p, int* err) {
+  pdl_launch_dependents();
   const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const long long per_tok = static_cast<long long>(p.Hk) * p.row_vecs;
   if (i >= per_tok * p.T) return;

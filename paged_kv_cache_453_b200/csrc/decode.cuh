@@ -205,7 +205,7 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
   const int max_len = p.MB * BS;
 
   // The merge kernel may be scheduled now; it waits for this grid to finish.
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  pdl_launch_dependents();
 
   if (lane == 0) {
     for (int i = 0; i < NS; ++i) mbar_init(bars + (warp * NS + i) * 8, 1);
@@ -215,6 +215,10 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
     tma_prefetch_desc(&p.tmv);
   }
   fence_mbar_init();
+  // This grid may have started before the previous kernel in the stream
+  // finished (programmatic dependent launch): nothing above touches global
+  // memory; everything below may.
+  pdl_wait();
 
   // ---- total work and each thread's chunk prefix (every CTA, redundantly) ----
   {
@@ -337,6 +341,7 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
     }
     Cursor<BS> pc = cur;
     const long long lo = a;
+
     unsigned long long* wp = p.words + owner;
     const unsigned own_len = static_cast<unsigned>(hi - a);
     bool claiming = claim;
@@ -769,7 +774,8 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
 // merge); (3) the pieces' running maxima per head; (4) the rescaled sums.
 template <bool QBF, int D>
 __global__ void __launch_bounds__(128, 8) decode_merge_kernel(const __grid_constant__ DecodeParams p) {
-  asm volatile("griddepcontrol.wait;" ::: "memory");  // the decode grid has finished
+  pdl_wait();  // the decode grid has finished
+  pdl_launch_dependents();
   constexpr int NT = 128;
   constexpr int kCap = 2048;  // pieces of one cut unit
   constexpr int ND = 1 + kMaxSteals;

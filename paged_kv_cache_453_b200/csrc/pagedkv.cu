@@ -168,18 +168,21 @@ DecodeLaunch* decode_entry() {
   return &e;
 }
 
-// Stage counts: about 96 KB of ring per 4-warp CTA (two CTAs per SM) where
-// a stage is 8 KB or less; 32-token 16-bit blocks use three 16 KB stages
-// per warp (one CTA per SM).
+// Warps per CTA (NC) and ring stages per warp (NS), measured on B200. Two
+// CTAs of ~96 KB share an SM where a stage is 8 KB or less: 16-bit, D = 128,
+// 16-token blocks do best with 3 warps x 4 stages (deeper per-warp rings);
+// 4 KB stages (fp8, D = 64) with 4 warps x 6 stages (more math per byte
+// wants more warps); 32-token 16-bit blocks use 4 warps x 3 stages of 16 KB
+// (one CTA per SM).
 DecodeLaunch* pick_decode(int ck, bool qbf, int D, int BS) {
   constexpr int NC = 4;
   if (ck == kCacheBF16) {
-    if (D == 128 && BS == 16) return decode_entry<kCacheBF16, true, 128, 16, NC, 3>();
+    if (D == 128 && BS == 16) return decode_entry<kCacheBF16, true, 128, 16, 3, 4>();
     if (D == 128 && BS == 32) return decode_entry<kCacheBF16, true, 128, 32, NC, 3>();
     if (D == 64 && BS == 16) return decode_entry<kCacheBF16, true, 64, 16, NC, 6>();
     if (D == 64 && BS == 32) return decode_entry<kCacheBF16, true, 64, 32, NC, 3>();
   } else if (ck == kCacheF16) {
-    if (D == 128 && BS == 16) return decode_entry<kCacheF16, false, 128, 16, NC, 3>();
+    if (D == 128 && BS == 16) return decode_entry<kCacheF16, false, 128, 16, 3, 4>();
     if (D == 128 && BS == 32) return decode_entry<kCacheF16, false, 128, 32, NC, 3>();
     if (D == 64 && BS == 16) return decode_entry<kCacheF16, false, 64, 16, NC, 6>();
     if (D == 64 && BS == 32) return decode_entry<kCacheF16, false, 64, 32, NC, 3>();
@@ -398,21 +401,23 @@ int launch_decode(const DecodeArgs& a, bool fp8, void* ws, size_t ws_bytes, bool
   p.part_o = reinterpret_cast<float*>(w + L.part_o);
   p.part_ml = reinterpret_cast<float*>(w + L.part_ml);
 
-  e->kernel<<<grid, e->threads, e->smem, stream>>>(p);
-  if (cudaGetLastError() != cudaSuccess) return PKV_ERR_CUDA;
-  // The merge kernel is launched as a programmatic dependent of the decode
-  // kernel: its CTAs can be resident before the decode grid ends and start
-  // the moment it has (griddepcontrol.wait), hiding the launch gap.
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(nwt));
-  cfg.blockDim = dim3(128);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = stream;
+  // Both kernels are launched as programmatic dependents of the kernel
+  // before them in the stream: their CTAs can be resident before it ends and
+  // start work the moment it has (griddepcontrol.wait), hiding launch gaps.
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(static_cast<unsigned>(e->threads));
+  cfg.dynamicSmemBytes = static_cast<size_t>(e->smem);
+  cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, e->kernel, p) != cudaSuccess) return PKV_ERR_CUDA;
+  cfg.gridDim = dim3(static_cast<unsigned>(nwt));
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
   if (cudaLaunchKernelEx(&cfg, e->merge, p) != cudaSuccess) return PKV_ERR_CUDA;
   return PKV_OK;
 }
