@@ -220,14 +220,19 @@ def oracle_rate(s: W.Spec, host, seqs) -> tuple:
 
 
 def cpu_baseline(s: W.Spec, host, budget_s: float) -> dict:
+    """The oracle over the workload's sequences in order, cycling through them
+    until about budget_s seconds of CPU work have been done."""
     S = s.num_seqs
-    dt1, _ = oracle_rate(s, host, [0])
-    n = max(1, min(S, int(budget_s / max(dt1, 1e-3))))
-    seqs = list(range(n))
-    dt, nbytes = oracle_rate(s, host, seqs)
-    return {"value": nbytes / dt / 1e9, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
-            "sample": f"fp64 numpy oracle on the first {n} of {S} sequences ({nbytes} K/V bytes), "
-                      f"{dt:.1f} s", "seqs_per_s": n / dt}
+    tot_t, tot_b, done = 0.0, 0, 0
+    while tot_t < budget_s:
+        dt, nb = oracle_rate(s, host, [done % S])
+        tot_t += dt
+        tot_b += nb
+        done += 1
+    return {"value": tot_b / tot_t / 1e9, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"fp64 numpy oracle, one sequence per call, cycling over the workload's {S} "
+                      f"sequences: {done} sequence decodes ({tot_b} K/V bytes) in {tot_t:.1f} s",
+            "seqs_per_s": done / tot_t}
 
 
 # ---------------------------------------------------------------------------
