@@ -66,10 +66,44 @@ def workload_spec(a) -> W.Spec:
         over["cache_dtype"] = a.cache_dtype
         if a.cache_dtype in ("f16", "bf16"):
             over["q_dtype"] = a.cache_dtype
-    s = W.spec(a.workload, **over)
-    if s.lens[0] == "prefix":
-        raise SystemExit("bench.py times the layouts drawn by workloads.make_layout")
-    return s.replace(append=True)
+    return W.spec(a.workload, **over).replace(append=True)
+
+
+def prefix_layout(s: W.Spec, allocator_cls) -> W.Layout:
+    """The shared-prefix layout, built by a block allocator from the
+    workload's operation script; the step's appends (one copy-on-write among
+    them) give the slot mapping and the block-copy pairs. The timed arm uses
+    the library's allocator, the reference arm the oracle's."""
+    sc = W.prefix_script(s)
+    a = allocator_cls(sc.num_blocks, s.block_size, sc.free_order)
+    a.run(sc.setup)
+    width = -(-max(sc.final_lens) // s.block_size)
+
+    def tables():
+        t = torch.full((len(sc.seqs), width), -1, dtype=torch.int32)
+        for i, r in enumerate(sc.seqs):
+            row = a.table(r)
+            t[i, :len(row)] = torch.tensor(row, dtype=torch.int32)
+        return t
+
+    fill_tables = tables()
+    step = [a.append_slot(r) for r in sc.step_appends]
+    lens = torch.tensor(sc.final_lens, dtype=torch.int32)
+    lay = W.Layout(s, sc.num_blocks, lens, tables(), lens - 1, fill_tables)
+    lay.slot_mapping = torch.tensor([x[0] for x in step], dtype=torch.int64)
+    lay.cow_pairs = torch.tensor([[x[1], x[2]] for x in step if x[1] >= 0], dtype=torch.int32).reshape(-1, 2)
+    return lay
+
+
+def unique_kv_bytes(s: W.Spec, lay) -> int:
+    """K+V bytes of the distinct stored tokens the decode reads (a block shared
+    by several tables counts once, with its longest use)."""
+    B = s.block_size
+    fill = {}
+    for row, L in zip(lay.tables.tolist(), lay.lens.tolist()):
+        for b in range(-(-L // B)):
+            fill[row[b]] = max(fill.get(row[b], 0), min(B, L - b * B))
+    return sum(fill.values()) * 2 * s.num_kv_heads * s.head_dim * s.cache_elem_bytes
 
 
 def config_of(s: W.Spec, lay, kv_bytes: int) -> dict:
@@ -255,7 +289,11 @@ def dist_setup(a):
 def run_reference(a, s: W.Spec, ws: int, rank: int):
     if rank != 0:
         return
-    lay = W.make_layout(s)
+    if s.lens[0] == "prefix":
+        from oracle.allocator import BlockAllocator
+        lay = prefix_layout(s, BlockAllocator)
+    else:
+        lay = W.make_layout(s)
     t = W.make_tensors(s, lay.num_blocks, lay.fill_tables, lay.fill_lens, device="cpu")
     host = _host_inputs(s, lay, t)
     # Size each step's sample so that warm-up + steps take about 2 minutes.
@@ -316,18 +354,36 @@ def main():
         dist.barrier()
     dev = local
     torch.cuda.set_device(dev)
-    lay = W.make_layout(s)
+    shared = s.lens[0] == "prefix"
+    lay = prefix_layout(s, P.BlockAllocator) if shared else W.make_layout(s)
     t = W.make_tensors(s, lay.num_blocks, lay.fill_tables, lay.fill_lens, device=f"cuda:{dev}")
     tables, lens = lay.tables.cuda(), lay.lens.cuda()
     slots = lay.slot_mapping.cuda()
     out = torch.empty_like(t.q)
     fp8 = s.cache_dtype == "fp8_e4m3"
-    reshape = P.prepare_reshape(t.k_new, t.v_new, t.k_cache, t.v_cache, slots, t.k_scale, t.v_scale)
+    write = P.prepare_reshape(t.k_new, t.v_new, t.k_cache, t.v_cache, slots, t.k_scale, t.v_scale)
+    n_cow = int(lay.cow_pairs.shape[0])
+    if n_cow:
+        cow = P.prepare_copy_blocks(t.k_cache, t.v_cache, lay.cow_pairs.cuda())
+
+        def reshape():
+            cow()
+            write()
+    else:
+        reshape = write
     decode = P.prepare_decode(t.q, t.k_cache, t.v_cache, tables, lens, s.num_kv_heads, s.scale,
                               s.block_size, out, t.k_scale, t.v_scale)
     lens_l = lay.lens.tolist()
     kv_bytes = kv_bytes_of(s, lens_l)
     alg = decode_alg_bytes(s, lens_l)
+    extra = {}
+    if shared:
+        # Each request reads the shared prefix blocks again (mostly from L2);
+        # the roofline counts every distinct stored byte once.
+        uniq = unique_kv_bytes(s, lay)
+        alg = alg - kv_bytes + uniq
+        extra = {"kv_bytes_unique": uniq, "cow_copies_per_step": n_cow,
+                 "alg_bytes": "roofline counts distinct stored K/V bytes; value counts K/V bytes per request"}
 
     for _ in range(max(3, a.warmup)):
         reshape()
@@ -367,7 +423,7 @@ def main():
         raise SystemExit(f"device check failed: {P.status_string(st)}")
     step_s = elapsed_ms / 1e3 / K
     value = ws * kv_bytes / step_s / 1e9
-    launches_per_step = 3  # reshape_and_cache, decode_kernel, decode_merge_kernel
+    launches_per_step = 3 + (1 if n_cow else 0)  # [copy_blocks,] reshape_and_cache, decode, merge
 
     # ---- end to end through the public API: pinned host in, result out ----
     Ke = a.e2e_steps or max(3, min(K, 2000))
@@ -411,7 +467,7 @@ def main():
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": K, "warmup": a.warmup,
         "ms_per_step": elapsed_ms / K, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "fp8_e4m3" if fp8 else s.cache_dtype, "data": "synthetic",
-        "config": config_of(s, lay, kv_bytes) | {"parallelism": f"replicas x{ws}"},
+        "config": config_of(s, lay, kv_bytes) | {"parallelism": f"replicas x{ws}"} | extra,
         "seqs_per_s": ws * s.num_seqs / step_s,
         "pct_of_hbm_peak": 100.0 * value / ws / peak,
         "roofline": {"kernel": "paged_attn_decode (decode_kernel + decode_merge_kernel)", "bound": "hbm",
