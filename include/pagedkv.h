@@ -325,6 +325,34 @@ int pkv_alloc_stats(void* handle, int32_t* free_blocks, int32_t* used_blocks,
 /* Reference count of one block (>= 0) or PKV_ERR_INVALID_ARG. */
 int pkv_block_refcount(void* handle, int32_t block);
 
+/* Shared-prefix groups of a decode batch, for paged_attn_decode_cascade.
+ * Prefix sharing: "PagedAttention: treat the cache like virtual memory"
+ * (KV-Cache Management and PagedAttention) and "Shared System Prompts & Prefix
+ * Caching" (PagedAttention and KV Cache Management): requests that start with
+ * the same prompt point their block tables at the same physical blocks.
+ *
+ * Rows (batch positions) whose first block is full (lens[r] >= block_size)
+ * are bucketed by that first block id, buckets in order of their lowest row,
+ * rows ascending. A bucket of at least min_members rows is a group; its
+ * prefix is the longest run of leading table columns j that hold the same
+ * block in every member and are full in every member ((j + 1) * block_size
+ * <= lens[r]).
+ *   tables         host int32 [S, width], row-major (row stride width)
+ *   lens           host int32 [S]
+ *   group_start    host int32 [S + 1] out: group g's members are
+ *                  members[group_start[g] .. group_start[g + 1])
+ *   members        host int32 [S] out: rows, grouped
+ *   prefix_blocks  host int32 [S] out: the shared prefix of the row's group in
+ *                  blocks, 0 for rows in no group
+ *   num_groups, num_members  out: G and M
+ * Pure host function, no state. PKV_ERR_INVALID_ARG on a null pointer,
+ * S < 0, width < 1, block_size < 1 or min_members < 1; PKV_ERR_OOM if host
+ * memory runs out. */
+int pkv_prefix_groups(const int32_t* tables, int32_t S, int32_t width, const int32_t* lens,
+                      int32_t block_size, int32_t min_members, int32_t* group_start,
+                      int32_t* members, int32_t* prefix_blocks, int32_t* num_groups,
+                      int32_t* num_members);
+
 #ifdef __cplusplus
 }
 #endif

@@ -48,7 +48,7 @@ EXPORTED = (
     "pkv_device_error",
     "pkv_alloc_create", "pkv_alloc_destroy", "pkv_seq_allocate", "pkv_seq_append_slot",
     "pkv_seq_fork", "pkv_seq_free", "pkv_seq_num_tokens", "pkv_seq_block_table",
-    "pkv_build_block_tables", "pkv_alloc_stats", "pkv_block_refcount",
+    "pkv_build_block_tables", "pkv_alloc_stats", "pkv_block_refcount", "pkv_prefix_groups",
 )
 
 
@@ -257,6 +257,28 @@ def device_error(device: int = 0) -> int:
 # ---------------------------------------------------------------------------
 # Host block allocator
 # ---------------------------------------------------------------------------
+
+def prefix_groups(tables, lens, block_size: int, min_members: int = 2):
+    """Shared-prefix groups of a decode batch (pkv_prefix_groups).
+
+    tables: int32 [S, W] CPU tensor, lens: int32 [S] CPU tensor. Returns
+    (group_start int32 [G + 1], members int32 [M], prefix_blocks int32 [S]) as
+    CPU tensors."""
+    import torch
+    t = tables.to(torch.int32).contiguous()
+    ln = lens.to(torch.int32).contiguous()
+    S, W = int(t.shape[0]), int(t.shape[1])
+    gs = torch.empty(S + 1, dtype=torch.int32)
+    mem = torch.empty(max(S, 1), dtype=torch.int32)
+    pb = torch.empty(max(S, 1), dtype=torch.int32)
+    G, M = ctypes.c_int32(), ctypes.c_int32()
+    i32 = ctypes.POINTER(ctypes.c_int32)
+    _check(lib().pkv_prefix_groups(ctypes.cast(t.data_ptr(), i32), S, max(W, 1), ctypes.cast(ln.data_ptr(), i32),
+                                   int(block_size), int(min_members), ctypes.cast(gs.data_ptr(), i32),
+                                   ctypes.cast(mem.data_ptr(), i32), ctypes.cast(pb.data_ptr(), i32),
+                                   ctypes.byref(G), ctypes.byref(M)), "pkv_prefix_groups")
+    return gs[:G.value + 1].clone(), mem[:M.value].clone(), pb[:S].clone()
+
 
 class BlockAllocator:
     """The C++ block allocator (FIFO free list, refcounts, fork, copy-on-write)."""

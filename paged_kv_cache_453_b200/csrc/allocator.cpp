@@ -12,6 +12,7 @@
 // more than num_blocks ids), a refcount array and a hash map from sequence id
 // to (table, token count).
 
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
 #include <new>
@@ -263,6 +264,66 @@ int pkv_alloc_stats(void* handle, int32_t* free_blocks, int32_t* used_blocks,
 int pkv_block_refcount(void* handle, int32_t block) {
   if (!handle) return PKV_ERR_INVALID_ARG;
   return as_pool(handle)->refcount(block);
+}
+
+// Shared-prefix groups of a decode batch (prefix sharing: "PagedAttention:
+// treat the cache like virtual memory", "Shared System Prompts & Prefix
+// Caching"): rows whose first block is full are bucketed by that block id in
+// order of first appearance; a bucket of at least min_members rows is a group
+// whose prefix is the longest run of leading columns holding the same block,
+// full, in every member.
+int pkv_prefix_groups(const int32_t* tables, int32_t S, int32_t width, const int32_t* lens,
+                      int32_t block_size, int32_t min_members, int32_t* group_start,
+                      int32_t* members, int32_t* prefix_blocks, int32_t* num_groups,
+                      int32_t* num_members) {
+  if (S < 0 || width < 1 || block_size < 1 || min_members < 1 || !group_start || !members ||
+      !prefix_blocks || !num_groups || !num_members || (S > 0 && (!tables || !lens)))
+    return PKV_ERR_INVALID_ARG;
+  try {
+    std::unordered_map<int32_t, int32_t> bucket_of;  // first block -> bucket
+    std::vector<std::vector<int32_t>> buckets;
+    for (int32_t r = 0; r < S; ++r) {
+      prefix_blocks[r] = 0;
+      if (lens[r] < block_size) continue;
+      const int32_t key = tables[static_cast<int64_t>(r) * width];
+      auto it = bucket_of.find(key);
+      if (it == bucket_of.end()) {
+        bucket_of.emplace(key, static_cast<int32_t>(buckets.size()));
+        buckets.emplace_back(1, r);
+      } else {
+        buckets[it->second].push_back(r);
+      }
+    }
+    int32_t g = 0, m = 0;
+    group_start[0] = 0;
+    for (const auto& rows : buckets) {
+      if (static_cast<int32_t>(rows.size()) < min_members) continue;
+      int32_t min_len = lens[rows[0]];
+      for (int32_t r : rows) min_len = lens[r] < min_len ? lens[r] : min_len;
+      const int32_t lim = std::min<int64_t>(width, min_len / block_size);  // columns full in all
+      const int32_t* first = tables + static_cast<int64_t>(rows[0]) * width;
+      int32_t n = 0;
+      for (; n < lim; ++n) {
+        bool same = true;
+        for (int32_t r : rows)
+          if (tables[static_cast<int64_t>(r) * width + n] != first[n]) {
+            same = false;
+            break;
+          }
+        if (!same) break;
+      }
+      for (int32_t r : rows) {
+        members[m++] = r;
+        prefix_blocks[r] = n;
+      }
+      group_start[++g] = m;
+    }
+    *num_groups = g;
+    *num_members = m;
+  } catch (const std::bad_alloc&) {
+    return PKV_ERR_OOM;
+  }
+  return PKV_OK;
 }
 
 }  // extern "C"

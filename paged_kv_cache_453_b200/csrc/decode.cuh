@@ -153,18 +153,20 @@ struct Cursor {
   __device__ __forceinline__ long long unit_end() const { return k - b + n; }
 };
 
-template <int CK, bool QBF, int D, int BS, int NC, int NS>
+template <int CK, bool QBF, int D, int BS, int NC, int NS, int IB>
 struct DecodeCfg {
   static constexpr bool kFp8 = (CK == kCacheE4M3);
   static constexpr bool kMmaBF16 = (CK == kCacheBF16);
   static constexpr int EB = kFp8 ? 1 : 2;         // cache element bytes
   static constexpr int EPR = 128 / EB;            // elements per swizzled 128-byte row
   static constexpr int NH = (D * EB) / 128;       // 128-byte column groups per token row
-  static constexpr int TILE = BS * D * EB;        // one K (or V) tile
-  static constexpr int STAGE = 2 * TILE;
+  static constexpr int TILE = BS * D * EB;        // one K (or V) tile of one block
+  static constexpr int TOK = IB * BS;             // tokens per work item
+  static constexpr int KT = IB * TILE;            // K (or V) tiles of one item
+  static constexpr int STAGE = 2 * KT;
   static constexpr int KS = D / 16;               // k-steps of the QK^T product
   static constexpr int MT = D / 16;               // m-tiles of the PV product
-  static constexpr int TT = BS / 16;              // 16-token tiles per block
+  static constexpr int TT = TOK / 16;             // 16-token tiles per item
   static constexpr int NT = NC * 32;
   static constexpr int SMEM = 1024 + NC * NS * STAGE + NC * NS * 8 + (NT + NC + 1) * 8 + 64;
   static_assert((D * EB) % 128 == 0, "head_dim * elem bytes must be a multiple of 128");
@@ -181,9 +183,10 @@ __device__ __forceinline__ uint32_t swz(int t, int bcol) {
                                ((((bcol & 127) >> 4) ^ (t & 7)) << 4));
 }
 
-template <int CK, bool QBF, int D, int BS, int NC, int NS>
+template <int CK, bool QBF, int D, int BS, int NC, int NS, int IB>
 __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
-  using C = DecodeCfg<CK, QBF, D, BS, NC, NS>;
+  using C = DecodeCfg<CK, QBF, D, BS, NC, NS, IB>;
+  constexpr int TOK = C::TOK;
   constexpr bool FP8 = C::kFp8;
   constexpr bool MBF = C::kMmaBF16;
   constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s
@@ -231,7 +234,7 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
         if (blockIdx.x == 0) atomicOr(p.err, kErrBadLen);
         len = len < 0 ? 0 : max_len;
       }
-      sum += static_cast<long long>(p.Hk) * items_of<BS>(len);
+      sum += static_cast<long long>(p.Hk) * items_of<TOK>(len);
     }
     long long v = sum;  // inclusive warp scan, then warp totals
 #pragma unroll
@@ -267,7 +270,7 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
   if (lane == 0) p.desc[gw * (1 + kMaxSteals)] = make_int4(-1, 0, 0, 0);
 
   // Position of global item x: chunk by binary search, then a warp-wide walk.
-  auto locate = [&](long long x, Cursor<BS>& out) -> bool {
+  auto locate = [&](long long x, Cursor<TOK>& out) -> bool {
     int a = 0, bnd = C::NT - 1;
     while (a < bnd) {  // largest t with scan[t] <= x
       int m = (a + bnd + 1) >> 1;
@@ -284,7 +287,7 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
       if (s < s_hi) {
         len = __ldg(p.lens + s);
         len = len < 0 ? 0 : (len > max_len ? max_len : len);
-        w = static_cast<long long>(p.Hk) * items_of<BS>(len);
+        w = static_cast<long long>(p.Hk) * items_of<TOK>(len);
       }
       long long incl = w;
 #pragma unroll
@@ -297,7 +300,7 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
         const int j = __ffs(hit) - 1;
         const long long start = __shfl_sync(0xffffffffu, base + incl - w, j);
         const int L = __shfl_sync(0xffffffffu, len, j);
-        const int n = items_of<BS>(L);
+        const int n = items_of<TOK>(L);
         const long long off = x - start;
         out.k = x;
         out.s = s0 + j;
@@ -334,12 +337,12 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
   // hi drops to where thieves took over. Partials go to slots slot_base (+1).
   auto run_range = [&](long long a, long long hi, bool claim, int owner, int sub,
                        long long slot_base) -> bool {
-    Cursor<BS> cur;
+    Cursor<TOK> cur;
     if (!locate(a, cur)) {
       if (lane == 0) atomicOr(p.err, kErrBadLen);
       return false;
     }
-    Cursor<BS> pc = cur;
+    Cursor<TOK> pc = cur;
     const long long lo = a;
 
     unsigned long long* wp = p.words + owner;
@@ -353,27 +356,41 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
         if (lane == 0) mbar_arrive(bar);
         return;
       }
-      if (pc.s != tw_s || pc.b < tw_b0 || pc.b >= tw_b0 + 32) {
+      // blocks b0 .. b0 + nload - 1 of the sequence: the item's blocks that hold tokens
+      const int nb = (pc.L + BS - 1) / BS;
+      const int b0 = pc.b * IB;
+      const int nload = min(IB, nb - b0);
+      if (pc.s != tw_s || b0 < tw_b0 || b0 + nload > tw_b0 + 32) {
         tw_s = pc.s;
-        tw_b0 = pc.b;
-        const int nb = (pc.L + BS - 1) / BS;
+        tw_b0 = b0;
         tw_val = (tw_b0 + lane < nb) ? __ldg(p.tables + pc.s * p.t_s + tw_b0 + lane) : 0;
       }
-      int phys = __shfl_sync(0xffffffffu, tw_val, pc.b - tw_b0);
-      if (phys < 0 || phys >= p.NB) {
-        if (lane == 0) atomicOr(p.err, kErrBadBlock);
-        phys = 0;
+      int phys[IB];
+#pragma unroll
+      for (int ib = 0; ib < IB; ++ib) {
+        phys[ib] = __shfl_sync(0xffffffffu, tw_val, (b0 - tw_b0 + ib) & 31);
+        if (ib < nload && (phys[ib] < 0 || phys[ib] >= p.NB)) {
+          if (lane == 0) atomicOr(p.err, kErrBadBlock);
+          phys[ib] = 0;
+        }
       }
       if (lane == 0) {
         const uint32_t dk = my_stages + stage * C::STAGE;
-        const uint32_t dv = dk + C::TILE;
-        mbar_arrive_expect_tx(bar, C::STAGE);
+        const uint32_t dv = dk + C::KT;
+        mbar_arrive_expect_tx(bar, nload * 2 * C::TILE);
 #pragma unroll
-        for (int hh = 0; hh < C::NH; ++hh)
-          tma_load_4d(dk + hh * BS * 128, &p.tmk, bar, hh * C::EPR, 0, pc.h, phys, policy);
+        for (int ib = 0; ib < IB; ++ib) {
+          if (ib < nload) {
 #pragma unroll
-        for (int hh = 0; hh < C::NH; ++hh)
-          tma_load_4d(dv + hh * BS * 128, &p.tmv, bar, hh * C::EPR, 0, pc.h, phys, policy);
+            for (int hh = 0; hh < C::NH; ++hh)
+              tma_load_4d(dk + ib * C::TILE + hh * BS * 128, &p.tmk, bar, hh * C::EPR, 0, pc.h,
+                          phys[ib], policy);
+#pragma unroll
+            for (int hh = 0; hh < C::NH; ++hh)
+              tma_load_4d(dv + ib * C::TILE + hh * BS * 128, &p.tmv, bar, hh * C::EPR, 0, pc.h,
+                          phys[ib], policy);
+          }
+        }
       }
     };
     // Issue the item at pc into the next ring stage if it is ours; false when
@@ -538,8 +555,8 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
       bool refilled = false;
       if (cur.L > 0) {
         const uint32_t tk = my_stages + stage * C::STAGE;
-        const uint32_t tv = tk + C::TILE;
-        const int nvalid = min(BS, cur.L - cur.b * BS);
+        const uint32_t tv = tk + C::KT;
+        const int nvalid = min(TOK, cur.L - cur.b * TOK);
         // 16-token blocks: the V fragments go to registers right after QK^T
         // (the MMAs consume the K fragments, the context mask consumes the V
         // fragments), so the stage is refilled before the softmax and PV and
@@ -553,19 +570,21 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
 #pragma unroll
         for (int tt = 0; tt < C::TT; ++tt) {
           sacc[tt][0] = sacc[tt][1] = sacc[tt][2] = sacc[tt][3] = 0.f;
-          const int trow = tt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+          // 16-token tile tt lies inside block (tt * 16) / BS of the item
+          const uint32_t kt = tk + ((tt * 16) / BS) * C::TILE;
+          const int trow = (tt * 16) % BS + (lane & 7) + ((lane >> 3) & 1) * 8;
           if constexpr (!FP8) {
 #pragma unroll
             for (int ks = 0; ks < C::KS; ++ks) {
               uint32_t a0, a1, a2, a3;
-              ldsm_x4(tk + swz<BS>(trow, ks * 32 + (lane >> 4) * 16), a0, a1, a2, a3);
+              ldsm_x4(kt + swz<BS>(trow, ks * 32 + (lane >> 4) * 16), a0, a1, a2, a3);
               mma16816<MBF>(sacc[tt], a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
             }
           } else {
 #pragma unroll
             for (int kp = 0; kp < C::KS / 2; ++kp) {
               uint32_t x0, x1, x2, x3;
-              ldsm_x4(tk + swz<BS>(trow, kp * 32 + (lane >> 4) * 16), x0, x1, x2, x3);
+              ldsm_x4(kt + swz<BS>(trow, kp * 32 + (lane >> 4) * 16), x0, x1, x2, x3);
               mma16816<false>(sacc[tt], e4m3x2_to_f16x2(x0 & 0xffff),
                               e4m3x2_to_f16x2(x1 & 0xffff), e4m3x2_to_f16x2(x0 >> 16),
                               e4m3x2_to_f16x2(x1 >> 16), qb[2 * kp][0], qb[2 * kp][1]);
@@ -586,16 +605,18 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
           const uint32_t keep23 =
               (tb + 8 < nvalid ? 0x0000ffffu : 0u) | (tb + 9 < nvalid ? 0xffff0000u : 0u);
           if constexpr (!FP8) {
-            const int vrow = tt * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
-            ldsm_x4_t(tv + swz<BS>(vrow, i * 32 + ((lane >> 3) & 1) * 16), f[0], f[1], f[2], f[3]);
+            const int vrow = (tt * 16) % BS + (lane & 7) + ((lane >> 4) & 1) * 8;
+            ldsm_x4_t(tv + ((tt * 16) / BS) * C::TILE + swz<BS>(vrow, i * 32 + ((lane >> 3) & 1) * 16),
+                      f[0], f[1], f[2], f[3]);
             f[0] &= keep01;
             f[1] &= keep01;
             f[2] &= keep23;
             f[3] &= keep23;
           } else {
-            const int vrow = tt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+            const int vrow = (tt * 16) % BS + (lane & 7) + ((lane >> 3) & 1) * 8;
             uint32_t x0, x1, x2, x3;
-            ldsm_x4_t(tv + swz<BS>(vrow, i * 32 + (lane >> 4) * 16), x0, x1, x2, x3);
+            ldsm_x4_t(tv + ((tt * 16) / BS) * C::TILE + swz<BS>(vrow, i * 32 + (lane >> 4) * 16), x0,
+                      x1, x2, x3);
             const uint32_t e0 = prmt(x0, 0, 0x3120), e1 = prmt(x1, 0, 0x3120);
             const uint32_t e2 = prmt(x2, 0, 0x3120), e3 = prmt(x3, 0, 0x3120);
             f[0] = e4m3x2_to_f16x2(e0 & 0xffff) & keep01;

@@ -157,23 +157,24 @@ struct DecodeLaunch {
   int occ[kMaxDevices];  // resident CTAs per SM, 0 = not queried yet
 };
 
-template <int CK, bool QBF, int D, int BS, int NC, int NS>
+template <int CK, bool QBF, int D, int BS, int NC, int NS, int IB = 1>
 DecodeLaunch* decode_entry() {
-  static DecodeLaunch e = {&decode_kernel<CK, QBF, D, BS, NC, NS>,
+  static DecodeLaunch e = {&decode_kernel<CK, QBF, D, BS, NC, NS, IB>,
                            &decode_merge_kernel<QBF, D>,
                            NC * 32,
-                           DecodeCfg<CK, QBF, D, BS, NC, NS>::SMEM,
+                           DecodeCfg<CK, QBF, D, BS, NC, NS, IB>::SMEM,
                            NC,
                            {0}};
   return &e;
 }
 
-// Warps per CTA (NC) and ring stages per warp (NS), measured on B200. Two
-// CTAs of ~96 KB share an SM where a stage is 8 KB or less: 16-bit, D = 128,
-// 16-token blocks do best with 3 warps x 4 stages (deeper per-warp rings);
-// 4 KB stages (fp8, D = 64) with 4 warps x 6 stages (more math per byte
-// wants more warps); 32-token 16-bit blocks use 4 warps x 3 stages of 16 KB
-// (one CTA per SM).
+// Warps per CTA (NC), ring stages per warp (NS) and blocks per work item
+// (IB), measured on B200. Two CTAs of ~96 KB share an SM where a stage is
+// 8 KB or less: 16-bit, D = 128, 16-token blocks do best with 3 warps x 4
+// stages (deeper per-warp rings); D = 64 with 4 warps x 6 stages of 4 KB;
+// 32-token 16-bit blocks use 4 warps x 3 stages of 16 KB (one CTA per SM).
+// fp8 items take two 16-token blocks (32 tokens, 8 KB stages): the widening
+// makes fp8 issue-bound, and larger items halve the per-item overhead.
 DecodeLaunch* pick_decode(int ck, bool qbf, int D, int BS) {
   constexpr int NC = 4;
   if (ck == kCacheBF16) {
@@ -188,10 +189,10 @@ DecodeLaunch* pick_decode(int ck, bool qbf, int D, int BS) {
     if (D == 64 && BS == 32) return decode_entry<kCacheF16, false, 64, 32, NC, 3>();
   } else if (ck == kCacheE4M3 && D == 128) {
     if (qbf) {
-      if (BS == 16) return decode_entry<kCacheE4M3, true, 128, 16, NC, 6>();
+      if (BS == 16) return decode_entry<kCacheE4M3, true, 128, 16, NC, 3, 2>();
       if (BS == 32) return decode_entry<kCacheE4M3, true, 128, 32, NC, 3>();
     } else {
-      if (BS == 16) return decode_entry<kCacheE4M3, false, 128, 16, NC, 6>();
+      if (BS == 16) return decode_entry<kCacheE4M3, false, 128, 16, NC, 3, 2>();
       if (BS == 32) return decode_entry<kCacheE4M3, false, 128, 32, NC, 3>();
     }
   }

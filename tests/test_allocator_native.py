@@ -2,6 +2,8 @@
 against the oracle allocator on random operation sequences (bit-exact)."""
 import random
 
+import numpy as np
+
 import pytest
 
 import paged_kv_cache_453_b200 as P
@@ -113,3 +115,57 @@ def test_errors_are_atomic():
     with pytest.raises(P.PkvError) as e:
         P.BlockAllocator(3, 4, [0, 0, 1])
     assert e.value.status == P.PKV_ERR_INVALID_ARG
+
+
+# ---------------------------------------------------------------------------
+# pkv_prefix_groups against the oracle's definition (bit-exact)
+# ---------------------------------------------------------------------------
+
+def _fork_tree_layout(seed, B=4):
+    rng = np.random.default_rng(seed)
+    a = OracleAlloc(600, B)
+    seqs = []
+    for i in range(int(rng.integers(1, 6))):
+        a.allocate(i, int(rng.integers(0, 30)))
+        seqs.append(i)
+    nxt = len(seqs)
+    for _ in range(40):
+        op = rng.integers(4)
+        if op == 0:
+            a.fork(int(rng.choice(seqs)), nxt)
+            seqs.append(nxt)
+            nxt += 1
+        else:
+            r = int(rng.choice(seqs))
+            for _ in range(int(rng.integers(1, 9))):
+                a.append_slot(r)
+    rng.shuffle(seqs)
+    rows = [a.table(r) for r in seqs]
+    width = max(1, max(len(r) for r in rows))
+    t = np.full((len(rows), width), -1, dtype=np.int32)
+    for i, r in enumerate(rows):
+        t[i, :len(r)] = r
+    return t, np.array([a.num_tokens[r] for r in seqs], dtype=np.int32)
+
+
+@pytest.mark.parametrize("seed", range(20))
+def test_prefix_groups_match_oracle(seed):
+    import torch
+    from oracle.prefix import prefix_groups as oracle_groups
+    tables, lens = _fork_tree_layout(seed)
+    for mm in (1, 2, 3):
+        gs, mem, pb = P.prefix_groups(torch.from_numpy(tables), torch.from_numpy(lens), 4, mm)
+        ogs, omem, opb = oracle_groups(tables, lens, 4, mm)
+        assert gs.tolist() == ogs and mem.tolist() == omem and pb.tolist() == opb, (seed, mm)
+
+
+def test_prefix_groups_rejects_bad_arguments():
+    import torch
+    t = torch.zeros((2, 2), dtype=torch.int32)
+    ln = torch.full((2,), 8, dtype=torch.int32)
+    with pytest.raises(P.PkvError):
+        P.prefix_groups(t, ln, 0)
+    with pytest.raises(P.PkvError):
+        P.prefix_groups(t, ln, 4, 0)
+    gs, mem, pb = P.prefix_groups(t[:0], ln[:0], 4)
+    assert gs.tolist() == [0] and mem.tolist() == [] and pb.tolist() == []
