@@ -55,6 +55,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cascade", action="store_true",
+                    help="decode a shared-prefix workload with the plain decode")
     return ap.parse_args()
 
 
@@ -371,8 +373,14 @@ def main():
             write()
     else:
         reshape = write
-    decode = P.prepare_decode(t.q, t.k_cache, t.v_cache, tables, lens, s.num_kv_heads, s.scale,
-                              s.block_size, out, t.k_scale, t.v_scale)
+    cascade = shared and not a.no_cascade
+    if cascade:
+        groups = P.PrefixGroups(lay.tables, lay.lens, s.block_size, device=f"cuda:{dev}")
+        decode = P.prepare_decode_cascade(t.q, t.k_cache, t.v_cache, tables, lens, groups, s.num_kv_heads,
+                                          s.scale, s.block_size, out)
+    else:
+        decode = P.prepare_decode(t.q, t.k_cache, t.v_cache, tables, lens, s.num_kv_heads, s.scale,
+                                  s.block_size, out, t.k_scale, t.v_scale)
     lens_l = lay.lens.tolist()
     kv_bytes = kv_bytes_of(s, lens_l)
     alg = decode_alg_bytes(s, lens_l)
@@ -383,7 +391,8 @@ def main():
         uniq = unique_kv_bytes(s, lay)
         alg = alg - kv_bytes + uniq
         extra = {"kv_bytes_unique": uniq, "cow_copies_per_step": n_cow,
-                 "alg_bytes": "roofline counts distinct stored K/V bytes; value counts K/V bytes per request"}
+                 "alg_bytes": "roofline counts distinct stored K/V bytes; value counts K/V bytes per request",
+                 "decode": "prefix-aware (shared prefix read once per group)" if cascade else "plain"}
 
     for _ in range(max(3, a.warmup)):
         reshape()
@@ -423,15 +432,20 @@ def main():
         raise SystemExit(f"device check failed: {P.status_string(st)}")
     step_s = elapsed_ms / 1e3 / K
     value = ws * kv_bytes / step_s / 1e9
-    launches_per_step = 3 + (1 if n_cow else 0)  # [copy_blocks,] reshape_and_cache, decode, merge
+    # [copy_blocks,] reshape_and_cache, decode, merge [, prefix pass, prefix merge]
+    launches_per_step = 3 + (1 if n_cow else 0) + (2 if cascade else 0)
 
     # ---- end to end through the public API: pinned host in, result out ----
     Ke = a.e2e_steps or max(3, min(K, 2000))
     pin = lambda x: x.cpu().pin_memory()  # noqa: E731
     h_in = {"q": pin(t.q), "k_new": pin(t.k_new), "v_new": pin(t.v_new), "slots": pin(lay.slot_mapping),
             "tables": pin(lay.tables), "lens": pin(lay.lens)}
-    h_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
     d_in = {"q": t.q, "k_new": t.k_new, "v_new": t.v_new, "slots": slots, "tables": tables, "lens": lens}
+    if cascade:
+        for k_ in ("prefix_blocks", "group_start", "members"):
+            h_in[k_] = pin(getattr(groups, k_))
+            d_in[k_] = getattr(groups, k_)
+    h_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
     h2d = sum(x.numel() * x.element_size() for x in h_in.values())
     d2h = h_out.numel() * h_out.element_size()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -470,7 +484,9 @@ def main():
         "config": config_of(s, lay, kv_bytes) | {"parallelism": f"replicas x{ws}"} | extra,
         "seqs_per_s": ws * s.num_seqs / step_s,
         "pct_of_hbm_peak": 100.0 * value / ws / peak,
-        "roofline": {"kernel": "paged_attn_decode (decode_kernel + decode_merge_kernel)", "bound": "hbm",
+        "roofline": {"kernel": ("paged_attn_decode_cascade (decode, merge, prefix pass, prefix merge)"
+                                if cascade else "paged_attn_decode (decode_kernel + decode_merge_kernel)"),
+                     "bound": "hbm",
                      "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": profiled_traffic(s), "peak_source": peak_src,
                      "alg_bytes_per_launch": alg, "us_per_launch": dec_ms * 1e3},

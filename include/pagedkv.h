@@ -164,6 +164,49 @@ int paged_attn_decode_ex(const pkv_tensor* q, const pkv_tensor* k_cache,
                          size_t workspace_bytes, void* stream);
 
 /*
+ * paged_attn_decode_cascade - paged_attn_decode for a batch whose sequences
+ * share prompt prefixes, reading each shared prefix block once per group
+ * instead of once per sequence. Prefix sharing: "PagedAttention: treat the
+ * cache like virtual memory" (KV-Cache Management and PagedAttention) and
+ * "Shared System Prompts & Prefix Caching" (PagedAttention and KV Cache
+ * Management); the result is the attention paged_attn_decode defines (the
+ * softmax over a sequence's tokens is split into its prefix and the rest and
+ * recombined with the log-sum-exp rule), equal to it up to rounding order.
+ *
+ * Same q, caches (16-bit only), block_tables, context_lens, num_kv_heads,
+ * scale, block_size, out and stream as paged_attn_decode, plus a grouping of
+ * the batch (pkv_prefix_groups computes one from the tables on the host):
+ *   prefix_blocks  device int32 [S]: the leading table entries sequence s
+ *                  shares with its group (whole, full blocks), 0 if s is in
+ *                  no group
+ *   group_start    device int32 [num_groups + 1], group_members device
+ *                  int32 [M]: group g's members (batch rows) are
+ *                  group_members[group_start[g] .. group_start[g + 1])
+ *   num_groups, max_group_size (members of the largest group),
+ *   max_prefix_blocks (largest prefix_blocks): host ints sizing the launch
+ * Contract: a member's first prefix_blocks entries equal those of its
+ * group's first member, are full (prefix_blocks * block_size <= length), and
+ * are not written by this step; prefix_blocks[s] > 0 exactly for members.
+ * Rows breaking it are flagged (PKV_ERR_DEVICE_CHECK) where the kernels can
+ * see it, else their output rows are undefined.
+ *
+ * Kernels, in stream order: decode over each sequence's tokens after its
+ * prefix (sequences with a prefix leave fp32 partials), the split-KV merge,
+ * one prefix pass per (group, kv head, 64 query columns, prefix-block chunk)
+ * in which every query head of every member attends the shared blocks, and a
+ * final merge writing out. Uses a library-owned device buffer (grown with
+ * cudaMalloc when a larger batch needs it; fp32 partials of S * Hq rows plus
+ * the prefix chunks). PKV_ERR_UNSUPPORTED for fp8 caches.
+ */
+int paged_attn_decode_cascade(const pkv_tensor* q, const pkv_tensor* k_cache,
+                              const pkv_tensor* v_cache, const pkv_tensor* block_tables,
+                              const pkv_tensor* context_lens, const pkv_tensor* prefix_blocks,
+                              const pkv_tensor* group_start, const pkv_tensor* group_members,
+                              int num_groups, int max_group_size, int max_prefix_blocks,
+                              int num_kv_heads, float scale, int block_size, pkv_tensor* out,
+                              void* stream);
+
+/*
  * paged_attn_decode_noalloc - paged_attn_decode / paged_attn_decode_fp8 for
  * callers that cannot allocate device memory when they call: for example an
  * engine that hands almost all of HBM to its own KV-block pool at start-up

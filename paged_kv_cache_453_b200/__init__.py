@@ -44,7 +44,7 @@ PKV_ERR_SCRATCH_LIMIT = -10
 EXPORTED = (
     "pkv_status_string", "pkv_version",
     "paged_attn_decode", "paged_attn_decode_fp8", "paged_attn_decode_workspace_bytes",
-    "paged_attn_decode_ex", "paged_attn_decode_noalloc", "reshape_and_cache", "reshape_and_cache_fp8", "copy_blocks",
+    "paged_attn_decode_ex", "paged_attn_decode_noalloc", "paged_attn_decode_cascade", "reshape_and_cache", "reshape_and_cache_fp8", "copy_blocks",
     "pkv_device_error",
     "pkv_alloc_create", "pkv_alloc_destroy", "pkv_seq_allocate", "pkv_seq_append_slot",
     "pkv_seq_fork", "pkv_seq_free", "pkv_seq_num_tokens", "pkv_seq_block_table",
@@ -105,6 +105,11 @@ def lib() -> ctypes.CDLL:
             "pkv_alloc_stats": (ctypes.c_int, [vp, ctypes.POINTER(i32), ctypes.POINTER(i32),
                                                ctypes.POINTER(i32), ctypes.POINTER(i64)]),
             "pkv_block_refcount": (ctypes.c_int, [vp, i32]),
+            "paged_attn_decode_cascade": (ctypes.c_int, [P, P, P, P, P, P, P, P, ctypes.c_int, ctypes.c_int,
+                                                         ctypes.c_int, ctypes.c_int, f32, ctypes.c_int, P, vp]),
+            "pkv_prefix_groups": (ctypes.c_int, [ctypes.POINTER(i32), i32, i32, ctypes.POINTER(i32), i32, i32,
+                                                 ctypes.POINTER(i32), ctypes.POINTER(i32), ctypes.POINTER(i32),
+                                                 ctypes.POINTER(i32), ctypes.POINTER(i32)]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -176,6 +181,42 @@ def paged_attn_decode(q, k_cache, v_cache, block_tables, context_lens, num_kv_he
     _check(lib().paged_attn_decode(_ref(ds[0]), _ref(ds[1]), _ref(ds[2]), _ref(ds[3]), _ref(ds[4]),
                                    int(num_kv_heads), float(scale), int(block_size), _ref(ds[5]),
                                    _stream(stream)), "paged_attn_decode")
+
+
+class PrefixGroups:
+    """A batch's shared-prefix grouping on the device (from pkv_prefix_groups)."""
+
+    def __init__(self, tables, lens, block_size: int, min_members: int = 2, device=None):
+        import torch
+        gs, mem, pb = prefix_groups(tables.cpu(), lens.cpu(), block_size, min_members)
+        dev = device if device is not None else "cuda"
+        self.num_groups = int(gs.numel() - 1)
+        sizes = (gs[1:] - gs[:-1]).tolist()
+        self.max_group_size = int(max(sizes)) if sizes else 0
+        self.max_prefix_blocks = int(pb.max()) if pb.numel() else 0
+        self.group_start = gs.to(dev)
+        self.members = mem.to(dev) if mem.numel() else torch.zeros(0, dtype=torch.int32, device=dev)
+        self.prefix_blocks = pb.to(dev)
+
+
+def paged_attn_decode_cascade(q, k_cache, v_cache, block_tables, context_lens, groups: PrefixGroups,
+                              num_kv_heads: int, scale: float, block_size: int, out, stream=None) -> None:
+    ds = [_desc(x) for x in (q, k_cache, v_cache, block_tables, context_lens, groups.prefix_blocks,
+                             groups.group_start, groups.members, out)]
+    _check(lib().paged_attn_decode_cascade(*[_ref(d) for d in ds[:8]], groups.num_groups,
+                                           groups.max_group_size, groups.max_prefix_blocks,
+                                           int(num_kv_heads), float(scale), int(block_size), _ref(ds[8]),
+                                           _stream(stream)), "paged_attn_decode_cascade")
+
+
+def prepare_decode_cascade(q, k_cache, v_cache, block_tables, context_lens, groups: PrefixGroups,
+                           num_kv_heads: int, scale: float, block_size: int, out, stream=None) -> "Prepared":
+    ds = [_desc(x) for x in (q, k_cache, v_cache, block_tables, context_lens, groups.prefix_blocks,
+                             groups.group_start, groups.members, out)]
+    args = tuple(ctypes.byref(d) for d in ds[:8]) + (
+        groups.num_groups, groups.max_group_size, groups.max_prefix_blocks, int(num_kv_heads),
+        float(scale), int(block_size), ctypes.byref(ds[8]))
+    return Prepared("paged_attn_decode_cascade", lib().paged_attn_decode_cascade, args, (ds, groups), stream)
 
 
 def paged_attn_decode_fp8(q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,

@@ -1,0 +1,394 @@
+// Prefix-aware ("cascade") paged decode for sm_100a.
+//
+// Requests that share a system prompt point their block tables at the same
+// physical blocks ("PagedAttention: treat the cache like virtual memory" and
+// "Shared System Prompts & Prefix Caching"). The plain decode reads such a
+// block once per request; here it is read once per group: the query heads of
+// all members of a group become the N dimension of the prefix products, so
+// one K/V tile in shared memory serves every member.
+//
+// The result is the one paged_attn_decode defines: softmax over all tokens of
+// a sequence splits into the shared-prefix tokens and the rest, each side is
+// reduced to (running max m, sum l, unnormalised O) and the two are combined
+// with the log-sum-exp rule, the same way split-KV pieces are.
+//
+// Three steps, chained on one stream:
+//   1. decode_kernel over the tokens after the prefix (its table rows start
+//      skip[s] entries in); a sequence with a prefix leaves (m, l, O) per
+//      query head instead of an output row (decode_merge_kernel likewise).
+//   2. cascade_prefix_kernel: one CTA per (group, kv head, column chunk of 64
+//      query columns, chunk of prefix blocks). A column is one query head of
+//      one member (member-major). The CTA's 4 warps take 16 columns each; a
+//      ring of NS stages holds one prefix block's K and V tiles (TMA,
+//      128-byte swizzle) and every warp reads every stage. Per 16-token tile:
+//      S^T = K Q^T with two 8-column n-tiles per warp, online softmax per
+//      column, O^T += V^T P^T; partials (m, l, O) per column per chunk.
+//   3. cascade_merge_kernel: one warp per (member, query head) folds the
+//      prefix chunks' partials and the step-1 partial, normalises and writes
+//      the output row.
+#pragma once
+
+#include "decode.cuh"
+
+namespace pkv {
+
+constexpr int kCasCols = 64;  // query columns per prefix CTA (4 warps x 16)
+
+// Single-thread bounded wait on an mbarrier phase; false after `limit_ns`.
+__device__ __forceinline__ bool lane_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+  uint64_t t0 = 0;
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (it == 0) t0 = global_ns();
+    else if ((it & 63) == 0 && global_ns() - t0 > limit_ns) return false;
+  }
+}
+
+struct CascadeParams {
+  CUtensorMap tmk;  // K pool viewed as {D, B, Hk, NB}
+  CUtensorMap tmv;
+  const void* q;
+  long long q_s, q_h;
+  void* out;
+  long long o_s, o_h;
+  const int* tables;
+  long long t_s;
+  const int* prefix_blocks;  // [S]
+  const int* group_start;    // [G + 1]
+  const int* members;        // [M]
+  float scale_log2;
+  int S, Hk, g, NB, MB, G, M;
+  int ncc;  // column chunks per (group, kv head)
+  int nkc;  // prefix-block chunks per column chunk
+  int cb;   // prefix blocks per chunk
+  int* err;
+  float* pre_o;         // [G * Hk * ncc * nkc][kCasCols][D]
+  float* pre_ml;        // [G * Hk * ncc * nkc][kCasCols][2]
+  const float* suf_o;   // [S * Hq][D] step-1 partials
+  const float* suf_ml;  // [S * Hq][2]
+};
+
+template <bool QBF, int D, int BS, int NS>
+struct PrefixCfg {
+  static constexpr int EPR = 64;           // 16-bit elements per 128-byte row
+  static constexpr int NH = (D * 2) / 128;  // 128-byte column groups per token row
+  static constexpr int TILE = BS * D * 2;
+  static constexpr int STAGE = 2 * TILE;
+  static constexpr int KS = D / 16;
+  static constexpr int MT = D / 16;
+  static constexpr int TT = BS / 16;
+  static constexpr int SMEM = 1024 + NS * STAGE + 2 * NS * 8;
+  static_assert(D % 64 == 0, "head_dim must be a multiple of 64");
+  static_assert(BS % 16 == 0, "block_size must be a multiple of 16");
+};
+
+template <bool QBF, int D, int BS, int NS>
+__global__ void __launch_bounds__(128, 1) cascade_prefix_kernel(const __grid_constant__ CascadeParams p) {
+  using C = PrefixCfg<QBF, D, BS, NS>;
+  constexpr uint64_t kWaitNs = 2000000000ull;
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t sbase = (smem_addr(smem_raw) + 1023u) & ~1023u;
+  const uint32_t full = sbase + NS * C::STAGE;
+  const uint32_t empty = full + NS * 8;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int r = lane >> 2, c = lane & 3;
+  const int kc = blockIdx.x, cc = blockIdx.y;
+  const int gi = blockIdx.z / p.Hk, h = blockIdx.z % p.Hk;
+
+  pdl_launch_dependents();
+  if (tid == 0) {
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(full + i * 8, 1);
+      mbar_init(empty + i * 8, 4);
+    }
+    tma_prefetch_desc(&p.tmk);
+    tma_prefetch_desc(&p.tmv);
+  }
+  fence_mbar_init();
+  __syncthreads();
+  pdl_wait();
+
+  const int m0 = __ldg(p.group_start + gi), m1 = __ldg(p.group_start + gi + 1);
+  if (m0 < 0 || m1 < m0 || m1 > p.M) {
+    if (tid == 0) atomicOr(p.err, kErrBadLen);
+    return;
+  }
+  const int first = __ldg(p.members + m0);
+  if (first < 0 || first >= p.S) {
+    if (tid == 0) atomicOr(p.err, kErrBadLen);
+    return;
+  }
+  const int nb = __ldg(p.prefix_blocks + first);
+  if (nb < 0 || nb > p.MB) {
+    if (tid == 0) atomicOr(p.err, kErrBadLen);
+    return;
+  }
+  const int ncol = (m1 - m0) * p.g;
+  const int b_lo = kc * p.cb, b_hi = min(nb, b_lo + p.cb);
+  if (cc * kCasCols >= ncol || b_lo >= b_hi) return;  // nothing of this group here
+  const int n = b_hi - b_lo;
+
+  const uint64_t policy = l2_policy_evict_first();
+  auto issue = [&](int j) {  // thread 0: prefix block b_lo + j into stage j % NS
+    const int stage = j % NS;
+    int phys = __ldg(p.tables + first * p.t_s + b_lo + j);
+    if (phys < 0 || phys >= p.NB) {
+      atomicOr(p.err, kErrBadBlock);
+      phys = 0;
+    }
+    const uint32_t bar = full + stage * 8;
+    const uint32_t dk = sbase + stage * C::STAGE, dv = dk + C::TILE;
+    mbar_arrive_expect_tx(bar, C::STAGE);
+#pragma unroll
+    for (int hh = 0; hh < C::NH; ++hh)
+      tma_load_4d(dk + hh * BS * 128, &p.tmk, bar, hh * C::EPR, 0, h, phys, policy);
+#pragma unroll
+    for (int hh = 0; hh < C::NH; ++hh)
+      tma_load_4d(dv + hh * BS * 128, &p.tmv, bar, hh * C::EPR, 0, h, phys, policy);
+  };
+  if (tid == 0)
+    for (int j = 0; j < min(NS, n); ++j) issue(j);
+
+  // Q^T fragments of this warp's 16 columns: n-tile jt holds columns
+  // cc * 64 + warp * 16 + jt * 8 + (0..7); lane r carries column 8 jt + r.
+  uint32_t qb[2][C::KS][2];
+  bool col_ok[2][2];
+#pragma unroll
+  for (int jt = 0; jt < 2; ++jt) {
+    const int col = cc * kCasCols + warp * 16 + jt * 8 + r;
+    const bool ok = col < ncol;
+    const int mi = ok ? col / p.g : 0;
+    const int s = ok ? __ldg(p.members + m0 + mi) : 0;
+    const bool s_ok = ok && s >= 0 && s < p.S;
+    const uint32_t* qp = reinterpret_cast<const uint32_t*>(
+        static_cast<const uint16_t*>(p.q) + s * p.q_s + (static_cast<long long>(h) * p.g + col % p.g) * p.q_h);
+#pragma unroll
+    for (int ks = 0; ks < C::KS; ++ks) {
+      qb[jt][ks][0] = s_ok ? __ldg(qp + (ks * 16 + 2 * c) / 2) : 0u;
+      qb[jt][ks][1] = s_ok ? __ldg(qp + (ks * 16 + 8 + 2 * c) / 2) : 0u;
+    }
+    // the two accumulator columns of this lane: 8 jt + 2c and + 1
+    const int cb0 = cc * kCasCols + warp * 16 + jt * 8 + 2 * c;
+    col_ok[jt][0] = cb0 < ncol;
+    col_ok[jt][1] = cb0 + 1 < ncol;
+  }
+
+  float acc[2][C::MT][4];
+  float mrun[2][2], lrun[2][2];
+#pragma unroll
+  for (int jt = 0; jt < 2; ++jt) {
+#pragma unroll
+    for (int mt = 0; mt < C::MT; ++mt) acc[jt][mt][0] = acc[jt][mt][1] = acc[jt][mt][2] = acc[jt][mt][3] = 0.f;
+    mrun[jt][0] = mrun[jt][1] = -INFINITY;
+    lrun[jt][0] = lrun[jt][1] = 0.f;
+  }
+  const float sl = p.scale_log2;
+  bool failed = false;
+  int issued = min(NS, n);  // thread 0's count of blocks issued
+  int jfail = n;            // first block this warp gave up on
+
+  for (int j = 0; j < n; ++j) {
+    const int stage = j % NS;
+    const uint32_t parity = static_cast<uint32_t>((j / NS) & 1);
+    if (!warp_wait(full + stage * 8, parity, kWaitNs)) {
+      if (lane == 0) atomicOr(p.err, kErrWaitTimeout);
+      failed = true;
+      jfail = j;
+      break;
+    }
+    const uint32_t tk = sbase + stage * C::STAGE, tv = tk + C::TILE;
+#pragma unroll
+    for (int tt = 0; tt < C::TT; ++tt) {
+      // S^T = K Q^T for both n-tiles (K fragments shared)
+      float sacc[2][4];
+#pragma unroll
+      for (int jt = 0; jt < 2; ++jt) sacc[jt][0] = sacc[jt][1] = sacc[jt][2] = sacc[jt][3] = 0.f;
+      const int trow = tt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+      for (int ks = 0; ks < C::KS; ++ks) {
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(tk + swz<BS>(trow, ks * 32 + (lane >> 4) * 16), a0, a1, a2, a3);
+#pragma unroll
+        for (int jt = 0; jt < 2; ++jt) mma16816<QBF>(sacc[jt], a0, a1, a2, a3, qb[jt][ks][0], qb[jt][ks][1]);
+      }
+      // online softmax per column (every prefix token is valid)
+      uint32_t pb[2][2];
+#pragma unroll
+      for (int jt = 0; jt < 2; ++jt) {
+        float x0 = sacc[jt][0] * sl, x1 = sacc[jt][1] * sl, x2 = sacc[jt][2] * sl, x3 = sacc[jt][3] * sl;
+        float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+        }
+        const float mn0 = fmaxf(mrun[jt][0], mx0), mn1 = fmaxf(mrun[jt][1], mx1);
+        const float al0 = exp2f(mrun[jt][0] - mn0), al1 = exp2f(mrun[jt][1] - mn1);
+        lrun[jt][0] *= al0;
+        lrun[jt][1] *= al1;
+#pragma unroll
+        for (int mt = 0; mt < C::MT; ++mt) {
+          acc[jt][mt][0] *= al0;
+          acc[jt][mt][1] *= al1;
+          acc[jt][mt][2] *= al0;
+          acc[jt][mt][3] *= al1;
+        }
+        mrun[jt][0] = mn0;
+        mrun[jt][1] = mn1;
+        const float p0 = exp2f(x0 - mn0), p1 = exp2f(x1 - mn1);
+        const float p2 = exp2f(x2 - mn0), p3 = exp2f(x3 - mn1);
+        lrun[jt][0] += p0 + p2;
+        lrun[jt][1] += p1 + p3;
+        pb[jt][0] = movmatrix_t(pack2<QBF>(p0, p1));
+        pb[jt][1] = movmatrix_t(pack2<QBF>(p2, p3));
+      }
+      // O^T += V^T P^T (V fragments shared by both n-tiles)
+#pragma unroll
+      for (int i = 0; i < C::MT; ++i) {
+        const int vrow = tt * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
+        uint32_t f0, f1, f2, f3;
+        ldsm_x4_t(tv + swz<BS>(vrow, i * 32 + ((lane >> 3) & 1) * 16), f0, f1, f2, f3);
+#pragma unroll
+        for (int jt = 0; jt < 2; ++jt) mma16816<QBF>(acc[jt][i], f0, f1, f2, f3, pb[jt][0], pb[jt][1]);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty + stage * 8);
+    if (tid == 0 && j + NS < n) {
+      // the stage is refilled once all four warps have read it
+      if (!lane_wait(empty + stage * 8, parity, kWaitNs)) {
+        atomicOr(p.err, kErrWaitTimeout);
+      } else {
+        issue(j + NS);
+        ++issued;
+      }
+    }
+  }
+  if (failed) {
+    // let copies still in flight (issued, not yet waited for) land before the
+    // CTA's shared memory is reused
+    if (tid == 0)
+      for (int i = jfail; i < issued; ++i)
+        lane_wait(full + (i % NS) * 8, static_cast<uint32_t>((i / NS) & 1), 100000000ull);
+    return;
+  }
+
+  // partials of this chunk: one row of D floats (and m, l) per column
+  const long long item = ((static_cast<long long>(blockIdx.z) * p.ncc + cc) * p.nkc + kc);
+  float* po = p.pre_o + item * kCasCols * D;
+  float* pm = p.pre_ml + item * kCasCols * 2;
+#pragma unroll
+  for (int jt = 0; jt < 2; ++jt) {
+    float l0 = lrun[jt][0], l1 = lrun[jt][1];
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+    }
+    const int cl = warp * 16 + jt * 8 + 2 * c;  // column within the chunk
+#pragma unroll
+    for (int mt = 0; mt < C::MT; ++mt) {
+      const int da = 16 * mt + r, db = da + 8;
+      if (col_ok[jt][0]) {
+        po[cl * D + da] = acc[jt][mt][0];
+        po[cl * D + db] = acc[jt][mt][2];
+      }
+      if (col_ok[jt][1]) {
+        po[(cl + 1) * D + da] = acc[jt][mt][1];
+        po[(cl + 1) * D + db] = acc[jt][mt][3];
+      }
+    }
+    if (r == 0) {
+      if (col_ok[jt][0]) {
+        pm[cl * 2] = mrun[jt][0];
+        pm[cl * 2 + 1] = l0;
+      }
+      if (col_ok[jt][1]) {
+        pm[(cl + 1) * 2] = mrun[jt][1];
+        pm[(cl + 1) * 2 + 1] = l1;
+      }
+    }
+  }
+}
+
+// One warp per (member j, query head hq): fold the prefix chunks of j's group
+// and the partial of j's own tokens, normalise, write out[s, hq].
+template <bool QBF, int D>
+__global__ void __launch_bounds__(128) cascade_merge_kernel(const __grid_constant__ CascadeParams p) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int lane = threadIdx.x & 31;
+  const long long wid = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int Hq = p.Hk * p.g;
+  if (wid >= static_cast<long long>(p.M) * Hq) return;
+  const int j = static_cast<int>(wid / Hq), hq = static_cast<int>(wid % Hq);
+  // group of member j: the last g with group_start[g] <= j
+  int lo = 0, hi = p.G - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(p.group_start + mid) <= j) lo = mid;
+    else hi = mid - 1;
+  }
+  const int gi = lo;
+  const int s = __ldg(p.members + j);
+  if (s < 0 || s >= p.S) {
+    if (lane == 0) atomicOr(p.err, kErrBadLen);
+    return;
+  }
+  const int h = hq / p.g;
+  const int col = (j - __ldg(p.group_start + gi)) * p.g + hq % p.g;
+  const int cc = col / kCasCols, cl = col % kCasCols;
+  if (cc >= p.ncc) {  // a group larger than the launch was sized for
+    if (lane == 0) atomicOr(p.err, kErrBadLen);
+    return;
+  }
+  const int nb = __ldg(p.prefix_blocks + __ldg(p.members + __ldg(p.group_start + gi)));
+  const int nk = min(p.nkc, (max(nb, 0) + p.cb - 1) / p.cb);
+  const long long item0 = (static_cast<long long>(gi * p.Hk + h) * p.ncc + cc) * p.nkc;
+  const long long srow = static_cast<long long>(s) * Hq + hq;
+
+  // pieces: prefix chunks 0 .. nk-1, then the sequence's own partial (nk)
+  constexpr int V = D / 32;  // floats per lane
+  float mx = -INFINITY;
+  for (int k = lane; k <= nk; k += 32) {
+    const float m = k < nk ? p.pre_ml[((item0 + k) * kCasCols + cl) * 2] : p.suf_ml[srow * 2];
+    mx = fmaxf(mx, m);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  float lsum = 0.f, a[V];
+#pragma unroll
+  for (int v = 0; v < V; ++v) a[v] = 0.f;
+  if (mx != -INFINITY) {
+    for (int k = 0; k <= nk; ++k) {
+      const float* ml = k < nk ? p.pre_ml + ((item0 + k) * kCasCols + cl) * 2 : p.suf_ml + srow * 2;
+      const float* o = k < nk ? p.pre_o + ((item0 + k) * kCasCols + cl) * D : p.suf_o + srow * D;
+      const float m = ml[0];
+      if (m == -INFINITY) continue;
+      const float w = exp2f(m - mx);
+      lsum += ml[1] * w;
+      if constexpr (V == 4) {
+        const float4 x = reinterpret_cast<const float4*>(o)[lane];
+        a[0] += x.x * w;
+        a[1] += x.y * w;
+        a[2] += x.z * w;
+        a[3] += x.w * w;
+      } else {
+        const float2 x = reinterpret_cast<const float2*>(o)[lane];
+        a[0] += x.x * w;
+        a[1] += x.y * w;
+      }
+    }
+  }
+  const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+  uint16_t* oh = static_cast<uint16_t*>(p.out) + s * p.o_s + hq * p.o_h + lane * V;
+#pragma unroll
+  for (int v = 0; v < V; ++v) {
+    if constexpr (QBF) oh[v] = __bfloat16_as_ushort(__float2bfloat16_rn(a[v] * inv));
+    else oh[v] = __half_as_ushort(__float2half_rn(a[v] * inv));
+  }
+}
+
+}  // namespace pkv

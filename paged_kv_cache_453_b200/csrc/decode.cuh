@@ -80,6 +80,13 @@ struct DecodeParams {
   int4* desc;                 // [nwt][1 + kMaxSteals] last-piece descriptor per sub-range
   float* part_o;              // [2 nwt + pool_slots][g][D]
   float* part_ml;             // [2 nwt + pool_slots][g][2]
+  // Prefix-aware decode (null otherwise): the first skip[s] table entries of
+  // sequence s are a shared prefix attended elsewhere; its remaining tokens
+  // leave fp32 partials (m, l, unnormalised O) per query head in cas_o /
+  // cas_ml instead of an output row when skip[s] > 0.
+  const int* skip;            // [S] blocks
+  float* cas_o;               // [S * Hq][D]
+  float* cas_ml;              // [S * Hq][2]
 };
 
 __device__ __forceinline__ uint64_t global_ns() {
@@ -125,15 +132,36 @@ __device__ __forceinline__ int items_of(int L) {
   return n > 0 ? n : 1;
 }
 
+// Tokens of sequence s this kernel attends (its context length clamped to the
+// table row, minus a shared prefix of sk blocks), and sk.
+template <int BS>
+__device__ __forceinline__ int seq_len(const DecodeParams& p, int s, int max_len, int& sk,
+                                       bool report) {
+  int len = __ldg(p.lens + s);
+  bool bad = len < 0 || len > max_len;
+  len = len < 0 ? 0 : (len > max_len ? max_len : len);
+  sk = 0;
+  if (p.skip) {
+    sk = __ldg(p.skip + s);
+    if (sk < 0 || sk * BS > len) {
+      bad = true;
+      sk = sk < 0 ? 0 : len / BS;
+    }
+  }
+  if (bad && report) atomicOr(p.err, kErrBadLen);
+  return len - sk * BS;
+}
+
 __device__ __forceinline__ long long range_lo(long long w, long long W, int nwt) {
   return (w * W) / nwt;
 }
 
-template <int BS>
+template <int BS, int TOK>
 struct Cursor {
   long long k;  // global item index
-  int s, h, b;  // sequence, kv head, block within the unit
-  int L, n;     // context length of s, items per unit of s
+  int s, h, b;  // sequence, kv head, item within the unit
+  int L, n;     // tokens of s attended here, items per unit of s
+  int sk;       // table entries of s skipped (shared prefix)
 
   __device__ __forceinline__ void advance(const DecodeParams& p, int max_len) {
     ++k;
@@ -142,9 +170,8 @@ struct Cursor {
       if (++h == p.Hk) {
         h = 0;
         if (++s < p.S) {
-          int len = __ldg(p.lens + s);
-          L = len < 0 ? 0 : (len > max_len ? max_len : len);
-          n = items_of<BS>(L);
+          L = seq_len<BS>(p, s, max_len, sk, false);
+          n = items_of<TOK>(L);
         }
       }
     }
@@ -229,11 +256,8 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
     const int s1 = static_cast<int>((static_cast<long long>(tid + 1) * p.S) / C::NT);
     long long sum = 0;
     for (int s = s0; s < s1; ++s) {
-      int len = __ldg(p.lens + s);
-      if (len < 0 || len > max_len) {
-        if (blockIdx.x == 0) atomicOr(p.err, kErrBadLen);
-        len = len < 0 ? 0 : max_len;
-      }
+      int sk;
+      const int len = seq_len<BS>(p, s, max_len, sk, blockIdx.x == 0);
       sum += static_cast<long long>(p.Hk) * items_of<TOK>(len);
     }
     long long v = sum;  // inclusive warp scan, then warp totals
@@ -270,7 +294,7 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
   if (lane == 0) p.desc[gw * (1 + kMaxSteals)] = make_int4(-1, 0, 0, 0);
 
   // Position of global item x: chunk by binary search, then a warp-wide walk.
-  auto locate = [&](long long x, Cursor<TOK>& out) -> bool {
+  auto locate = [&](long long x, Cursor<BS, TOK>& out) -> bool {
     int a = 0, bnd = C::NT - 1;
     while (a < bnd) {  // largest t with scan[t] <= x
       int m = (a + bnd + 1) >> 1;
@@ -282,11 +306,10 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
     long long base = scan[a];
     for (int s0 = s_lo; s0 < s_hi; s0 += 32) {
       const int s = s0 + lane;
-      int len = 0;
+      int len = 0, sk = 0;
       long long w = 0;
       if (s < s_hi) {
-        len = __ldg(p.lens + s);
-        len = len < 0 ? 0 : (len > max_len ? max_len : len);
+        len = seq_len<BS>(p, s, max_len, sk, false);
         w = static_cast<long long>(p.Hk) * items_of<TOK>(len);
       }
       long long incl = w;
@@ -300,6 +323,7 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
         const int j = __ffs(hit) - 1;
         const long long start = __shfl_sync(0xffffffffu, base + incl - w, j);
         const int L = __shfl_sync(0xffffffffu, len, j);
+        out.sk = __shfl_sync(0xffffffffu, sk, j);
         const int n = items_of<TOK>(L);
         const long long off = x - start;
         out.k = x;
@@ -337,12 +361,12 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
   // hi drops to where thieves took over. Partials go to slots slot_base (+1).
   auto run_range = [&](long long a, long long hi, bool claim, int owner, int sub,
                        long long slot_base) -> bool {
-    Cursor<TOK> cur;
+    Cursor<BS, TOK> cur;
     if (!locate(a, cur)) {
       if (lane == 0) atomicOr(p.err, kErrBadLen);
       return false;
     }
-    Cursor<TOK> pc = cur;
+    Cursor<BS, TOK> pc = cur;
     const long long lo = a;
 
     unsigned long long* wp = p.words + owner;
@@ -363,7 +387,7 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
       if (pc.s != tw_s || b0 < tw_b0 || b0 + nload > tw_b0 + 32) {
         tw_s = pc.s;
         tw_b0 = b0;
-        tw_val = (tw_b0 + lane < nb) ? __ldg(p.tables + pc.s * p.t_s + tw_b0 + lane) : 0;
+        tw_val = (tw_b0 + lane < nb) ? __ldg(p.tables + pc.s * p.t_s + pc.sk + tw_b0 + lane) : 0;
       }
       int phys[IB];
 #pragma unroll
@@ -473,7 +497,36 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
       if constexpr (FP8) vs = __ldg(p.v_scale + cur.h);
       const long long ub = cur.unit_begin(), ue = cur.unit_end();
       const int hq0 = cur.h * p.g + 2 * c;
-      if (ub >= lo && ue <= hi) {  // whole unit in this sub-range: final output
+      if (ub >= lo && ue <= hi && cur.sk > 0) {
+        // whole unit of a sequence with a shared prefix: its partial goes to
+        // the prefix-aware merge
+        const long long row = static_cast<long long>(cur.s) * p.g * p.Hk + hq0;
+        float* po = p.cas_o + row * D;
+#pragma unroll
+        for (int mt = 0; mt < C::MT; ++mt) {
+          const int da = FP8 ? 16 * mt + 2 * r : 16 * mt + r;
+          const int db = FP8 ? da + 1 : da + 8;
+          if (h0_ok) {
+            po[da] = acc[mt][0] * vs;
+            po[db] = acc[mt][2] * vs;
+          }
+          if (h1_ok) {
+            po[D + da] = acc[mt][1] * vs;
+            po[D + db] = acc[mt][3] * vs;
+          }
+        }
+        if (r == 0) {
+          float* pm = p.cas_ml + row * 2;
+          if (h0_ok) {
+            pm[0] = m0;
+            pm[1] = l0;
+          }
+          if (h1_ok) {
+            pm[2] = m1;
+            pm[3] = l1;
+          }
+        }
+      } else if (ub >= lo && ue <= hi) {  // whole unit in this sub-range: final output
         const float i0 = l0 > 0.f ? vs / l0 : 0.f;
         const float i1 = l1 > 0.f ? vs / l1 : 0.f;
         uint16_t* o = static_cast<uint16_t*>(p.out) + cur.s * p.o_s;
@@ -978,7 +1031,17 @@ __global__ void __launch_bounds__(128, 8) decode_merge_kernel(const __grid_const
         }
       }
     }
-    if (pg == 0) {
+    const bool cascade = p.skip != nullptr && __ldg(p.skip + s) > 0;
+    if (pg == 0 && cascade) {  // partial of a sequence with a shared prefix
+      const long long row = static_cast<long long>(s) * g * p.Hk + static_cast<long long>(h) * g + hi8;
+      float4* po = reinterpret_cast<float4*>(p.cas_o + row * D + d8);
+      po[0] = make_float4(ra[0], ra[1], ra[2], ra[3]);
+      po[1] = make_float4(ra[4], ra[5], ra[6], ra[7]);
+      if (d8 == 0) {
+        p.cas_ml[row * 2] = rm;
+        p.cas_ml[row * 2 + 1] = rl;
+      }
+    } else if (pg == 0) {
       const float inv = rl > 0.f ? 1.f / rl : 0.f;
       uint16_t* oh = static_cast<uint16_t*>(p.out) + s * p.o_s +
                      (static_cast<long long>(h) * g + hi8) * p.o_h + d8;

@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -15,6 +16,7 @@
 
 #include "../../include/pagedkv.h"
 #include "cache_ops.cuh"
+#include "cascade.cuh"
 #include "decode.cuh"
 
 namespace pkv {
@@ -32,6 +34,8 @@ struct DeviceState {
   int* err = nullptr;  // device address of g_pkv_err
   void* ws = nullptr;  // library-owned decode workspace
   size_t ws_bytes = 0;
+  void* cas = nullptr;  // library-owned prefix-aware decode partials
+  size_t cas_bytes = 0;
 };
 DeviceState g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -330,12 +334,21 @@ int check_decode(const DecodeArgs& a, bool fp8, int* ck_out, DecodeLaunch** entr
   return *entry ? PKV_OK : PKV_ERR_UNSUPPORTED;
 }
 
+// Prefix-aware decode: table entries each sequence skips, and where the
+// sequences with a prefix leave their partials.
+struct CascadeTail {
+  const int* skip;
+  float* o;
+  float* ml;
+};
+
 // Launch decode + merge. lib_ws: use (and grow) the library's workspace for
 // this device; otherwise `ws` is the caller's. fit: shrink the steal-slot pool
 // to fit ws_bytes; clear: zero the claim state first (callers that cannot
 // vouch for it).
 int launch_decode(const DecodeArgs& a, bool fp8, void* ws, size_t ws_bytes, bool lib_ws,
-                  cudaStream_t stream, bool fit = false, bool clear = false) {
+                  cudaStream_t stream, bool fit = false, bool clear = false,
+                  const CascadeTail* tail = nullptr) {
   int ck = 0;
   DecodeLaunch* e = nullptr;
   int st = check_decode(a, fp8, &ck, &e);
@@ -401,6 +414,11 @@ int launch_decode(const DecodeArgs& a, bool fp8, void* ws, size_t ws_bytes, bool
   p.desc = reinterpret_cast<int4*>(w + L.desc);
   p.part_o = reinterpret_cast<float*>(w + L.part_o);
   p.part_ml = reinterpret_cast<float*>(w + L.part_ml);
+  if (tail) {
+    p.skip = tail->skip;
+    p.cas_o = tail->o;
+    p.cas_ml = tail->ml;
+  }
 
   // Both kernels are launched as programmatic dependents of the kernel
   // before them in the stream: their CTAs can be resident before it ends and
@@ -420,6 +438,161 @@ int launch_decode(const DecodeArgs& a, bool fp8, void* ws, size_t ws_bytes, bool
   cfg.blockDim = dim3(128);
   cfg.dynamicSmemBytes = 0;
   if (cudaLaunchKernelEx(&cfg, e->merge, p) != cudaSuccess) return PKV_ERR_CUDA;
+  return PKV_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Prefix-aware decode
+// ---------------------------------------------------------------------------
+
+struct CascadeLaunch {
+  void (*prefix)(CascadeParams);
+  void (*merge)(CascadeParams);
+  int smem;
+  bool attr_set[kMaxDevices];
+};
+
+template <bool QBF, int D, int BS>
+CascadeLaunch* cascade_entry() {
+  constexpr int NS = 4;
+  static CascadeLaunch e = {&cascade_prefix_kernel<QBF, D, BS, NS>, &cascade_merge_kernel<QBF, D>,
+                            PrefixCfg<QBF, D, BS, NS>::SMEM, {false}};
+  return &e;
+}
+
+CascadeLaunch* pick_cascade(bool qbf, int D, int BS) {
+  if (qbf) {
+    if (D == 128 && BS == 16) return cascade_entry<true, 128, 16>();
+    if (D == 128 && BS == 32) return cascade_entry<true, 128, 32>();
+    if (D == 64 && BS == 16) return cascade_entry<true, 64, 16>();
+    if (D == 64 && BS == 32) return cascade_entry<true, 64, 32>();
+  } else {
+    if (D == 128 && BS == 16) return cascade_entry<false, 128, 16>();
+    if (D == 128 && BS == 32) return cascade_entry<false, 128, 32>();
+    if (D == 64 && BS == 16) return cascade_entry<false, 64, 16>();
+    if (D == 64 && BS == 32) return cascade_entry<false, 64, 32>();
+  }
+  return nullptr;
+}
+
+int launch_cascade(const DecodeArgs& a, const pkv_tensor* pblk, const pkv_tensor* gstart,
+                   const pkv_tensor* gmem, int G, int max_members, int max_prefix,
+                   cudaStream_t stream) {
+  int ck = 0;
+  DecodeLaunch* e = nullptr;
+  int st = check_decode(a, false, &ck, &e);
+  if (st != PKV_OK) return st;
+  if (!pblk || !gstart || !gmem || G < 0 || max_members < 0 || max_prefix < 0)
+    return PKV_ERR_INVALID_ARG;
+  const int64_t S = a.q->shape[0];
+  if (!well_formed(pblk, 1, PKV_I32) || pblk->shape[0] != S || (S > 0 && pblk->stride[0] != 1))
+    return PKV_ERR_INVALID_ARG;
+  if (!well_formed(gstart, 1, PKV_I32) || gstart->shape[0] != G + 1 || gstart->stride[0] != 1)
+    return PKV_ERR_INVALID_ARG;
+  if (!well_formed(gmem, 1, PKV_I32) || (gmem->shape[0] > 0 && gmem->stride[0] != 1) ||
+      gmem->shape[0] > S || gmem->shape[0] > INT32_MAX)
+    return PKV_ERR_INVALID_ARG;
+  const int M = static_cast<int>(gmem->shape[0]);
+  if (!e) return PKV_OK;  // S == 0
+  if (max_prefix > a.bt->shape[1] || max_members > S || (G > 0 && (max_members < 1 || M < 1)))
+    return PKV_ERR_INVALID_ARG;
+  const int D = static_cast<int>(a.q->shape[2]);
+  const int g = static_cast<int>(a.q->shape[1] / a.Hk);
+  CascadeLaunch* ce = pick_cascade(a.q->dtype == PKV_BF16, D, a.BS);
+  if (!ce) return PKV_ERR_UNSUPPORTED;
+  int dev;
+  if ((st = current_device(&dev)) != PKV_OK) return st;
+  DeviceState* ds;
+  if ((st = device_state(dev, &ds)) != PKV_OK) return st;
+
+  // prefix chunks: about two CTAs per SM over all (group, head, column chunk)
+  const int ncc = std::max(1, (max_members * g + kCasCols - 1) / kCasCols);
+  const long long pairs = static_cast<long long>(G) * a.Hk * ncc * std::max(max_prefix, 1);
+  int cb = static_cast<int>((pairs + 2LL * ds->sms - 1) / (2LL * ds->sms));
+  cb = std::max(cb, std::min(4, std::max(max_prefix, 1)));
+  const int nkc = std::max(1, (max_prefix + cb - 1) / cb);
+  const long long items = static_cast<long long>(G) * a.Hk * ncc * nkc;
+  const int Hq = a.Hk * g;
+  const size_t suf_o = 0;
+  const size_t suf_ml = round_up(suf_o + static_cast<size_t>(S) * Hq * D * 4, 256);
+  const size_t pre_o = round_up(suf_ml + static_cast<size_t>(S) * Hq * 2 * 4, 256);
+  const size_t pre_ml = round_up(pre_o + static_cast<size_t>(items) * kCasCols * D * 4, 256);
+  const size_t total = round_up(pre_ml + static_cast<size_t>(items) * kCasCols * 2 * 4, 256);
+  if (nkc > 65535 || ncc > 65535 || static_cast<long long>(G) * a.Hk > 65535)
+    return PKV_ERR_UNSUPPORTED;
+  uint8_t* cw;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (ds->cas_bytes < total) {
+      if (ds->cas) cudaFree(ds->cas);
+      ds->cas = nullptr;
+      ds->cas_bytes = 0;
+      if (cudaMalloc(&ds->cas, total) != cudaSuccess) return PKV_ERR_CUDA;
+      ds->cas_bytes = total;
+    }
+    cw = static_cast<uint8_t*>(ds->cas);
+    if (!ce->attr_set[dev]) {
+      if (cudaFuncSetAttribute(ce->prefix, cudaFuncAttributeMaxDynamicSharedMemorySize, ce->smem) !=
+          cudaSuccess)
+        return PKV_ERR_CUDA;
+      ce->attr_set[dev] = true;
+    }
+  }
+  CascadeTail tail{static_cast<const int*>(pblk->data), reinterpret_cast<float*>(cw + suf_o),
+                   reinterpret_cast<float*>(cw + suf_ml)};
+  if ((st = launch_decode(a, false, nullptr, 0, true, stream, false, false, &tail)) != PKV_OK)
+    return st;
+  if (G == 0 || M == 0) return PKV_OK;
+
+  CascadeParams p;
+  std::memset(&p, 0, sizeof(p));
+  if ((st = encode_pool_map(&p.tmk, a.kc, a.q->dtype)) != PKV_OK) return st;
+  if ((st = encode_pool_map(&p.tmv, a.vc, a.q->dtype)) != PKV_OK) return st;
+  p.q = a.q->data;
+  p.q_s = a.q->stride[0];
+  p.q_h = a.q->stride[1];
+  p.out = a.out->data;
+  p.o_s = a.out->stride[0];
+  p.o_h = a.out->stride[1];
+  p.tables = static_cast<const int*>(a.bt->data);
+  p.t_s = a.bt->stride[0];
+  p.prefix_blocks = static_cast<const int*>(pblk->data);
+  p.group_start = static_cast<const int*>(gstart->data);
+  p.members = static_cast<const int*>(gmem->data);
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+  p.S = static_cast<int>(S);
+  p.Hk = a.Hk;
+  p.g = g;
+  p.NB = static_cast<int>(a.kc->shape[0]);
+  p.MB = static_cast<int>(a.bt->shape[1]);
+  p.G = G;
+  p.M = M;
+  p.ncc = ncc;
+  p.nkc = nkc;
+  p.cb = cb;
+  p.err = ds->err;
+  p.pre_o = reinterpret_cast<float*>(cw + pre_o);
+  p.pre_ml = reinterpret_cast<float*>(cw + pre_ml);
+  p.suf_o = reinterpret_cast<const float*>(cw + suf_o);
+  p.suf_ml = reinterpret_cast<const float*>(cw + suf_ml);
+
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(nkc), static_cast<unsigned>(ncc),
+                     static_cast<unsigned>(G * a.Hk));
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = static_cast<size_t>(ce->smem);
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, ce->prefix, p) != cudaSuccess) return PKV_ERR_CUDA;
+  const long long warps = static_cast<long long>(M) * Hq;
+  if ((warps + 3) / 4 > INT32_MAX) return PKV_ERR_UNSUPPORTED;
+  cfg.gridDim = dim3(static_cast<unsigned>((warps + 3) / 4));
+  cfg.dynamicSmemBytes = 0;
+  if (cudaLaunchKernelEx(&cfg, ce->merge, p) != cudaSuccess) return PKV_ERR_CUDA;
   return PKV_OK;
 }
 
@@ -565,6 +738,19 @@ int paged_attn_decode_fp8(const pkv_tensor* q, const pkv_tensor* k_cache,
   DecodeArgs a{q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
                num_kv_heads, scale, block_size, out};
   return launch_decode(a, true, nullptr, 0, true, static_cast<cudaStream_t>(stream));
+}
+
+int paged_attn_decode_cascade(const pkv_tensor* q, const pkv_tensor* k_cache,
+                              const pkv_tensor* v_cache, const pkv_tensor* block_tables,
+                              const pkv_tensor* context_lens, const pkv_tensor* prefix_blocks,
+                              const pkv_tensor* group_start, const pkv_tensor* group_members,
+                              int num_groups, int max_group_size, int max_prefix_blocks,
+                              int num_kv_heads, float scale, int block_size, pkv_tensor* out,
+                              void* stream) {
+  DecodeArgs a{q, k_cache, v_cache, nullptr, nullptr, block_tables, context_lens,
+               num_kv_heads, scale, block_size, out};
+  return launch_cascade(a, prefix_blocks, group_start, group_members, num_groups, max_group_size,
+                        max_prefix_blocks, static_cast<cudaStream_t>(stream));
 }
 
 size_t paged_attn_decode_workspace_bytes(int num_q_heads, int num_kv_heads, int head_dim,
