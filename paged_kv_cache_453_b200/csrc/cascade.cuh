@@ -33,6 +33,7 @@
 namespace pkv {
 
 constexpr int kCasCols = 64;  // query columns per prefix CTA (4 warps x 16)
+constexpr int kCasMaxChunk = 256;  // prefix blocks per chunk, at most
 
 // Single-thread bounded wait on an mbarrier phase; false after `limit_ns`.
 __device__ __forceinline__ bool lane_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
@@ -77,7 +78,7 @@ struct PrefixCfg {
   static constexpr int KS = D / 16;
   static constexpr int MT = D / 16;
   static constexpr int TT = BS / 16;
-  static constexpr int SMEM = 1024 + NS * STAGE + 2 * NS * 8;
+  static constexpr int SMEM = 1024 + NS * STAGE + 2 * NS * 8 + kCasMaxChunk * 4;
   static_assert(D % 64 == 0, "head_dim must be a multiple of 64");
   static_assert(BS % 16 == 0, "block_size must be a multiple of 16");
 };
@@ -91,13 +92,22 @@ __global__ void __launch_bounds__(128, 1) cascade_prefix_kernel(const __grid_con
   const uint32_t sbase = (smem_addr(smem_raw) + 1023u) & ~1023u;
   const uint32_t full = sbase + NS * C::STAGE;
   const uint32_t empty = full + NS * 8;
+  int* s_phys = reinterpret_cast<int*>(smem_raw + (sbase - smem_addr(smem_raw)) + NS * C::STAGE + 2 * NS * 8);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int r = lane >> 2, c = lane & 3;
   const int kc = blockIdx.x, cc = blockIdx.y;
   const int gi = blockIdx.z / p.Hk, h = blockIdx.z % p.Hk;
 
+  // This grid is launched once the decode grid has finished (the split-KV
+  // merge before it releases its dependents only after its own wait), so
+  // the inputs read here are final; it reads nothing the merge writes.
+  // griddepcontrol.wait runs at exit, so that this grid finishing implies the
+  // merge finished (the prefix merge after it reads the merge's partials).
   pdl_launch_dependents();
+  struct WaitAtExit {
+    __device__ ~WaitAtExit() { pdl_wait(); }
+  } wait_at_exit;
   if (tid == 0) {
     for (int i = 0; i < NS; ++i) {
       mbar_init(full + i * 8, 1);
@@ -107,8 +117,6 @@ __global__ void __launch_bounds__(128, 1) cascade_prefix_kernel(const __grid_con
     tma_prefetch_desc(&p.tmv);
   }
   fence_mbar_init();
-  __syncthreads();
-  pdl_wait();
 
   const int m0 = __ldg(p.group_start + gi), m1 = __ldg(p.group_start + gi + 1);
   if (m0 < 0 || m1 < m0 || m1 > p.M) {
@@ -121,7 +129,7 @@ __global__ void __launch_bounds__(128, 1) cascade_prefix_kernel(const __grid_con
     return;
   }
   const int nb = __ldg(p.prefix_blocks + first);
-  if (nb < 0 || nb > p.MB) {
+  if (nb < 0 || nb > p.MB || p.cb > kCasMaxChunk) {
     if (tid == 0) atomicOr(p.err, kErrBadLen);
     return;
   }
@@ -129,15 +137,20 @@ __global__ void __launch_bounds__(128, 1) cascade_prefix_kernel(const __grid_con
   const int b_lo = kc * p.cb, b_hi = min(nb, b_lo + p.cb);
   if (cc * kCasCols >= ncol || b_lo >= b_hi) return;  // nothing of this group here
   const int n = b_hi - b_lo;
-
-  const uint64_t policy = l2_policy_evict_first();
-  auto issue = [&](int j) {  // thread 0: prefix block b_lo + j into stage j % NS
-    const int stage = j % NS;
+  for (int j = tid; j < n; j += 128) {  // the chunk's physical blocks, checked
     int phys = __ldg(p.tables + first * p.t_s + b_lo + j);
     if (phys < 0 || phys >= p.NB) {
       atomicOr(p.err, kErrBadBlock);
       phys = 0;
     }
+    s_phys[j] = phys;
+  }
+  __syncthreads();
+
+  const uint64_t policy = l2_policy_evict_first();
+  auto issue = [&](int j) {  // thread 0: prefix block b_lo + j into stage j % NS
+    const int stage = j % NS;
+    const int phys = s_phys[j];
     const uint32_t bar = full + stage * 8;
     const uint32_t dk = sbase + stage * C::STAGE, dv = dk + C::TILE;
     mbar_arrive_expect_tx(bar, C::STAGE);
@@ -313,73 +326,103 @@ __global__ void __launch_bounds__(128, 1) cascade_prefix_kernel(const __grid_con
   }
 }
 
-// One warp per (member j, query head hq): fold the prefix chunks of j's group
-// and the partial of j's own tokens, normalise, write out[s, hq].
+// One warp per (member j, query head hq), grid (members x heads, groups):
+// fold the prefix chunks of j's group and the partial of j's own tokens,
+// normalise, write out[s, hq].
 template <bool QBF, int D>
 __global__ void __launch_bounds__(128) cascade_merge_kernel(const __grid_constant__ CascadeParams p) {
-  pdl_wait();
+  // The group data are inputs of the call: read them before waiting for the
+  // prefix grid (and through it the split-KV merge), whose partials follow.
+  // Every thread waits before it exits, so this grid finishing implies the
+  // kernels before it finished.
   pdl_launch_dependents();
+  struct WaitAtExit {
+    __device__ ~WaitAtExit() { pdl_wait(); }
+  } wait_at_exit;
   const int lane = threadIdx.x & 31;
   const long long wid = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int Hq = p.Hk * p.g;
-  if (wid >= static_cast<long long>(p.M) * Hq) return;
-  const int j = static_cast<int>(wid / Hq), hq = static_cast<int>(wid % Hq);
-  // group of member j: the last g with group_start[g] <= j
-  int lo = 0, hi = p.G - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (__ldg(p.group_start + mid) <= j) lo = mid;
-    else hi = mid - 1;
+  const int gi = blockIdx.y;
+  const int m0 = __ldg(p.group_start + gi), m1 = __ldg(p.group_start + gi + 1);
+  if (blockIdx.x == 0 && threadIdx.x == 0 &&
+      static_cast<long long>(m1 - m0) * Hq > static_cast<long long>(gridDim.x) * (blockDim.x >> 5))
+    atomicOr(p.err, kErrBadLen);  // a group larger than max_group_size
+  if (wid >= static_cast<long long>(m1 - m0) * Hq) return;
+  const int jl = static_cast<int>(wid / Hq), hq = static_cast<int>(wid % Hq);
+  if (m0 < 0 || m1 > p.M) {
+    if (lane == 0) atomicOr(p.err, kErrBadLen);
+    return;
   }
-  const int gi = lo;
-  const int s = __ldg(p.members + j);
+  const int s = __ldg(p.members + m0 + jl);
   if (s < 0 || s >= p.S) {
     if (lane == 0) atomicOr(p.err, kErrBadLen);
     return;
   }
   const int h = hq / p.g;
-  const int col = (j - __ldg(p.group_start + gi)) * p.g + hq % p.g;
+  const int col = jl * p.g + hq % p.g;
   const int cc = col / kCasCols, cl = col % kCasCols;
   if (cc >= p.ncc) {  // a group larger than the launch was sized for
     if (lane == 0) atomicOr(p.err, kErrBadLen);
     return;
   }
-  const int nb = __ldg(p.prefix_blocks + __ldg(p.members + __ldg(p.group_start + gi)));
+  const int nb = __ldg(p.prefix_blocks + s);  // equal for all members
   const int nk = min(p.nkc, (max(nb, 0) + p.cb - 1) / p.cb);
   const long long item0 = (static_cast<long long>(gi * p.Hk + h) * p.ncc + cc) * p.nkc;
   const long long srow = static_cast<long long>(s) * Hq + hq;
+  pdl_wait();  // (a second wait at exit returns at once)
 
-  // pieces: prefix chunks 0 .. nk-1, then the sequence's own partial (nk)
+  // pieces: prefix chunks 0 .. nk-1, then the sequence's own partial (nk).
+  // Lane k holds piece base + k's (m, l); all row loads of a batch are in
+  // flight together.
   constexpr int V = D / 32;  // floats per lane
-  float mx = -INFINITY;
-  for (int k = lane; k <= nk; k += 32) {
-    const float m = k < nk ? p.pre_ml[((item0 + k) * kCasCols + cl) * 2] : p.suf_ml[srow * 2];
-    mx = fmaxf(mx, m);
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  float lsum = 0.f, a[V];
+  float mx = -INFINITY, lsum = 0.f, a[V];
 #pragma unroll
   for (int v = 0; v < V; ++v) a[v] = 0.f;
-  if (mx != -INFINITY) {
-    for (int k = 0; k <= nk; ++k) {
+  for (int base = 0; base <= nk; base += 32) {
+    const int k = base + lane;
+    float m = -INFINITY, l = 0.f;
+    if (k <= nk) {
       const float* ml = k < nk ? p.pre_ml + ((item0 + k) * kCasCols + cl) * 2 : p.suf_ml + srow * 2;
-      const float* o = k < nk ? p.pre_o + ((item0 + k) * kCasCols + cl) * D : p.suf_o + srow * D;
-      const float m = ml[0];
-      if (m == -INFINITY) continue;
-      const float w = exp2f(m - mx);
-      lsum += ml[1] * w;
-      if constexpr (V == 4) {
-        const float4 x = reinterpret_cast<const float4*>(o)[lane];
-        a[0] += x.x * w;
-        a[1] += x.y * w;
-        a[2] += x.z * w;
-        a[3] += x.w * w;
-      } else {
-        const float2 x = reinterpret_cast<const float2*>(o)[lane];
-        a[0] += x.x * w;
-        a[1] += x.y * w;
+      m = ml[0];
+      l = ml[1];
+    }
+    float cm = m;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, o));
+    if (cm == -INFINITY) continue;  // nothing in this batch
+    const float mn = fmaxf(mx, cm);
+    const float sa = mx == -INFINITY ? 0.f : exp2f(mx - mn);
+    lsum *= sa;
+#pragma unroll
+    for (int v = 0; v < V; ++v) a[v] *= sa;
+    mx = mn;
+    const float w = m == -INFINITY ? 0.f : exp2f(m - mn);
+    float lw = l * w;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, o);
+    lsum += lw;
+    const int cnt = min(32, nk + 1 - base);
+    for (int k0 = 0; k0 < cnt; k0 += 8) {
+      float x[8][V];
+      float wk[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int kk = base + k0 + u;
+        wk[u] = __shfl_sync(0xffffffffu, w, (k0 + u) & 31);
+        if (k0 + u < cnt && wk[u] != 0.f) {
+          const float* o = kk < nk ? p.pre_o + ((item0 + kk) * kCasCols + cl) * D : p.suf_o + srow * D;
+#pragma unroll
+          for (int v = 0; v < V; ++v) x[u][v] = o[lane * V + v];
+        } else {
+#pragma unroll
+          for (int v = 0; v < V; ++v) x[u][v] = 0.f;
+          wk[u] = 0.f;
+        }
       }
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+#pragma unroll
+        for (int v = 0; v < V; ++v) a[v] += x[u][v] * wk[u];
     }
   }
   const float inv = lsum > 0.f ? 1.f / lsum : 0.f;

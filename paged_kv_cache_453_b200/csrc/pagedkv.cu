@@ -509,7 +509,7 @@ int launch_cascade(const DecodeArgs& a, const pkv_tensor* pblk, const pkv_tensor
   const int ncc = std::max(1, (max_members * g + kCasCols - 1) / kCasCols);
   const long long pairs = static_cast<long long>(G) * a.Hk * ncc * std::max(max_prefix, 1);
   int cb = static_cast<int>((pairs + 2LL * ds->sms - 1) / (2LL * ds->sms));
-  cb = std::max(cb, std::min(4, std::max(max_prefix, 1)));
+  cb = std::min(std::max(cb, std::min(4, std::max(max_prefix, 1))), kCasMaxChunk);
   const int nkc = std::max(1, (max_prefix + cb - 1) / cb);
   const long long items = static_cast<long long>(G) * a.Hk * ncc * nkc;
   const int Hq = a.Hk * g;
@@ -588,9 +588,9 @@ int launch_cascade(const DecodeArgs& a, const pkv_tensor* pblk, const pkv_tensor
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, ce->prefix, p) != cudaSuccess) return PKV_ERR_CUDA;
-  const long long warps = static_cast<long long>(M) * Hq;
-  if ((warps + 3) / 4 > INT32_MAX) return PKV_ERR_UNSUPPORTED;
-  cfg.gridDim = dim3(static_cast<unsigned>((warps + 3) / 4));
+  const long long warps = static_cast<long long>(max_members) * Hq;
+  if ((warps + 3) / 4 > INT32_MAX || G > 65535) return PKV_ERR_UNSUPPORTED;
+  cfg.gridDim = dim3(static_cast<unsigned>((warps + 3) / 4), static_cast<unsigned>(G));
   cfg.dynamicSmemBytes = 0;
   if (cudaLaunchKernelEx(&cfg, ce->merge, p) != cudaSuccess) return PKV_ERR_CUDA;
   return PKV_OK;
