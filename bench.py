@@ -55,6 +55,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--op", default="decode", choices=["decode", "swap"],
+                    help="swap: time preemption by swapping (blocks to page-locked host memory and back)")
     ap.add_argument("--no-cascade", action="store_true",
                     help="decode a shared-prefix workload with the plain decode")
     return ap.parse_args()
@@ -338,9 +340,73 @@ def run_reference(a, s: W.Spec, ws: int, rank: int):
     }))
 
 
+def run_swap(a, s: W.Spec):
+    """Swap a quarter of the workload's sequences out to page-locked host
+    memory and back into other blocks, per step; compared with torch's own
+    device<->pinned-host copies of the same bytes (the host link's rate)."""
+    import paged_kv_cache_453_b200 as P
+    from paged_kv_cache_453_b200.build import build
+    build()
+    torch.cuda.set_device(0)
+    lay = W.make_layout(s.replace(append=False))
+    t = W.make_tensors(s.replace(append=False), lay.num_blocks, lay.tables, lay.lens, device="cuda:0")
+    n_seq = max(1, s.num_seqs // 4)
+    blocks = [int(b) for i in range(n_seq) for b in lay.tables[i, :-(-int(lay.lens[i]) // s.block_size)]]
+    used = set(int(b) for b in lay.tables.flatten() if b >= 0)
+    spare = [b for b in range(lay.num_blocks) if b not in used]
+    dst = (spare + blocks)[:len(blocks)]  # into free blocks first (same data if they run out)
+    src_t = torch.tensor(blocks, dtype=torch.int32, device="cuda:0")
+    dst_t = torch.tensor(dst, dtype=torch.int32, device="cuda:0")
+    rec = P.swap_record_bytes(t.k_cache)
+    nbytes = len(blocks) * rec
+    host = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    dev_buf = torch.empty(nbytes, dtype=torch.uint8, device="cuda:0")
+
+    def timed(fn, K):
+        for _ in range(max(3, a.warmup)):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(K):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / K / 1e3
+
+    K = max(1, min(a.steps, 200))
+    clocks = ClockSampler(0)
+    t_out = timed(lambda: P.swap_out_blocks(t.k_cache, t.v_cache, src_t, host), K)
+    t_in = timed(lambda: P.swap_in_blocks(host, dst_t, t.k_cache, t.v_cache), K)
+    clk = clocks.stop()
+    t_d2h = timed(lambda: host.copy_(dev_buf, non_blocking=True), K)
+    t_h2d = timed(lambda: dev_buf.copy_(host, non_blocking=True), K)
+    st = P.device_error(0)
+    if st != P.PKV_OK:
+        raise SystemExit(f"device check failed: {P.status_string(st)}")
+    link = 2 * nbytes / (t_d2h + t_h2d) / 1e9
+    value = 2 * nbytes / (t_out + t_in) / 1e9
+    print(json.dumps({
+        "metric": "preemption swap GB/s (K+V block bytes out to page-locked host memory and back)",
+        "value": value, "unit": "GB/s", "n_gpus": 1, "steps": K, "warmup": max(3, a.warmup),
+        "ms_per_step": (t_out + t_in) * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": s.cache_dtype, "data": "synthetic",
+        "config": {"workload": W.describe(s), "blocks_per_step": len(blocks), "bytes_each_way": nbytes,
+                   "step": "swap_out_blocks then swap_in_blocks into other blocks"},
+        "swap_out_gbs": nbytes / t_out / 1e9, "swap_in_gbs": nbytes / t_in / 1e9,
+        "roofline": {"bound": "host link", "achieved": value, "peak": link, "unit": "GB/s", "frac": value / link,
+                     "peak_source": "torch device<->pinned-host copies of the same bytes in this run",
+                     "d2h_gbs": nbytes / t_d2h / 1e9, "h2d_gbs": nbytes / t_h2d / 1e9, "traffic": None},
+        "clocks": clk, "gpu_launches": 2 * K,
+    }))
+
+
 def main():
     a = parse()
     s = workload_spec(a)
+    if a.op == "swap":
+        run_swap(a, s)
+        return
     ws, rank, local, dist = dist_setup(a)
     if a.impl == "reference":
         run_reference(a, s, ws, rank)

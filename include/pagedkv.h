@@ -164,6 +164,34 @@ int paged_attn_decode_ex(const pkv_tensor* q, const pkv_tensor* k_cache,
                          size_t workspace_bytes, void* stream);
 
 /*
+ * swap_out_blocks / swap_in_blocks - the device half of preemption by
+ * swapping ("Preemption and eviction", KV-Cache Management and
+ * PagedAttention; "Preemption & GPU Swapping", PagedAttention and KV Cache
+ * Management): blocks of both pools to page-locked host memory and back,
+ * bit-exact, so a preempted sequence can resume in other blocks
+ * (pkv_seq_swap_out / pkv_seq_swap_in pick them).
+ *
+ *   k_cache, v_cache  device [NB, Hk, B, D] pools, same type (f16, bf16 or fp8
+ *                     codes; bytes are copied), same strides, rows 16-byte
+ *                     multiples
+ *   blocks            device int32 [n]: block ids, in record order
+ *   host_dst/host_src page-locked host memory mapped into the device's
+ *                     address space (cudaHostAlloc, or torch pin_memory),
+ *                     16-byte aligned, host_bytes >= n * record bytes;
+ *                     record i = block blocks[i]'s K tile [Hk, B, D]
+ *                     (row-major) then its V tile, 2 * Hk * B * D * e bytes
+ * The kernel reads or writes the host memory itself through its device
+ * mapping (no staging copy). Asynchronous on `stream`; the host buffer must
+ * stay allocated until the stream reaches that point. PKV_ERR_INVALID_ARG
+ * for pageable or unmapped host memory or a short buffer; a block id outside
+ * the pool is flagged (PKV_ERR_DEVICE_CHECK) and its record skipped.
+ */
+int swap_out_blocks(const pkv_tensor* k_cache, const pkv_tensor* v_cache, const pkv_tensor* blocks,
+                    void* host_dst, size_t host_bytes, void* stream);
+int swap_in_blocks(const void* host_src, size_t host_bytes, const pkv_tensor* blocks,
+                   pkv_tensor* k_cache, pkv_tensor* v_cache, void* stream);
+
+/*
  * paged_attn_decode_cascade - paged_attn_decode for a batch whose sequences
  * share prompt prefixes, reading each shared prefix block once per group
  * instead of once per sequence. Prefix sharing: "PagedAttention: treat the
@@ -367,6 +395,72 @@ int pkv_alloc_stats(void* handle, int32_t* free_blocks, int32_t* used_blocks,
 
 /* Reference count of one block (>= 0) or PKV_ERR_INVALID_ARG. */
 int pkv_block_refcount(void* handle, int32_t block);
+
+/* Preemption by swapping ("Preemption and eviction", KV-Cache Management and
+ * PagedAttention; "Preemption & GPU Swapping", PagedAttention and KV Cache
+ * Management).
+ *
+ * pkv_seq_swap_out: writes the sequence's blocks, in table order, to
+ * blocks[0 .. *n) (cap entries available) and drops this sequence's reference
+ * on each (a block whose count reaches 0 returns to the tail of the free
+ * list). Copy those blocks to host memory (swap_out_blocks) before anything
+ * reuses them. The sequence keeps its token count and becomes swapped out:
+ * every call but pkv_seq_free (which forgets it) and pkv_seq_swap_in answers
+ * PKV_ERR_UNKNOWN_SEQ for it, and its id stays taken (PKV_ERR_EXISTS).
+ * pkv_seq_swap_in: takes ceil(tokens / block_size) fresh blocks for a
+ * swapped-out sequence, writes them to blocks[0 .. *n) in table order (fill
+ * them with swap_in_blocks) and makes the sequence live again.
+ * Errors change nothing: PKV_ERR_UNKNOWN_SEQ, PKV_ERR_INVALID_ARG (cap too
+ * small, null pointer), PKV_ERR_OOM (not enough free blocks). */
+int pkv_seq_swap_out(void* handle, int64_t seq, int32_t* blocks, int32_t cap, int32_t* n);
+int pkv_seq_swap_in(void* handle, int64_t seq, int32_t* blocks, int32_t cap, int32_t* n);
+
+/* Utilisation figures of the pool ("Managing the KV cache": blocks stored with
+ * sharing versus storing each request's blocks separately, and the memory
+ * that saves; tokens held over the slots of used blocks): *table_blocks =
+ * the sum of all live sequences' table lengths (the blocks a pool without
+ * sharing would hold), *sequences = live sequences. With pkv_alloc_stats'
+ * used blocks U and tokens T: saved = 1 - U / table_blocks, utilisation =
+ * T / (U * block_size), and U * block_size - T <= (block_size - 1) *
+ * sequences (at most one partly filled block per sequence). */
+int pkv_alloc_utilisation(void* handle, int64_t* table_blocks, int32_t* sequences);
+
+/* A new sequence whose first num_blocks table entries are the given blocks
+ * (blocks in use, e.g. a prefix-cache match: one more reference each) and
+ * whose remaining ceil(num_tokens / block_size) - num_blocks blocks are
+ * fresh; num_blocks * block_size <= num_tokens. PKV_ERR_EXISTS,
+ * PKV_ERR_INVALID_ARG, PKV_ERR_OOM change nothing. */
+int pkv_seq_allocate_prefix(void* handle, int64_t seq, const int32_t* blocks, int32_t num_blocks,
+                            int32_t num_tokens);
+
+/* Prefix cache over an allocator ("RadixAttention — reuse a shared prefix";
+ * "Shared System Prompts & Prefix Caching"): a radix tree whose nodes are
+ * full blocks, keyed by their block_size token ids; the cache holds one
+ * reference on each node's block, so cached blocks outlive the sequences
+ * that wrote them. pkv_cache_destroy drops those references; destroying the
+ * allocator first detaches its caches (their calls then return
+ * PKV_ERR_INVALID_ARG; destroy them still). Host-only; not thread-safe (one
+ * caller at a time, allocator and caches together).
+ *   pkv_cache_insert: walk sequence seq's first n / block_size full blocks
+ *     (tokens: its first n token ids); a block whose tokens are already
+ *     cached on that path is left alone, others become nodes. *added = nodes
+ *     added. PKV_ERR_UNKNOWN_SEQ, PKV_ERR_INVALID_ARG (n above the sequence's
+ *     token count); PKV_ERR_OOM may leave a leading part cached.
+ *   pkv_cache_match: the blocks of the longest run of leading full blocks of
+ *     tokens[0..n) found in the tree (at most cap) into blocks, *matched =
+ *     their count; every node on the run counts as used now.
+ *   pkv_cache_evict: up to n times, release the least recently used leaf
+ *     whose block only the cache references (ties: the older node), its
+ *     block returning to the free list; *num_freed blocks written to freed.
+ *   The use clock advances once per insert and per match.
+ *   pkv_cache_nodes: cached blocks (>= 0). */
+int pkv_cache_create(void* alloc, void** cache);
+void pkv_cache_destroy(void* cache);
+int pkv_cache_insert(void* cache, int64_t seq, const int32_t* tokens, int32_t n, int32_t* added);
+int pkv_cache_match(void* cache, const int32_t* tokens, int32_t n, int32_t* blocks, int32_t cap,
+                    int32_t* matched);
+int pkv_cache_evict(void* cache, int32_t n, int32_t* freed, int32_t* num_freed);
+int pkv_cache_nodes(void* cache);
 
 /* Shared-prefix groups of a decode batch, for paged_attn_decode_cascade.
  * Prefix sharing: "PagedAttention: treat the cache like virtual memory"

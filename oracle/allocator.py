@@ -22,6 +22,13 @@ and KV Cache Management", in a structure of its own:
   * Freeing a sequence drops one reference on each block in table order; a
     block whose count reaches 0 returns to the free list.
 
+Preemption by swapping ("Preemption and eviction" of "PagedAttention: treat
+the cache like virtual memory" on the KV-Cache Management page; "Preemption &
+GPU Swapping" of "PagedAttention and KV Cache Management"): a swapped-out
+sequence gives up its blocks (its data goes to host memory first) and keeps
+only its token count; swapping it in takes fresh blocks, in table order,
+which the device fills from host memory.
+
 Readings where the listing is silent or would misbehave (each is a status
 code here, never a partial update):
   * Copy-on-write happens only when the slot to be written lies in a shared
@@ -35,6 +42,11 @@ code here, never a partial update):
   * Freeing an unknown sequence is a no-op (as in the listing); other calls
     on an unknown sequence raise UNKNOWN_SEQ; creating an existing one
     raises EXISTS; a reference count that would go below 0 raises DOUBLE_FREE.
+  * Swap: swapping out drops one reference on each block (in table order,
+    shared blocks included: the host copy is the sequence's own) and returns
+    the blocks to copy; a swapped-out sequence is unknown to every other call
+    but free (which forgets it) and swap_in, and its id stays taken. Swapping
+    in needs ceil(tokens / B) free blocks (OOM otherwise, nothing changes).
 """
 from __future__ import annotations
 
@@ -63,6 +75,7 @@ class BlockAllocator:
         self.refcount = [0] * num_blocks
         self.tables: Dict[int, List[int]] = {}
         self.num_tokens: Dict[int, int] = {}
+        self.swapped: Dict[int, int] = {}  # swapped-out sequence -> tokens
 
     # -- block level ---------------------------------------------------------
     def _take(self) -> int:
@@ -88,7 +101,7 @@ class BlockAllocator:
 
     # -- sequence level ------------------------------------------------------
     def allocate(self, seq: int, num_tokens: int) -> List[int]:
-        if seq in self.tables:
+        if seq in self.tables or seq in self.swapped:
             raise AllocError(ERR_EXISTS, f"sequence {seq} exists")
         if num_tokens < 0:
             raise AllocError(ERR_INVALID, "negative token count")
@@ -128,7 +141,7 @@ class BlockAllocator:
 
     def fork(self, src: int, dst: int) -> None:
         table = self._table(src)
-        if dst in self.tables:
+        if dst in self.tables or dst in self.swapped:
             raise AllocError(ERR_EXISTS, f"sequence {dst} exists")
         for blk in table:
             self.refcount[blk] += 1
@@ -136,12 +149,36 @@ class BlockAllocator:
         self.num_tokens[dst] = self.num_tokens[src]
 
     def free(self, seq: int) -> None:
+        self.swapped.pop(seq, None)
         if seq not in self.tables:
             return
         for blk in self.tables[seq]:
             self._drop(blk)
         del self.tables[seq]
         del self.num_tokens[seq]
+
+    def swap_out(self, seq: int) -> List[int]:
+        """The sequence's blocks in table order (to copy to host memory before
+        they are reused); each loses this sequence's reference."""
+        table = self._table(seq)
+        for blk in table:
+            self._drop(blk)
+        self.swapped[seq] = self.num_tokens.pop(seq)
+        del self.tables[seq]
+        return list(table)
+
+    def swap_in(self, seq: int) -> List[int]:
+        """Fresh blocks for a swapped-out sequence, in table order (to fill
+        from host memory)."""
+        if seq not in self.swapped:
+            raise AllocError(ERR_UNKNOWN_SEQ, f"sequence {seq} is not swapped out")
+        n_tok = self.swapped[seq]
+        n = -(-n_tok // self.block_size)
+        self._need(n)
+        del self.swapped[seq]
+        self.tables[seq] = [self._take() for _ in range(n)]
+        self.num_tokens[seq] = n_tok
+        return list(self.tables[seq])
 
     # -- queries -------------------------------------------------------------
     def num_free(self) -> int:
@@ -166,8 +203,11 @@ class BlockAllocator:
         used = sum(1 for r in self.refcount if r > 0)
         shared = sum(1 for r in self.refcount if r > 1)
         tokens = sum(fill.values())
+        table_blocks = sum(len(t) for t in self.tables.values())
         return {"free": self.num_free(), "used": used, "shared": shared, "tokens": tokens,
-                "utilisation": (tokens / (used * B)) if used else 1.0}
+                "utilisation": (tokens / (used * B)) if used else 1.0,
+                "table_blocks": table_blocks, "sequences": len(self.tables),
+                "saved": (1.0 - used / table_blocks) if table_blocks else 0.0}
 
     def run(self, ops) -> None:
         """Execute ("allocate", seq, n) / ("fork", src, dst) / ("free", seq) /
@@ -181,5 +221,9 @@ class BlockAllocator:
                 self.free(op[1])
             elif op[0] == "append":
                 self.append_tokens(op[1], op[2])
+            elif op[0] == "swap_out":
+                self.swap_out(op[1])
+            elif op[0] == "swap_in":
+                self.swap_in(op[1])
             else:
                 raise ValueError(op)

@@ -16,6 +16,13 @@ token slots into it ("Parallel Sampling & Beam Search via Copy-on-Write",
 "PagedAttention and KV Cache Management"). With one pool per layer that is
 every slot of the block, K and V, all heads, bit for bit. All copies of one
 call read the pool as it was before the call.
+
+swap_out / swap_in: the device half of preemption by swapping ("Preemption
+and eviction", KV-Cache Management page; "Preemption & GPU Swapping",
+"PagedAttention and KV Cache Management"): a preempted sequence's blocks go to
+host memory and later come back, possibly into other blocks. Host layout:
+one record per block in the order given, the block's K bytes ([Hk, B, D],
+row-major) then its V bytes.
 """
 from __future__ import annotations
 
@@ -66,6 +73,28 @@ def copy_blocks(k_pool, v_pool, pairs):
         k_new[dst] = k_old[src]
         v_new[dst] = v_old[src]
     return k_new, v_new
+
+
+def swap_out(k_pool, v_pool, blocks) -> np.ndarray:
+    """uint8 [n, 2 * Hk * B * D * e]: the records of the given blocks."""
+    recs = []
+    for blk in blocks:
+        kb = np.ascontiguousarray(k_pool[int(blk)]).view(np.uint8).reshape(-1)
+        vb = np.ascontiguousarray(v_pool[int(blk)]).view(np.uint8).reshape(-1)
+        recs.append(np.concatenate([kb, vb]))
+    width = 2 * int(np.prod(k_pool.shape[1:])) * k_pool.dtype.itemsize
+    return np.stack(recs) if recs else np.zeros((0, width), dtype=np.uint8)
+
+
+def swap_in(records, k_pool, v_pool, blocks):
+    """New (k_pool, v_pool) with record i written into block blocks[i]."""
+    k_pool = np.array(k_pool, copy=True)
+    v_pool = np.array(v_pool, copy=True)
+    half = records.shape[1] // 2 if len(blocks) else 0
+    for i, blk in enumerate(blocks):
+        k_pool[int(blk)] = records[i, :half].view(k_pool.dtype).reshape(k_pool.shape[1:])
+        v_pool[int(blk)] = records[i, half:].view(v_pool.dtype).reshape(v_pool.shape[1:])
+    return k_pool, v_pool
 
 
 def slot_of(table_row, position: int, block_size: int) -> int:

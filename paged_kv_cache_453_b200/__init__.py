@@ -49,6 +49,9 @@ EXPORTED = (
     "pkv_alloc_create", "pkv_alloc_destroy", "pkv_seq_allocate", "pkv_seq_append_slot",
     "pkv_seq_fork", "pkv_seq_free", "pkv_seq_num_tokens", "pkv_seq_block_table",
     "pkv_build_block_tables", "pkv_alloc_stats", "pkv_block_refcount", "pkv_prefix_groups",
+    "swap_out_blocks", "swap_in_blocks", "pkv_seq_swap_out", "pkv_seq_swap_in",
+    "pkv_alloc_utilisation", "pkv_seq_allocate_prefix", "pkv_cache_create", "pkv_cache_destroy",
+    "pkv_cache_insert", "pkv_cache_match", "pkv_cache_evict", "pkv_cache_nodes",
 )
 
 
@@ -107,6 +110,19 @@ def lib() -> ctypes.CDLL:
             "pkv_block_refcount": (ctypes.c_int, [vp, i32]),
             "paged_attn_decode_cascade": (ctypes.c_int, [P, P, P, P, P, P, P, P, ctypes.c_int, ctypes.c_int,
                                                          ctypes.c_int, ctypes.c_int, f32, ctypes.c_int, P, vp]),
+            "pkv_alloc_utilisation": (ctypes.c_int, [vp, ctypes.POINTER(i64), ctypes.POINTER(i32)]),
+            "pkv_seq_allocate_prefix": (ctypes.c_int, [vp, i64, ctypes.POINTER(i32), i32, i32]),
+            "pkv_cache_create": (ctypes.c_int, [vp, ctypes.POINTER(vp)]),
+            "pkv_cache_destroy": (None, [vp]),
+            "pkv_cache_insert": (ctypes.c_int, [vp, i64, ctypes.POINTER(i32), i32, ctypes.POINTER(i32)]),
+            "pkv_cache_match": (ctypes.c_int, [vp, ctypes.POINTER(i32), i32, ctypes.POINTER(i32), i32,
+                                               ctypes.POINTER(i32)]),
+            "pkv_cache_evict": (ctypes.c_int, [vp, i32, ctypes.POINTER(i32), ctypes.POINTER(i32)]),
+            "pkv_cache_nodes": (ctypes.c_int, [vp]),
+            "swap_out_blocks": (ctypes.c_int, [P, P, P, vp, ctypes.c_size_t, vp]),
+            "swap_in_blocks": (ctypes.c_int, [vp, ctypes.c_size_t, P, P, P, vp]),
+            "pkv_seq_swap_out": (ctypes.c_int, [vp, i64, ctypes.POINTER(i32), i32, ctypes.POINTER(i32)]),
+            "pkv_seq_swap_in": (ctypes.c_int, [vp, i64, ctypes.POINTER(i32), i32, ctypes.POINTER(i32)]),
             "pkv_prefix_groups": (ctypes.c_int, [ctypes.POINTER(i32), i32, i32, ctypes.POINTER(i32), i32, i32,
                                                  ctypes.POINTER(i32), ctypes.POINTER(i32), ctypes.POINTER(i32),
                                                  ctypes.POINTER(i32), ctypes.POINTER(i32)]),
@@ -219,6 +235,32 @@ def prepare_decode_cascade(q, k_cache, v_cache, block_tables, context_lens, grou
     return Prepared("paged_attn_decode_cascade", lib().paged_attn_decode_cascade, args, (ds, groups), stream)
 
 
+def swap_record_bytes(k_cache) -> int:
+    """Bytes of one host record of a block (its K tile then its V tile)."""
+    return 2 * k_cache[0].numel() * k_cache.element_size()
+
+
+def swap_out_blocks(k_cache, v_cache, blocks, host, stream=None) -> None:
+    """Copy blocks[i] of both pools into record i of `host` (page-locked)."""
+    fp8 = k_cache.dtype in _FP8_TYPES()
+    ds = [_desc(k_cache, fp8), _desc(v_cache, fp8), _desc(blocks)]
+    _check(lib().swap_out_blocks(_ref(ds[0]), _ref(ds[1]), _ref(ds[2]), ctypes.c_void_p(host.data_ptr()),
+                                 host.numel() * host.element_size(), _stream(stream)), "swap_out_blocks")
+
+
+def swap_in_blocks(host, blocks, k_cache, v_cache, stream=None) -> None:
+    """Copy record i of `host` (page-locked) into block blocks[i] of both pools."""
+    fp8 = k_cache.dtype in _FP8_TYPES()
+    ds = [_desc(blocks), _desc(k_cache, fp8), _desc(v_cache, fp8)]
+    _check(lib().swap_in_blocks(ctypes.c_void_p(host.data_ptr()), host.numel() * host.element_size(), _ref(ds[0]),
+                                _ref(ds[1]), _ref(ds[2]), _stream(stream)), "swap_in_blocks")
+
+
+def _FP8_TYPES():
+    import torch
+    return (torch.uint8, torch.float8_e4m3fn)
+
+
 def paged_attn_decode_fp8(q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
                           num_kv_heads: int, scale: float, block_size: int, out, stream=None) -> None:
     ds = [_desc(q), _desc(k_cache, True), _desc(v_cache, True), _desc(k_scale), _desc(v_scale),
@@ -299,6 +341,52 @@ def device_error(device: int = 0) -> int:
 # Host block allocator
 # ---------------------------------------------------------------------------
 
+class PrefixCache:
+    """Radix tree of cached full blocks over a BlockAllocator (C++)."""
+
+    def __init__(self, alloc: "BlockAllocator"):
+        self._alloc = alloc  # keeps the allocator alive while the cache exists
+        self._h = ctypes.c_void_p()
+        _check(lib().pkv_cache_create(alloc._h, ctypes.byref(self._h)), "pkv_cache_create")
+
+    def close(self) -> None:
+        if self._h:
+            lib().pkv_cache_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    @staticmethod
+    def _toks(tokens):
+        return (ctypes.c_int32 * max(1, len(tokens)))(*[int(x) for x in tokens])
+
+    def insert(self, seq: int, tokens: Sequence[int]) -> int:
+        added = ctypes.c_int32()
+        _check(lib().pkv_cache_insert(self._h, int(seq), self._toks(tokens), len(tokens), ctypes.byref(added)),
+               "pkv_cache_insert")
+        return added.value
+
+    def match(self, tokens: Sequence[int]) -> List[int]:
+        cap = max(1, len(tokens))
+        buf, m = (ctypes.c_int32 * cap)(), ctypes.c_int32()
+        _check(lib().pkv_cache_match(self._h, self._toks(tokens), len(tokens), buf, cap, ctypes.byref(m)),
+               "pkv_cache_match")
+        return list(buf[:m.value])
+
+    def evict(self, n: int) -> List[int]:
+        buf, k = (ctypes.c_int32 * max(1, n))(), ctypes.c_int32()
+        _check(lib().pkv_cache_evict(self._h, int(n), buf, ctypes.byref(k)), "pkv_cache_evict")
+        return list(buf[:k.value])
+
+    @property
+    def nodes(self) -> int:
+        return int(lib().pkv_cache_nodes(self._h))
+
+
 def prefix_groups(tables, lens, block_size: int, min_members: int = 2):
     """Shared-prefix groups of a decode batch (pkv_prefix_groups).
 
@@ -362,6 +450,37 @@ class BlockAllocator:
 
     def free(self, seq: int) -> None:
         _check(lib().pkv_seq_free(self._h, int(seq)), "pkv_seq_free")
+
+    def allocate_prefix(self, seq: int, blocks: Sequence[int], num_tokens: int) -> None:
+        arr = (ctypes.c_int32 * max(1, len(blocks)))(*[int(b) for b in blocks])
+        _check(lib().pkv_seq_allocate_prefix(self._h, int(seq), arr, len(blocks), int(num_tokens)),
+               "pkv_seq_allocate_prefix")
+
+    def utilisation(self):
+        """Pool figures: blocks stored vs blocks without sharing, and fill."""
+        tb, ns = ctypes.c_int64(), ctypes.c_int32()
+        _check(lib().pkv_alloc_utilisation(self._h, ctypes.byref(tb), ctypes.byref(ns)), "pkv_alloc_utilisation")
+        st = self.stats()
+        used, tokens = st["used"], st["tokens"]
+        return {"blocks_stored": used, "blocks_without_sharing": int(tb.value), "sequences": int(ns.value),
+                "tokens": tokens, "saved": (1.0 - used / tb.value) if tb.value else 0.0,
+                "utilisation": (tokens / (used * self.block_size)) if used else 1.0,
+                "waste_slots": used * self.block_size - tokens,
+                "waste_bound": (self.block_size - 1) * int(ns.value)}
+
+    def swap_out(self, seq: int) -> List[int]:
+        """The sequence's blocks (to copy out first); it becomes swapped out."""
+        cap = max(1, self.num_blocks)
+        buf, n = (ctypes.c_int32 * cap)(), ctypes.c_int32()
+        _check(lib().pkv_seq_swap_out(self._h, int(seq), buf, cap, ctypes.byref(n)), "pkv_seq_swap_out")
+        return list(buf[:n.value])
+
+    def swap_in(self, seq: int) -> List[int]:
+        """Fresh blocks for a swapped-out sequence (to copy back into)."""
+        cap = max(1, self.num_blocks)
+        buf, n = (ctypes.c_int32 * cap)(), ctypes.c_int32()
+        _check(lib().pkv_seq_swap_in(self._h, int(seq), buf, cap, ctypes.byref(n)), "pkv_seq_swap_in")
+        return list(buf[:n.value])
 
     def num_tokens(self, seq: int) -> int:
         n = lib().pkv_seq_num_tokens(self._h, int(seq))

@@ -10,6 +10,12 @@
 // copy_blocks: the device half of copy-on-write ("Parallel Sampling & Beam
 // Search via Copy-on-Write"): block dst := block src in both pools, bit-exact,
 // 16-byte vectors.
+//
+// swap_blocks_kernel: the device half of preemption by swapping ("Preemption
+// and eviction", "Preemption & GPU Swapping"): record i of a page-locked host
+// buffer <-> block blocks[i] (its K tile [Hk, B, D] then its V tile), read or
+// written by the kernel through the buffer's device mapping, 16-byte vectors:
+// a warp moves 512 contiguous bytes of the record.
 #pragma once
 
 #include <cuda_fp8.h>
@@ -156,6 +162,45 @@ __global__ void copy_blocks_kernel(const __grid_constant__ CopyParams p, int* er
     const long long so = src * p.c_s0 + o, d = dst * p.c_s0 + o;
     *reinterpret_cast<int4*>(p.kc + d) = *reinterpret_cast<const int4*>(p.kc + so);
     *reinterpret_cast<int4*>(p.vc + d) = *reinterpret_cast<const int4*>(p.vc + so);
+  }
+}
+
+struct SwapParams {
+  uint8_t* kc;
+  uint8_t* vc;
+  long long c_s0, c_s1, c_s2;  // byte strides of the pools [NB, Hk, B, D]
+  uint8_t* host;               // device address of the host records
+  const int* blocks;
+  long long bl_s;
+  int n, Hk, B, NB;
+  int row_vecs;         // 16-byte vectors per (head, token) row
+  long long rec_bytes;  // bytes of one record: K tile then V tile
+};
+
+template <bool kOut>
+__global__ void swap_blocks_kernel(const __grid_constant__ SwapParams p, int* err) {
+  const int i = blockIdx.x;
+  const int blk = p.blocks[i * p.bl_s];
+  if (blk < 0 || blk >= p.NB) {
+    if (threadIdx.x == 0 && blockIdx.y == 0) atomicOr(err, kErrBadBlock);
+    return;
+  }
+  const int per_head = p.B * p.row_vecs;
+  const int total = p.Hk * per_head;  // vectors per tile
+  uint8_t* rec = p.host + static_cast<long long>(i) * p.rec_bytes;
+  for (int v = blockIdx.y * blockDim.x + threadIdx.x; v < total; v += gridDim.y * blockDim.x) {
+    const int h = v / per_head, rem = v % per_head;
+    const int row = rem / p.row_vecs, vec = rem % p.row_vecs;
+    const long long o = blk * p.c_s0 + h * p.c_s1 + row * p.c_s2 + vec * 16;
+    int4* rk = reinterpret_cast<int4*>(rec + static_cast<long long>(v) * 16);
+    int4* rv = reinterpret_cast<int4*>(rec + (static_cast<long long>(total) + v) * 16);
+    if constexpr (kOut) {
+      *rk = *reinterpret_cast<const int4*>(p.kc + o);
+      *rv = *reinterpret_cast<const int4*>(p.vc + o);
+    } else {
+      *reinterpret_cast<int4*>(p.kc + o) = *rk;
+      *reinterpret_cast<int4*>(p.vc + o) = *rv;
+    }
   }
 }
 

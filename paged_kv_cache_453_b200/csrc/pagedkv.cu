@@ -600,6 +600,64 @@ int launch_cascade(const DecodeArgs& a, const pkv_tensor* pblk, const pkv_tensor
 // Cache writes and block copies
 // ---------------------------------------------------------------------------
 
+// Swap blocks between the pools and page-locked host records.
+int launch_swap(const pkv_tensor* kc, const pkv_tensor* vc, const pkv_tensor* blocks,
+                const void* host, size_t host_bytes, bool out, cudaStream_t stream) {
+  if (!kc || !vc || !blocks) return PKV_ERR_INVALID_ARG;
+  const int dt = kc->dtype;
+  const int eb = elem_bytes(dt);
+  if (eb == 0 || eb > 2 || !pool_ok(kc, dt) || !pool_ok(vc, dt) || !same_shape(kc, vc))
+    return PKV_ERR_INVALID_ARG;
+  if (!well_formed(blocks, 1, PKV_I32)) return PKV_ERR_INVALID_ARG;
+  const int64_t n = blocks->shape[0];
+  if ((kc->shape[3] * eb) % 16 != 0) return PKV_ERR_UNSUPPORTED;
+  if (n > INT32_MAX || kc->shape[0] > INT32_MAX) return PKV_ERR_UNSUPPORTED;
+  const long long rec = 2LL * kc->shape[1] * kc->shape[2] * kc->shape[3] * eb;
+  if (static_cast<unsigned long long>(n) * rec > host_bytes) return PKV_ERR_INVALID_ARG;
+  if (n == 0) return PKV_OK;
+  if (!host || !aligned(host, 16)) return PKV_ERR_INVALID_ARG;
+  // the host buffer must be page-locked and mapped into the device's space
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, host) != cudaSuccess || at.type != cudaMemoryTypeHost ||
+      !at.devicePointer) {
+    cudaGetLastError();
+    return PKV_ERR_INVALID_ARG;
+  }
+  int dev, st;
+  if ((st = current_device(&dev)) != PKV_OK) return st;
+  DeviceState* ds;
+  if ((st = device_state(dev, &ds)) != PKV_OK) return st;
+  SwapParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.kc = static_cast<uint8_t*>(kc->data);
+  p.vc = static_cast<uint8_t*>(vc->data);
+  p.c_s0 = kc->stride[0] * eb;
+  p.c_s1 = kc->stride[1] * eb;
+  p.c_s2 = kc->stride[2] * eb;
+  if (vc->stride[0] != kc->stride[0] || vc->stride[1] != kc->stride[1] ||
+      vc->stride[2] != kc->stride[2])
+    return PKV_ERR_INVALID_ARG;
+  p.host = static_cast<uint8_t*>(at.devicePointer);
+  p.blocks = static_cast<const int*>(blocks->data);
+  p.bl_s = blocks->stride[0];
+  p.n = static_cast<int>(n);
+  p.Hk = static_cast<int>(kc->shape[1]);
+  p.B = static_cast<int>(kc->shape[2]);
+  p.NB = static_cast<int>(kc->shape[0]);
+  p.row_vecs = static_cast<int>(kc->shape[3] * eb / 16);
+  p.rec_bytes = rec;
+  const int total = p.Hk * p.B * p.row_vecs;
+  const int tpb = 256;
+  int chunks = (total + tpb - 1) / tpb;
+  if (chunks > 65535) chunks = 65535;
+  dim3 grid(static_cast<unsigned>(n), static_cast<unsigned>(chunks));
+  if (out)
+    swap_blocks_kernel<true><<<grid, tpb, 0, stream>>>(p, ds->err);
+  else
+    swap_blocks_kernel<false><<<grid, tpb, 0, stream>>>(p, ds->err);
+  return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
 int launch_reshape(const pkv_tensor* k, const pkv_tensor* v, pkv_tensor* kc, pkv_tensor* vc,
                    const pkv_tensor* slots, const pkv_tensor* ks, const pkv_tensor* vs, bool fp8,
                    cudaStream_t stream) {
@@ -871,6 +929,18 @@ int copy_blocks(pkv_tensor* k_cache, pkv_tensor* v_cache, const pkv_tensor* pair
   dim3 grid(static_cast<unsigned>(n), static_cast<unsigned>(chunks));
   copy_blocks_kernel<<<grid, tpb, 0, static_cast<cudaStream_t>(stream)>>>(p, ds->err);
   return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+int swap_out_blocks(const pkv_tensor* k_cache, const pkv_tensor* v_cache, const pkv_tensor* blocks,
+                    void* host_dst, size_t host_bytes, void* stream) {
+  return launch_swap(k_cache, v_cache, blocks, host_dst, host_bytes, true,
+                     static_cast<cudaStream_t>(stream));
+}
+
+int swap_in_blocks(const void* host_src, size_t host_bytes, const pkv_tensor* blocks,
+                   pkv_tensor* k_cache, pkv_tensor* v_cache, void* stream) {
+  return launch_swap(k_cache, v_cache, blocks, host_src, host_bytes, false,
+                     static_cast<cudaStream_t>(stream));
 }
 
 int pkv_device_error(int device) {

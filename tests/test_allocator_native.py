@@ -1,5 +1,6 @@
 """The C++ block allocator (through the C ABI) against the pages' demo run and
 against the oracle allocator on random operation sequences (bit-exact)."""
+import ctypes
 import random
 
 import numpy as np
@@ -42,17 +43,24 @@ def test_random_ops_match_oracle(seed):
     order = rng.sample(range(N), N)
     a = P.BlockAllocator(N, B, order)
     o = OracleAlloc(N, B, order)
-    live, nxt = [], 0
+    live, nxt, out = [], 0, []
     for step in range(2000):
         op = rng.random()
         if op < 0.2 or not live:
             args, name = (nxt, rng.randint(0, 3 * B)), "allocate"
         elif op < 0.3:
             args, name = (rng.choice(live), nxt), "fork"
-        elif op < 0.42:
+        elif op < 0.4:
             args, name = (rng.choice(live),), "free"
-        elif op < 0.45:
+        elif op < 0.43:
             args, name = (10_000 + rng.randint(0, 5),), "append_slot"   # unknown sequence
+        elif op < 0.47:
+            args, name = (rng.choice(live),), "swap_out"
+        elif op < 0.51:
+            # a swapped-out sequence mostly, sometimes a live one (an error)
+            args, name = (rng.choice(out) if out and rng.random() < 0.8 else rng.choice(live),), "swap_in"
+        elif op < 0.52 and out:
+            args, name = (rng.choice(out),), "append_slot"              # swapped out: unknown
         else:
             args, name = (rng.choice(live),), "append_slot"
         err_o = err_a = None
@@ -66,13 +74,19 @@ def test_random_ops_match_oracle(seed):
             err_a = e.status
         assert err_o == err_a, (step, name, args, err_o, err_a)
         if err_o is None:
-            if name == "append_slot":
+            if name in ("append_slot", "swap_out", "swap_in"):
                 assert ra == ro
             if name in ("allocate", "fork"):
                 live.append(nxt)
                 nxt += 1
             if name == "free":
                 live.remove(args[0])
+            if name == "swap_out":
+                live.remove(args[0])
+                out.append(args[0])
+            if name == "swap_in":
+                out.remove(args[0])
+                live.append(args[0])
         _same(a, o, live)
 
 
@@ -169,3 +183,84 @@ def test_prefix_groups_rejects_bad_arguments():
         P.prefix_groups(t, ln, 4, 0)
     gs, mem, pb = P.prefix_groups(t[:0], ln[:0], 4)
     assert gs.tolist() == [0] and mem.tolist() == [] and pb.tolist() == []
+
+
+# ---------------------------------------------------------------------------
+# Prefix cache, prefix allocation and utilisation against the oracle
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("seed", [4, 5, 6])
+def test_prefix_cache_random_ops_match_oracle(seed):
+    from oracle.radix import PrefixCache as OracleCache, allocate_prefix
+    rng = random.Random(seed)
+    N, B = 200, rng.choice([1, 2, 4])
+    a = P.BlockAllocator(N, B)
+    o = OracleAlloc(N, B)
+    ca, co = P.PrefixCache(a), OracleCache(o)
+    prompts = [[rng.randint(0, 2) for _ in range(rng.randint(0, 6 * B))] for _ in range(4)]
+    live, toks, nxt = [], {}, 0
+    for step in range(600):
+        r = rng.random()
+        if r < 0.25 or not live:
+            # a new request: a prompt plus a suffix, reusing what the cache holds
+            t = rng.choice(prompts) + [rng.randint(0, 2) for _ in range(rng.randint(0, 3 * B))]
+            ma, mo = ca.match(t), co.match(t)
+            assert ma == mo, step
+            err_a = err_o = None
+            try:
+                a.allocate_prefix(nxt, ma, len(t))
+            except P.PkvError as e:
+                err_a = e.status
+            try:
+                allocate_prefix(o, nxt, mo, len(t))
+            except AllocError as e:
+                err_o = e.code
+            assert err_a == err_o
+            if err_a is None:
+                live.append(nxt)
+                toks[nxt] = t
+            nxt += 1
+        elif r < 0.45:
+            s = rng.choice(live)
+            assert ca.insert(s, toks[s]) == co.insert(s, toks[s])
+        elif r < 0.6:
+            s = rng.choice(live)
+            a.free(s)
+            o.free(s)
+            live.remove(s)
+        elif r < 0.7:
+            n = rng.randint(0, 4)
+            assert ca.evict(n) == co.evict(n)
+        else:
+            s = rng.choice(live)
+            err_a = err_o = None
+            try:
+                ra = a.append_slot(s)
+            except P.PkvError as e:
+                err_a = e.status
+            try:
+                ro = o.append_slot(s)
+            except AllocError as e:
+                err_o = e.code
+            assert err_a == err_o
+            if err_a is None:
+                assert ra == ro
+                toks[s].append(rng.randint(0, 2))
+        assert ca.nodes == co.nodes
+        _same(a, o, live)
+        u, ost = a.utilisation(), o.stats()
+        assert u["blocks_without_sharing"] == ost["table_blocks"] and u["sequences"] == ost["sequences"]
+    ca.close()
+
+
+def test_cache_outliving_its_allocator_is_detached():
+    a = P.BlockAllocator(8, 2)
+    c = P.PrefixCache(a)
+    a.allocate(1, 4)
+    assert c.insert(1, [1, 2, 3, 4]) == 2
+    lib = P.lib()
+    lib.pkv_alloc_destroy(a._h)          # the allocator goes first
+    a._h = None
+    buf, n = (ctypes.c_int32 * 2)(), ctypes.c_int32()
+    assert lib.pkv_cache_evict(c._h, 2, buf, ctypes.byref(n)) == P.PKV_ERR_INVALID_ARG
+    c.close()                            # safe: nothing left to release

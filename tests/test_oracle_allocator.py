@@ -166,4 +166,5 @@ def test_stats_utilisation():
     a.allocate(1, 6)
     a.fork(1, 2)
     st = a.stats()
-    assert st == {"free": 8, "used": 2, "shared": 2, "tokens": 6, "utilisation": 6 / 8}
+    assert st == {"free": 8, "used": 2, "shared": 2, "tokens": 6, "utilisation": 6 / 8,
+                  "table_blocks": 4, "sequences": 2, "saved": 0.5}
