@@ -32,6 +32,8 @@ import sys
 import threading
 import time
 
+import numpy as np
+
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
@@ -55,8 +57,11 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--op", default="decode", choices=["decode", "swap"],
-                    help="swap: time preemption by swapping (blocks to page-locked host memory and back)")
+    ap.add_argument("--op", default="decode", choices=["decode", "swap", "prefill"],
+                    help="swap: preemption by swapping (blocks to page-locked host memory and back); "
+                         "prefill: causal attention of --q-tokens new tokens per sequence")
+    ap.add_argument("--q-tokens", type=int, default=4,
+                    help="new tokens per sequence for --op prefill (4: speculative verification)")
     ap.add_argument("--no-cascade", action="store_true",
                     help="decode a shared-prefix workload with the plain decode")
     return ap.parse_args()
@@ -401,11 +406,70 @@ def run_swap(a, s: W.Spec):
     }))
 
 
+def run_prefill(a, s: W.Spec):
+    """Causal attention of --q-tokens new tokens per sequence (the last ones of
+    each context) over the workload's paged cache, inputs resident."""
+    import paged_kv_cache_453_b200 as P
+    from paged_kv_cache_453_b200.build import build
+    build()
+    torch.cuda.set_device(0)
+    s = s.replace(append=False)
+    lay = W.make_layout(s)
+    t = W.make_tensors(s, lay.num_blocks, lay.tables, lay.lens, device="cuda:0")
+    lens = lay.lens.tolist()
+    nq = [min(a.q_tokens, L) for L in lens]
+    q_start = torch.tensor([0] + list(np.cumsum(nq)), dtype=torch.int32)
+    T = int(q_start[-1])
+    g = torch.Generator(device="cuda:0").manual_seed(s.seed + 77)
+    q = torch.randn((T, s.num_q_heads, s.head_dim), generator=g, device="cuda:0").to(t.q.dtype)
+    out = torch.empty_like(q)
+    call = P.prepare_prefill(q, t.k_cache, t.v_cache, lay.tables.cuda(), lay.lens.cuda(), q_start.cuda(),
+                             max(nq), s.num_kv_heads, s.scale, s.block_size, out)
+    kv = kv_bytes_of(s, lens)
+    alg = kv + 2 * T * s.num_q_heads * s.head_dim * 2 + sum(-(-L // s.block_size) for L in lens) * 4 + 8 * s.num_seqs
+    keys = sum(sum(L - n + j + 1 for j in range(n)) for L, n in zip(lens, nq))
+    flops = 4.0 * s.head_dim * s.num_q_heads * keys
+    for _ in range(max(3, a.warmup)):
+        call()
+    torch.cuda.synchronize()
+    K = a.steps
+    clocks = ClockSampler(0)
+    time.sleep(0.3 if clocks.proc else 0)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(K):
+        call()
+    e1.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    st = P.device_error(0)
+    if st != P.PKV_OK:
+        raise SystemExit(f"device check failed: {P.status_string(st)}")
+    sec = e0.elapsed_time(e1) / K / 1e3
+    peak, src = measured_peak_hbm()
+    print(json.dumps({
+        "metric": "multi-token paged attention HBM GB/s (KV bytes read/s) and TFLOP/s",
+        "value": kv / sec / 1e9, "unit": "GB/s", "n_gpus": 1, "steps": K, "warmup": max(3, a.warmup),
+        "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": s.cache_dtype, "data": "synthetic",
+        "config": {"workload": W.describe(s), "new_tokens_per_seq": a.q_tokens, "query_rows": T,
+                   "kv_bytes": kv, "l2": "inputs larger than L2 (K/V pool > 126 MB), no flush"},
+        "tflops": flops / sec / 1e12,
+        "roofline": {"kernel": "prefill_kernel", "bound": "hbm", "achieved": alg / sec / 1e9, "peak": peak,
+                     "unit": "GB/s", "frac": alg / sec / 1e9 / peak, "peak_source": src, "traffic": None,
+                     "alg_bytes_per_launch": alg, "flops_per_launch": flops},
+        "clocks": clk, "gpu_launches": K,
+    }))
+
+
 def main():
     a = parse()
     s = workload_spec(a)
     if a.op == "swap":
         run_swap(a, s)
+        return
+    if a.op == "prefill":
+        run_prefill(a, s)
         return
     ws, rank, local, dist = dist_setup(a)
     if a.impl == "reference":

@@ -164,6 +164,36 @@ int paged_attn_decode_ex(const pkv_tensor* q, const pkv_tensor* k_cache,
                          size_t workspace_bytes, void* stream);
 
 /*
+ * paged_attn_prefill - causal attention of several new tokens per sequence
+ * over the paged cache: a prompt, or a chunk of one, whose K/V were written
+ * to the blocks allocated for it ("How Block Paging Operates During
+ * Generation": a request's prompt gets its blocks when it starts; "Dynamic
+ * Request Insertion": a waiting request's prefill joins the running
+ * iteration), or speculative tokens being verified. Sequence s has
+ * n_s = q_start[s + 1] - q_start[s] new tokens, the last n_s of its
+ * L_s = context_lens[s] (0 <= n_s <= L_s); query row q_start[s] + j is the
+ * token at position L_s - n_s + j and attends to positions 0 .. L_s - n_s + j.
+ * n_s = 1 for every s is the decode step.
+ *
+ *   q             device [T, Hq, D] f16 | bf16, rows grouped by sequence
+ *   k_cache, v_cache, block_tables, context_lens, num_kv_heads, scale,
+ *   block_size    as paged_attn_decode (16-bit caches)
+ *   q_start       device int32 [S + 1], non-decreasing, q_start[S] <= T
+ *   max_q_tokens  host int >= every n_s (sizes the launch)
+ *   out           device [T, Hq, D] like q; rows of tokens in no sequence
+ *                 are left untouched
+ * One CTA per (sequence, kv head, 16 / 32 / 64 query columns), a column being
+ * one query head of one new token: the chunk's columns share every K/V tile
+ * read, so the cache is read once per chunk. Asynchronous on `stream`; an
+ * inconsistent q_start / context_lens row or block id is flagged
+ * (PKV_ERR_DEVICE_CHECK) and that row skipped.
+ */
+int paged_attn_prefill(const pkv_tensor* q, const pkv_tensor* k_cache, const pkv_tensor* v_cache,
+                       const pkv_tensor* block_tables, const pkv_tensor* context_lens,
+                       const pkv_tensor* q_start, int max_q_tokens, int num_kv_heads, float scale,
+                       int block_size, pkv_tensor* out, void* stream);
+
+/*
  * swap_out_blocks / swap_in_blocks - the device half of preemption by
  * swapping ("Preemption and eviction", KV-Cache Management and
  * PagedAttention; "Preemption & GPU Swapping", PagedAttention and KV Cache

@@ -92,3 +92,50 @@ def contiguous_attention_loops(qv, K, V, scale: float):
     l = math.fsum(w)
     D = len(V[0])
     return [math.fsum(w[t] * V[t][d] for t in range(L)) / l for d in range(D)]
+
+
+def paged_prefill(q, k_pool, v_pool, block_tables, context_lens, q_start, scale: float, block_size: int,
+                  q_kind: str, cache_kind: str, k_scale=None, v_scale=None,
+                  seqs: Optional[Iterable[int]] = None) -> np.ndarray:
+    """Causal attention of several new query tokens per sequence, fp64 [T, Hq, D].
+
+    Several new tokens of a sequence attend over its paged cache in one call
+    when a prompt (or a chunk of it) is processed after its K/V were written
+    to the blocks allocated for it ("How Block Paging Operates During
+    Generation": a request's prompt gets its blocks when it starts; "Dynamic
+    Request Insertion": a waiting request's prefill joins the running
+    iteration), or when speculative tokens are verified (the takeaways name
+    speculative decoding among the uses of shared blocks). Plain reading:
+    sequence s has n_s = q_start[s + 1] - q_start[s] new tokens, the last
+    n_s of its L_s = context_lens[s] tokens; query row q_start[s] + j holds
+    the token at position p = L_s - n_s + j, which attends (causally) to the
+    positions 0 .. p of the same sequence, through the block table exactly
+    as the decode query does. n_s = 1 is the decode step.
+    """
+    q = np.asarray(q)
+    T, Hq, D = q.shape
+    Hk = np.asarray(k_pool).shape[1]
+    g = Hq // Hk
+    out = np.zeros((T, Hq, D), dtype=np.float64)
+    q_start = np.asarray(q_start, dtype=np.int64)
+    S = len(q_start) - 1
+    seqs = range(S) if seqs is None else seqs
+    for s in seqs:
+        L = int(context_lens[s])
+        n = int(q_start[s + 1] - q_start[s])
+        assert 0 <= n <= L
+        if n == 0:
+            continue
+        for h in range(Hk):
+            ks = None if k_scale is None else float(np.asarray(k_scale)[h])
+            vs = None if v_scale is None else float(np.asarray(v_scale)[h])
+            K = gather_sequence(k_pool, block_tables[s], L, block_size, h, cache_kind, ks)
+            V = gather_sequence(v_pool, block_tables[s], L, block_size, h, cache_kind, vs)
+            for j in range(n):
+                p = L - n + j
+                for i in range(h * g, (h + 1) * g):
+                    qi = widen(q[q_start[s] + j, i], q_kind)
+                    x = scale * (K[:p + 1] @ qi)
+                    w = np.exp(x - x.max())
+                    out[q_start[s] + j, i] = (w @ V[:p + 1]) / w.sum()
+    return out

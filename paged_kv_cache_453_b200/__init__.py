@@ -51,7 +51,7 @@ EXPORTED = (
     "pkv_build_block_tables", "pkv_alloc_stats", "pkv_block_refcount", "pkv_prefix_groups",
     "swap_out_blocks", "swap_in_blocks", "pkv_seq_swap_out", "pkv_seq_swap_in",
     "pkv_alloc_utilisation", "pkv_seq_allocate_prefix", "pkv_cache_create", "pkv_cache_destroy",
-    "pkv_cache_insert", "pkv_cache_match", "pkv_cache_evict", "pkv_cache_nodes",
+    "pkv_cache_insert", "pkv_cache_match", "pkv_cache_evict", "pkv_cache_nodes", "paged_attn_prefill",
 )
 
 
@@ -110,6 +110,8 @@ def lib() -> ctypes.CDLL:
             "pkv_block_refcount": (ctypes.c_int, [vp, i32]),
             "paged_attn_decode_cascade": (ctypes.c_int, [P, P, P, P, P, P, P, P, ctypes.c_int, ctypes.c_int,
                                                          ctypes.c_int, ctypes.c_int, f32, ctypes.c_int, P, vp]),
+            "paged_attn_prefill": (ctypes.c_int, [P, P, P, P, P, P, ctypes.c_int, ctypes.c_int, f32, ctypes.c_int,
+                                                  P, vp]),
             "pkv_alloc_utilisation": (ctypes.c_int, [vp, ctypes.POINTER(i64), ctypes.POINTER(i32)]),
             "pkv_seq_allocate_prefix": (ctypes.c_int, [vp, i64, ctypes.POINTER(i32), i32, i32]),
             "pkv_cache_create": (ctypes.c_int, [vp, ctypes.POINTER(vp)]),
@@ -233,6 +235,23 @@ def prepare_decode_cascade(q, k_cache, v_cache, block_tables, context_lens, grou
         groups.num_groups, groups.max_group_size, groups.max_prefix_blocks, int(num_kv_heads),
         float(scale), int(block_size), ctypes.byref(ds[8]))
     return Prepared("paged_attn_decode_cascade", lib().paged_attn_decode_cascade, args, (ds, groups), stream)
+
+
+def paged_attn_prefill(q, k_cache, v_cache, block_tables, context_lens, q_start, max_q_tokens: int,
+                       num_kv_heads: int, scale: float, block_size: int, out, stream=None) -> None:
+    """Causal attention of several new tokens per sequence (q rows of sequence
+    s: q_start[s] .. q_start[s + 1], its last tokens; lens include them)."""
+    ds = [_desc(x) for x in (q, k_cache, v_cache, block_tables, context_lens, q_start, out)]
+    _check(lib().paged_attn_prefill(*[_ref(d) for d in ds[:6]], int(max_q_tokens), int(num_kv_heads), float(scale),
+                                    int(block_size), _ref(ds[6]), _stream(stream)), "paged_attn_prefill")
+
+
+def prepare_prefill(q, k_cache, v_cache, block_tables, context_lens, q_start, max_q_tokens: int,
+                    num_kv_heads: int, scale: float, block_size: int, out, stream=None) -> "Prepared":
+    ds = [_desc(x) for x in (q, k_cache, v_cache, block_tables, context_lens, q_start, out)]
+    args = tuple(ctypes.byref(d) for d in ds[:6]) + (int(max_q_tokens), int(num_kv_heads), float(scale),
+                                                    int(block_size), ctypes.byref(ds[6]))
+    return Prepared("paged_attn_prefill", lib().paged_attn_prefill, args, ds, stream)
 
 
 def swap_record_bytes(k_cache) -> int:

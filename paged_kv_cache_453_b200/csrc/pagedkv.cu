@@ -17,6 +17,7 @@
 #include "../../include/pagedkv.h"
 #include "cache_ops.cuh"
 #include "cascade.cuh"
+#include "prefill.cuh"
 #include "decode.cuh"
 
 namespace pkv {
@@ -597,6 +598,131 @@ int launch_cascade(const DecodeArgs& a, const pkv_tensor* pblk, const pkv_tensor
 }
 
 // ---------------------------------------------------------------------------
+// Multi-token (causal) paged attention
+// ---------------------------------------------------------------------------
+
+struct PrefillLaunch {
+  void (*kernel)(PrefillParams);
+  int threads, smem, cols;
+  bool attr_set[kMaxDevices];
+};
+
+template <bool QBF, int D, int BS, int NW>
+PrefillLaunch* prefill_entry() {
+  constexpr int NS = 4;
+  static PrefillLaunch e = {&prefill_kernel<QBF, D, BS, NS, NW>, NW * 32,
+                            PrefillCfg<QBF, D, BS, NS, NW>::SMEM, NW * 16, {false}};
+  return &e;
+}
+
+template <bool QBF, int D, int BS>
+PrefillLaunch* prefill_by_cols(int cols) {
+  if (cols <= 16) return prefill_entry<QBF, D, BS, 1>();
+  if (cols <= 32) return prefill_entry<QBF, D, BS, 2>();
+  return prefill_entry<QBF, D, BS, 4>();
+}
+
+PrefillLaunch* pick_prefill(bool qbf, int D, int BS, int cols) {
+  if (qbf) {
+    if (D == 128 && BS == 16) return prefill_by_cols<true, 128, 16>(cols);
+    if (D == 128 && BS == 32) return prefill_by_cols<true, 128, 32>(cols);
+    if (D == 64 && BS == 16) return prefill_by_cols<true, 64, 16>(cols);
+    if (D == 64 && BS == 32) return prefill_by_cols<true, 64, 32>(cols);
+  } else {
+    if (D == 128 && BS == 16) return prefill_by_cols<false, 128, 16>(cols);
+    if (D == 128 && BS == 32) return prefill_by_cols<false, 128, 32>(cols);
+    if (D == 64 && BS == 16) return prefill_by_cols<false, 64, 16>(cols);
+    if (D == 64 && BS == 32) return prefill_by_cols<false, 64, 32>(cols);
+  }
+  return nullptr;
+}
+
+int launch_prefill(const pkv_tensor* q, const pkv_tensor* kc, const pkv_tensor* vc,
+                   const pkv_tensor* bt, const pkv_tensor* cl, const pkv_tensor* qs, int max_q,
+                   int Hk, float scale, int BS, pkv_tensor* out, cudaStream_t stream) {
+  if (!q || !kc || !vc || !bt || !cl || !qs || !out) return PKV_ERR_INVALID_ARG;
+  const int qdt = q->dtype;
+  if (qdt != PKV_F16 && qdt != PKV_BF16) return PKV_ERR_INVALID_ARG;
+  if (!well_formed(q, 3, qdt) || !well_formed(out, 3, qdt) || !same_shape(q, out))
+    return PKV_ERR_INVALID_ARG;
+  if (!pool_ok(kc, qdt) || !pool_ok(vc, qdt) || !same_shape(kc, vc)) return PKV_ERR_INVALID_ARG;
+  const int64_t T = q->shape[0], Hq = q->shape[1], D = q->shape[2];
+  const int64_t NB = kc->shape[0];
+  if (kc->shape[1] != Hk || kc->shape[2] != BS || kc->shape[3] != D || Hk <= 0 || Hq % Hk != 0)
+    return PKV_ERR_INVALID_ARG;
+  if (!well_formed(bt, 2, PKV_I32) || !well_formed(cl, 1, PKV_I32)) return PKV_ERR_INVALID_ARG;
+  const int64_t S = bt->shape[0];
+  if (cl->shape[0] != S || (S > 0 && cl->stride[0] != 1)) return PKV_ERR_INVALID_ARG;
+  if (!well_formed(qs, 1, PKV_I32) || qs->shape[0] != S + 1 || qs->stride[0] != 1)
+    return PKV_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || max_q < 0) return PKV_ERR_INVALID_ARG;
+  if (T > 0 && (q->stride[0] % 2 || q->stride[1] % 2 || !aligned(q->data, 4)))
+    return PKV_ERR_INVALID_ARG;
+  const int64_t g = Hq / Hk;
+  if ((D != 64 && D != 128) || (BS != 16 && BS != 32)) return PKV_ERR_UNSUPPORTED;
+  if (NB > INT32_MAX || T > INT32_MAX || S * Hk > 65535LL * 65535LL ||
+      static_cast<int64_t>(max_q) * g > INT32_MAX / 2)
+    return PKV_ERR_UNSUPPORTED;
+  if (S == 0 || T == 0 || max_q == 0) return PKV_OK;
+  if (bt->shape[1] < 1 || NB < 1) return PKV_ERR_INVALID_ARG;
+  const int cols = static_cast<int>(max_q * g);
+  PrefillLaunch* e = pick_prefill(qdt == PKV_BF16, static_cast<int>(D), BS, cols);
+  if (!e) return PKV_ERR_UNSUPPORTED;
+  int dev, st;
+  if ((st = current_device(&dev)) != PKV_OK) return st;
+  DeviceState* ds;
+  if ((st = device_state(dev, &ds)) != PKV_OK) return st;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!e->attr_set[dev]) {
+      if (cudaFuncSetAttribute(e->kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, e->smem) !=
+          cudaSuccess)
+        return PKV_ERR_CUDA;
+      e->attr_set[dev] = true;
+    }
+  }
+  PrefillParams p;
+  std::memset(&p, 0, sizeof(p));
+  if ((st = encode_pool_map(&p.tmk, kc, qdt)) != PKV_OK) return st;
+  if ((st = encode_pool_map(&p.tmv, vc, qdt)) != PKV_OK) return st;
+  p.q = q->data;
+  p.q_t = q->stride[0];
+  p.q_h = q->stride[1];
+  p.out = out->data;
+  p.o_t = out->stride[0];
+  p.o_h = out->stride[1];
+  p.tables = static_cast<const int*>(bt->data);
+  p.t_s = bt->stride[0];
+  p.lens = static_cast<const int*>(cl->data);
+  p.q_start = static_cast<const int*>(qs->data);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.S = static_cast<int>(S);
+  p.T = static_cast<int>(T);
+  p.Hk = Hk;
+  p.g = static_cast<int>(g);
+  p.NB = static_cast<int>(NB);
+  p.MB = static_cast<int>(bt->shape[1]);
+  const int ncc = (cols + e->cols - 1) / e->cols;
+  p.evict_first = ncc == 1;
+  p.err = ds->err;
+  const long long sh = S * Hk;
+  const unsigned gy = static_cast<unsigned>(std::min<long long>(sh, 65535));
+  const unsigned gz = static_cast<unsigned>((sh + gy - 1) / gy);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(ncc), gy, gz);
+  cfg.blockDim = dim3(static_cast<unsigned>(e->threads));
+  cfg.dynamicSmemBytes = static_cast<size_t>(e->smem);
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, e->kernel, p) != cudaSuccess) return PKV_ERR_CUDA;
+  return PKV_OK;
+}
+
+// ---------------------------------------------------------------------------
 // Cache writes and block copies
 // ---------------------------------------------------------------------------
 
@@ -929,6 +1055,14 @@ int copy_blocks(pkv_tensor* k_cache, pkv_tensor* v_cache, const pkv_tensor* pair
   dim3 grid(static_cast<unsigned>(n), static_cast<unsigned>(chunks));
   copy_blocks_kernel<<<grid, tpb, 0, static_cast<cudaStream_t>(stream)>>>(p, ds->err);
   return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+int paged_attn_prefill(const pkv_tensor* q, const pkv_tensor* k_cache, const pkv_tensor* v_cache,
+                       const pkv_tensor* block_tables, const pkv_tensor* context_lens,
+                       const pkv_tensor* q_start, int max_q_tokens, int num_kv_heads, float scale,
+                       int block_size, pkv_tensor* out, void* stream) {
+  return launch_prefill(q, k_cache, v_cache, block_tables, context_lens, q_start, max_q_tokens,
+                        num_kv_heads, scale, block_size, out, static_cast<cudaStream_t>(stream));
 }
 
 int swap_out_blocks(const pkv_tensor* k_cache, const pkv_tensor* v_cache, const pkv_tensor* blocks,

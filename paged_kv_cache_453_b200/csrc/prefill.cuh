@@ -1,0 +1,318 @@
+// Multi-token (causal) paged attention for sm_100a: several new tokens of a
+// sequence attend over its paged cache in one call (a prompt or a chunk of
+// it after its K/V went into the blocks allocated for it, "How Block Paging
+// Operates During Generation" and "Dynamic Request Insertion"; speculative
+// tokens being verified). Sequence s has n_s new tokens, the last n_s of its
+// L_s; query row q_start[s] + j is the token at position L_s - n_s + j and
+// attends to positions 0 .. L_s - n_s + j through the block table.
+//
+// One CTA per (sequence, kv head, chunk of NW * 16 query columns), a column
+// being one query head of one new token (token-major). NW warps of 16
+// columns (two 8-column n-tiles) share a ring of NS stages that holds one
+// block's K and V tiles (TMA, 128-byte swizzle; warp 0 issues, every warp
+// reads every stage), so each K/V byte crosses HBM once per chunk. Per
+// 16-token tile: S^T = K Q^T (K fragments shared by the n-tiles), keys past a
+// column's position masked to -inf (blocks wholly before the chunk's first
+// position need no mask), online softmax per column in the exp2 domain,
+// O^T += V^T P^T with V rows past the sequence zeroed. Each column's output
+// row is normalised and written at the end.
+#pragma once
+
+#include "cascade.cuh"
+
+namespace pkv {
+
+struct PrefillParams {
+  CUtensorMap tmk;  // K pool viewed as {D, B, Hk, NB}
+  CUtensorMap tmv;
+  const void* q;
+  long long q_t, q_h;  // element strides of q [T, Hq, D]
+  void* out;
+  long long o_t, o_h;
+  const int* tables;
+  long long t_s;
+  const int* lens;
+  const int* q_start;  // [S + 1]
+  float scale_log2;
+  int S, T, Hk, g, NB, MB;
+  int evict_first;  // L2 hint for K/V tiles: 1 when one chunk reads them
+  int* err;
+};
+
+template <bool QBF, int D, int BS, int NS, int NW>
+struct PrefillCfg {
+  static constexpr int EPR = 64;
+  static constexpr int NH = (D * 2) / 128;
+  static constexpr int TILE = BS * D * 2;
+  static constexpr int STAGE = 2 * TILE;
+  static constexpr int KS = D / 16;
+  static constexpr int MT = D / 16;
+  static constexpr int TT = BS / 16;
+  static constexpr int COLS = NW * 16;
+  static constexpr int SMEM = 1024 + NS * STAGE + 2 * NS * 8;
+  static_assert(D % 64 == 0 && BS % 16 == 0, "head_dim multiple of 64, block_size of 16");
+};
+
+template <bool QBF, int D, int BS, int NS, int NW>
+__global__ void __launch_bounds__(NW * 32, 1) prefill_kernel(const __grid_constant__ PrefillParams p) {
+  using C = PrefillCfg<QBF, D, BS, NS, NW>;
+  constexpr uint64_t kWaitNs = 2000000000ull;
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t sbase = (smem_addr(smem_raw) + 1023u) & ~1023u;
+  const uint32_t full = sbase + NS * C::STAGE;
+  const uint32_t empty = full + NS * 8;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int r = lane >> 2, c = lane & 3;
+  const long long sh = static_cast<long long>(blockIdx.z) * gridDim.y + blockIdx.y;
+  const int s = static_cast<int>(sh / p.Hk), h = static_cast<int>(sh % p.Hk);
+
+  pdl_launch_dependents();
+  if (tid == 0) {
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(full + i * 8, 1);
+      mbar_init(empty + i * 8, NW);
+    }
+    tma_prefetch_desc(&p.tmk);
+    tma_prefetch_desc(&p.tmv);
+  }
+  fence_mbar_init();
+  __syncthreads();
+  pdl_wait();
+  if (s >= p.S) return;
+
+  const int q0 = __ldg(p.q_start + s), q1 = __ldg(p.q_start + s + 1);
+  const int L = __ldg(p.lens + s);
+  const int n = q1 - q0;
+  if (n < 0 || L < n || L > p.MB * BS || q0 < 0 || q1 > p.T) {
+    if (tid == 0 && blockIdx.x == 0) atomicOr(p.err, kErrBadLen);
+    return;
+  }
+  const int cols = n * p.g;
+  const int col0 = blockIdx.x * C::COLS;
+  if (col0 >= cols) return;
+  const int cend = min(cols, col0 + C::COLS);
+  const int lim_max = L - n + (cend - 1) / p.g;   // last position any column attends to
+  const int lim_min = L - n + col0 / p.g;         // first column's position
+  const int nblk = lim_max / BS + 1;
+  const int plain_blocks = (lim_min + 1) / BS;    // blocks no column needs masked
+
+  // warp 0: table entries of blocks 32w .. 32w + 31 (window w) and the next
+  int win = 0, tw_cur = 0, tw_nxt = 0;
+  const int* trow = p.tables + s * p.t_s;
+  if (warp == 0) {
+    tw_cur = lane < nblk ? __ldg(trow + lane) : 0;
+    tw_nxt = 32 + lane < nblk ? __ldg(trow + 32 + lane) : 0;
+  }
+  const uint64_t policy = p.evict_first ? l2_policy_evict_first() : l2_policy_evict_normal();
+  auto issue = [&](int b) {  // warp 0, all lanes: block b into stage b % NS
+    if ((b >> 5) != win) {   // next window: shift, fetch the one after
+      win = b >> 5;
+      tw_cur = tw_nxt;
+      const int nb2 = 32 * (win + 1) + lane;
+      tw_nxt = nb2 < nblk ? __ldg(trow + nb2) : 0;
+    }
+    int phys = __shfl_sync(0xffffffffu, tw_cur, b & 31);
+    if (phys < 0 || phys >= p.NB) {
+      if (lane == 0) atomicOr(p.err, kErrBadBlock);
+      phys = 0;
+    }
+    if (lane == 0) {
+      const int stage = b % NS;
+      const uint32_t bar = full + stage * 8;
+      const uint32_t dk = sbase + stage * C::STAGE, dv = dk + C::TILE;
+      mbar_arrive_expect_tx(bar, C::STAGE);
+#pragma unroll
+      for (int hh = 0; hh < C::NH; ++hh)
+        tma_load_4d(dk + hh * BS * 128, &p.tmk, bar, hh * C::EPR, 0, h, phys, policy);
+#pragma unroll
+      for (int hh = 0; hh < C::NH; ++hh)
+        tma_load_4d(dv + hh * BS * 128, &p.tmv, bar, hh * C::EPR, 0, h, phys, policy);
+    }
+  };
+  int issued = 0;
+  if (warp == 0) {
+    for (; issued < min(NS, nblk); ++issued) issue(issued);
+  }
+
+  // Q^T fragments of this warp's columns; lane r carries column 8 jt + r.
+  const bool active = col0 + warp * 16 < cols;
+  uint32_t qb[2][C::KS][2];
+  int lim[2][2];  // positions of this lane's two accumulator columns per n-tile
+  bool col_ok[2][2];
+#pragma unroll
+  for (int jt = 0; jt < 2; ++jt) {
+    const int col = col0 + warp * 16 + jt * 8 + r;
+    const bool ok = col < cols;
+    const int tok = ok ? col / p.g : 0;
+    const uint32_t* qp = reinterpret_cast<const uint32_t*>(
+        static_cast<const uint16_t*>(p.q) + (q0 + tok) * p.q_t +
+        (static_cast<long long>(h) * p.g + (ok ? col % p.g : 0)) * p.q_h);
+#pragma unroll
+    for (int ks = 0; ks < C::KS; ++ks) {
+      qb[jt][ks][0] = ok ? __ldg(qp + (ks * 16 + 2 * c) / 2) : 0u;
+      qb[jt][ks][1] = ok ? __ldg(qp + (ks * 16 + 8 + 2 * c) / 2) : 0u;
+    }
+    const int cb0 = col0 + warp * 16 + jt * 8 + 2 * c;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      col_ok[jt][u] = cb0 + u < cols;
+      // a column past the end attends like the last one (finite, not written)
+      lim[jt][u] = col_ok[jt][u] ? L - n + (cb0 + u) / p.g : lim_max;
+    }
+  }
+
+  float acc[2][C::MT][4];
+  float mrun[2][2], lrun[2][2];
+#pragma unroll
+  for (int jt = 0; jt < 2; ++jt) {
+#pragma unroll
+    for (int mt = 0; mt < C::MT; ++mt) acc[jt][mt][0] = acc[jt][mt][1] = acc[jt][mt][2] = acc[jt][mt][3] = 0.f;
+    mrun[jt][0] = mrun[jt][1] = -INFINITY;
+    lrun[jt][0] = lrun[jt][1] = 0.f;
+  }
+  const float sl = p.scale_log2;
+  int jfail = nblk;
+
+  for (int b = 0; b < nblk; ++b) {
+    const int stage = b % NS;
+    const uint32_t parity = static_cast<uint32_t>((b / NS) & 1);
+    if (!warp_wait(full + stage * 8, parity, kWaitNs)) {
+      if (lane == 0) atomicOr(p.err, kErrWaitTimeout);
+      jfail = b;
+      break;
+    }
+    if (active) {
+      const uint32_t tk = sbase + stage * C::STAGE, tv = tk + C::TILE;
+      const bool masked = b >= plain_blocks;
+      const int nvalid = min(BS, L - b * BS);  // rows holding tokens
+#pragma unroll
+      for (int tt = 0; tt < C::TT; ++tt) {
+        float sacc[2][4];
+#pragma unroll
+        for (int jt = 0; jt < 2; ++jt) sacc[jt][0] = sacc[jt][1] = sacc[jt][2] = sacc[jt][3] = 0.f;
+        const int trow = tt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+        for (int ks = 0; ks < C::KS; ++ks) {
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(tk + swz<BS>(trow, ks * 32 + (lane >> 4) * 16), a0, a1, a2, a3);
+#pragma unroll
+          for (int jt = 0; jt < 2; ++jt) mma16816<QBF>(sacc[jt], a0, a1, a2, a3, qb[jt][ks][0], qb[jt][ks][1]);
+        }
+        const int k0 = b * BS + tt * 16 + r, k1 = k0 + 8;  // keys of this lane's rows
+        uint32_t pb[2][2];
+#pragma unroll
+        for (int jt = 0; jt < 2; ++jt) {
+          float x0 = sacc[jt][0] * sl, x1 = sacc[jt][1] * sl, x2 = sacc[jt][2] * sl, x3 = sacc[jt][3] * sl;
+          if (masked) {
+            x0 = k0 <= lim[jt][0] ? x0 : -INFINITY;
+            x1 = k0 <= lim[jt][1] ? x1 : -INFINITY;
+            x2 = k1 <= lim[jt][0] ? x2 : -INFINITY;
+            x3 = k1 <= lim[jt][1] ? x3 : -INFINITY;
+          }
+          float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+          for (int o = 4; o < 32; o <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+          }
+          // finite from the first tile on: key 0 is every column's
+          const float mn0 = fmaxf(mrun[jt][0], mx0), mn1 = fmaxf(mrun[jt][1], mx1);
+          const float al0 = exp2f(mrun[jt][0] - mn0), al1 = exp2f(mrun[jt][1] - mn1);
+          lrun[jt][0] *= al0;
+          lrun[jt][1] *= al1;
+#pragma unroll
+          for (int mt = 0; mt < C::MT; ++mt) {
+            acc[jt][mt][0] *= al0;
+            acc[jt][mt][1] *= al1;
+            acc[jt][mt][2] *= al0;
+            acc[jt][mt][3] *= al1;
+          }
+          mrun[jt][0] = mn0;
+          mrun[jt][1] = mn1;
+          const float p0 = exp2f(x0 - mn0), p1 = exp2f(x1 - mn1);
+          const float p2 = exp2f(x2 - mn0), p3 = exp2f(x3 - mn1);
+          lrun[jt][0] += p0 + p2;
+          lrun[jt][1] += p1 + p3;
+          pb[jt][0] = movmatrix_t(pack2<QBF>(p0, p1));
+          pb[jt][1] = movmatrix_t(pack2<QBF>(p2, p3));
+        }
+        // V rows past the sequence's tokens zeroed (their P is 0, a NaN
+        // there would still poison the sum)
+        const int tb = tt * 16 + 2 * c;
+        const uint32_t keep01 = (tb < nvalid ? 0x0000ffffu : 0u) | (tb + 1 < nvalid ? 0xffff0000u : 0u);
+        const uint32_t keep23 = (tb + 8 < nvalid ? 0x0000ffffu : 0u) | (tb + 9 < nvalid ? 0xffff0000u : 0u);
+#pragma unroll
+        for (int i = 0; i < C::MT; ++i) {
+          const int vrow = tt * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
+          uint32_t f0, f1, f2, f3;
+          ldsm_x4_t(tv + swz<BS>(vrow, i * 32 + ((lane >> 3) & 1) * 16), f0, f1, f2, f3);
+          f0 &= keep01;
+          f1 &= keep01;
+          f2 &= keep23;
+          f3 &= keep23;
+#pragma unroll
+          for (int jt = 0; jt < 2; ++jt) mma16816<QBF>(acc[jt][i], f0, f1, f2, f3, pb[jt][0], pb[jt][1]);
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty + stage * 8);
+    if (warp == 0 && b + NS < nblk) {
+      // refill once every warp has read the stage
+      bool ok = true;
+      if (lane == 0) ok = lane_wait(empty + stage * 8, parity, kWaitNs);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) {
+        if (lane == 0) atomicOr(p.err, kErrWaitTimeout);
+      } else {
+        issue(b + NS);
+        ++issued;
+      }
+    }
+  }
+  if (jfail < nblk) {
+    // copies still in flight (issued, not waited for) land before the CTA's
+    // shared memory is reused
+    if (warp == 0 && lane == 0)
+      for (int i = jfail; i < issued; ++i)
+        lane_wait(full + (i % NS) * 8, static_cast<uint32_t>((i / NS) & 1), 100000000ull);
+    return;
+  }
+  if (!active) return;
+
+#pragma unroll
+  for (int jt = 0; jt < 2; ++jt) {
+    float l0 = lrun[jt][0], l1 = lrun[jt][1];
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+    }
+    const float i0 = l0 > 0.f ? 1.f / l0 : 0.f, i1 = l1 > 0.f ? 1.f / l1 : 0.f;
+    const int cb0 = col0 + warp * 16 + jt * 8 + 2 * c;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (!col_ok[jt][u]) continue;
+      const int col = cb0 + u;
+      uint16_t* o = static_cast<uint16_t*>(p.out) + (q0 + col / p.g) * p.o_t +
+                    (static_cast<long long>(h) * p.g + col % p.g) * p.o_h;
+      const float inv = u ? i1 : i0;
+#pragma unroll
+      for (int mt = 0; mt < C::MT; ++mt) {
+        const float x = acc[jt][mt][u] * inv, y = acc[jt][mt][u + 2] * inv;
+        const int da = 16 * mt + r, db = da + 8;
+        if constexpr (QBF) {
+          o[da] = __bfloat16_as_ushort(__float2bfloat16_rn(x));
+          o[db] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
+        } else {
+          o[da] = __half_as_ushort(__float2half_rn(x));
+          o[db] = __half_as_ushort(__float2half_rn(y));
+        }
+      }
+    }
+  }
+}
+
+}  // namespace pkv

@@ -1,0 +1,112 @@
+"""Multi-token (causal) paged attention on the GPU against the fp64 oracle
+(paged_prefill), through the C ABI. Tolerances as for the decode."""
+import numpy as np
+import pytest
+import torch
+
+import paged_kv_cache_453_b200 as P
+import workloads as W
+from gpu_cases import TOL, check_no_device_error, max_err
+from oracle.attention import paged_prefill
+from oracle_io import raw
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def setup():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from paged_kv_cache_453_b200.build import build
+    build()
+
+
+def _case(spec, nq, seed=5):
+    """Layout and pool from the workload; nq[s] new tokens per sequence (the
+    last ones of its context), their queries drawn here."""
+    s = spec.replace(append=False)
+    lay = W.make_layout(s, seed=seed)
+    t = W.make_tensors(s, lay.num_blocks, lay.tables, lay.lens, device="cuda", seed=seed)
+    nq = [min(int(n), int(L)) for n, L in zip(nq, lay.lens.tolist())]
+    q_start = torch.tensor(np.concatenate([[0], np.cumsum(nq)]), dtype=torch.int32)
+    T = int(q_start[-1])
+    g = torch.Generator(device="cuda").manual_seed(seed + 1)
+    dt = {"f16": torch.float16, "bf16": torch.bfloat16}[s.q_dtype]
+    q = torch.randn((T, s.num_q_heads, s.head_dim), generator=g, device="cuda").to(dt)
+    return s, lay, t, q, q_start, max(nq) if nq else 0
+
+
+def _run(s, lay, t, q, q_start, max_q):
+    out = torch.full_like(q, float("nan"))
+    P.paged_attn_prefill(q, t.k_cache, t.v_cache, lay.tables.cuda(), lay.lens.cuda(), q_start.cuda(), max_q,
+                         s.num_kv_heads, s.scale, s.block_size, out)
+    torch.cuda.synchronize()
+    return out
+
+
+def _oracle(s, lay, t, q, q_start, seqs=None):
+    return paged_prefill(raw(q), raw(t.k_cache), raw(t.v_cache), lay.tables.numpy(), lay.lens.numpy(),
+                         q_start.numpy(), s.scale, s.block_size, s.q_dtype, s.cache_dtype, seqs=seqs)
+
+
+CASES = {
+    # spec, new tokens per sequence
+    "verify_gqa": (W.scaled_down(W.spec("llama3_8b"), 8, 900), [4] * 8),
+    "verify_g8_b32": (W.scaled_down(W.spec("llama3_70b"), 4, 700, block_size=32).replace(lens=("uniform", 40, 700)),
+                      [5, 1, 7, 3]),
+    "chunk_mha_f16": (W.spec("llama3_8b").replace(num_seqs=3, num_q_heads=4, num_kv_heads=4, cache_dtype="f16",
+                                                  q_dtype="f16", lens=("fixed", [700, 300, 129]), table_width=None),
+                      [300, 300, 17]),
+    "whole_prompt_d64": (W.spec("tiny").replace(cache_dtype="bf16", q_dtype="bf16", block_size=32,
+                                                lens=("fixed", [1, 33, 64, 70]), pool_blocks=None),
+                         [1, 33, 64, 70]),
+    "mixed_counts": (W.spec("llama3_8b").replace(num_seqs=6, lens=("fixed", [16, 17, 1, 500, 48, 2]),
+                                                 table_width=None),
+                     [16, 0, 1, 40, 33, 2]),
+}
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_prefill_matches_oracle(name):
+    spec, nq = CASES[name]
+    s, lay, t, q, q_start, max_q = _case(spec, nq)
+    out = _run(s, lay, t, q, q_start, max_q)
+    check_no_device_error()
+    ref = _oracle(s, lay, t, q, q_start)
+    assert max_err(out, ref) <= TOL[s.cache_dtype], name
+
+
+def test_one_token_per_sequence_is_the_decode_step():
+    spec = W.scaled_down(W.spec("llama3_8b"), 8, 700)
+    s, lay, t, q, q_start, max_q = _case(spec, [1] * 8)
+    out = _run(s, lay, t, q, q_start, max_q)
+    dec = torch.full_like(q, float("nan"))
+    P.paged_attn_decode(q, t.k_cache, t.v_cache, lay.tables.cuda(), lay.lens.cuda(), s.num_kv_heads, s.scale,
+                        s.block_size, dec)
+    torch.cuda.synchronize()
+    assert (out.float() - dec.float()).abs().max().item() <= TOL[s.cache_dtype]
+    check_no_device_error()
+
+
+def test_full_size_verification_sampled():
+    # llama3_8b-shaped batch verifying 4 speculative tokens per sequence
+    spec = W.spec("llama3_8b")
+    s, lay, t, q, q_start, max_q = _case(spec, [4] * spec.num_seqs)
+    out = _run(s, lay, t, q, q_start, max_q)
+    check_no_device_error()
+    seqs = [0, 17, 40, 63]
+    ref = _oracle(s, lay, t, q, q_start, seqs=seqs)
+    rows = [r for sq in seqs for r in range(int(q_start[sq]), int(q_start[sq + 1]))]
+    assert max_err(out, ref, rows) <= TOL[s.cache_dtype]
+    assert torch.isfinite(out).all()
+
+
+def test_inconsistent_rows_are_flagged():
+    spec = W.scaled_down(W.spec("llama3_8b"), 4, 300)
+    s, lay, t, q, q_start, max_q = _case(spec, [3] * 4)
+    lens = lay.lens.clone()
+    lens[1] = 2                                   # fewer tokens than new ones
+    out = torch.zeros_like(q)
+    P.paged_attn_prefill(q, t.k_cache, t.v_cache, lay.tables.cuda(), lens.cuda(), q_start.cuda(), max_q,
+                         s.num_kv_heads, s.scale, s.block_size, out)
+    assert P.device_error(torch.cuda.current_device()) == P.PKV_ERR_DEVICE_CHECK
+    check_no_device_error()
