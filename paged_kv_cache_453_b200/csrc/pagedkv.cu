@@ -37,6 +37,8 @@ struct DeviceState {
   size_t ws_bytes = 0;
   void* cas = nullptr;  // library-owned prefix-aware decode partials
   size_t cas_bytes = 0;
+  void* pre = nullptr;  // library-owned multi-token partials
+  size_t pre_bytes = 0;
 };
 DeviceState g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -603,6 +605,7 @@ int launch_cascade(const DecodeArgs& a, const pkv_tensor* pblk, const pkv_tensor
 
 struct PrefillLaunch {
   void (*kernel)(PrefillParams);
+  void (*merge)(PrefillParams);
   int threads, smem, cols;
   bool attr_set[kMaxDevices];
 };
@@ -610,7 +613,7 @@ struct PrefillLaunch {
 template <bool QBF, int D, int BS, int NW>
 PrefillLaunch* prefill_entry() {
   constexpr int NS = 4;
-  static PrefillLaunch e = {&prefill_kernel<QBF, D, BS, NS, NW>, NW * 32,
+  static PrefillLaunch e = {&prefill_kernel<QBF, D, BS, NS, NW>, &prefill_merge_kernel<QBF, D>, NW * 32,
                             PrefillCfg<QBF, D, BS, NS, NW>::SMEM, NW * 16, {false}};
   return &e;
 }
@@ -660,7 +663,7 @@ int launch_prefill(const pkv_tensor* q, const pkv_tensor* kc, const pkv_tensor* 
     return PKV_ERR_INVALID_ARG;
   const int64_t g = Hq / Hk;
   if ((D != 64 && D != 128) || (BS != 16 && BS != 32)) return PKV_ERR_UNSUPPORTED;
-  if (NB > INT32_MAX || T > INT32_MAX || S * Hk > 65535LL * 65535LL ||
+  if (NB > INT32_MAX || T > INT32_MAX || S * Hk > 65535LL || S > 65535LL ||
       static_cast<int64_t>(max_q) * g > INT32_MAX / 2)
     return PKV_ERR_UNSUPPORTED;
   if (S == 0 || T == 0 || max_q == 0) return PKV_OK;
@@ -702,23 +705,52 @@ int launch_prefill(const pkv_tensor* q, const pkv_tensor* kc, const pkv_tensor* 
   p.g = static_cast<int>(g);
   p.NB = static_cast<int>(NB);
   p.MB = static_cast<int>(bt->shape[1]);
+  p.BS = BS;
   const int ncc = (cols + e->cols - 1) / e->cols;
   p.evict_first = ncc == 1;
   p.err = ds->err;
-  const long long sh = S * Hk;
-  const unsigned gy = static_cast<unsigned>(std::min<long long>(sh, 65535));
-  const unsigned gz = static_cast<unsigned>((sh + gy - 1) / gy);
+  p.ccols = e->cols;
+  // Few CTAs over long, uneven contexts (short queries): cut each (sequence,
+  // head)'s blocks into chunks of 32 (512 or 1024 tokens) so the CTAs are
+  // many and even; the partials are merged by a second kernel.
+  p.nkv = 1;
+  const long long ctas = S * Hk * ncc;
+  if (ctas < 4LL * ds->sms && bt->shape[1] > 32) {
+    p.kv_chunk = 32;
+    p.nkv = static_cast<int>((bt->shape[1] + p.kv_chunk - 1) / p.kv_chunk);
+    if (p.nkv > 65535) return PKV_ERR_UNSUPPORTED;
+    const size_t rows = static_cast<size_t>(T) * Hq * p.nkv;
+    const size_t po = 0, pm = round_up(rows * D * 4, 256), total = round_up(pm + rows * 2 * 4, 256);
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (ds->pre_bytes < total) {
+      if (ds->pre) cudaFree(ds->pre);
+      ds->pre = nullptr;
+      ds->pre_bytes = 0;
+      if (cudaMalloc(&ds->pre, total) != cudaSuccess) return PKV_ERR_CUDA;
+      ds->pre_bytes = total;
+    }
+    p.part_o = reinterpret_cast<float*>(static_cast<uint8_t*>(ds->pre) + po);
+    p.part_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(ds->pre) + pm);
+  }
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(ncc), gy, gz);
+  cfg.gridDim = dim3(static_cast<unsigned>(ncc), static_cast<unsigned>(p.nkv), static_cast<unsigned>(S * Hk));
   cfg.blockDim = dim3(static_cast<unsigned>(e->threads));
   cfg.dynamicSmemBytes = static_cast<size_t>(e->smem);
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, e->kernel, p) != cudaSuccess) return PKV_ERR_CUDA;
+  if (p.nkv > 1) {
+    const long long warps = static_cast<long long>(max_q) * Hq;
+    if ((warps + 3) / 4 > INT32_MAX) return PKV_ERR_UNSUPPORTED;
+    cfg.gridDim = dim3(static_cast<unsigned>((warps + 3) / 4), static_cast<unsigned>(S));
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = 0;
+    if (cudaLaunchKernelEx(&cfg, e->merge, p) != cudaSuccess) return PKV_ERR_CUDA;
+  }
   return PKV_OK;
 }
 

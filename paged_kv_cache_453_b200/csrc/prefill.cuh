@@ -16,6 +16,12 @@
 // position need no mask), online softmax per column in the exp2 domain,
 // O^T += V^T P^T with V rows past the sequence zeroed. Each column's output
 // row is normalised and written at the end.
+//
+// Short queries over long, uneven contexts (speculative verification) give
+// too few, unequal CTAs; there the blocks of each (sequence, head) are also
+// cut into chunks of kv_chunk blocks, one CTA each, which leave fp32
+// partials (m, l, unnormalised O) per column, and prefill_merge_kernel folds
+// a row's chunks with the log-sum-exp rule.
 #pragma once
 
 #include "cascade.cuh"
@@ -34,9 +40,14 @@ struct PrefillParams {
   const int* lens;
   const int* q_start;  // [S + 1]
   float scale_log2;
-  int S, T, Hk, g, NB, MB;
+  int S, T, Hk, g, NB, MB, BS;
   int evict_first;  // L2 hint for K/V tiles: 1 when one chunk reads them
   int* err;
+  int nkv;          // KV chunks per (sequence, head); 1: no split, outputs written directly
+  int ccols;        // query columns per CTA (the kernel's NW * 16)
+  int kv_chunk;     // blocks per KV chunk (split only)
+  float* part_o;    // [T * Hq * nkv][D] (split only)
+  float* part_ml;   // [T * Hq * nkv][2]
 };
 
 template <bool QBF, int D, int BS, int NS, int NW>
@@ -65,8 +76,10 @@ __global__ void __launch_bounds__(NW * 32, 1) prefill_kernel(const __grid_consta
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int r = lane >> 2, c = lane & 3;
-  const long long sh = static_cast<long long>(blockIdx.z) * gridDim.y + blockIdx.y;
+  // grid: x = column chunk, y = KV chunk, z = (sequence, head)
+  const long long sh = blockIdx.z;
   const int s = static_cast<int>(sh / p.Hk), h = static_cast<int>(sh % p.Hk);
+  const int kc = blockIdx.y;
 
   pdl_launch_dependents();
   if (tid == 0) {
@@ -91,27 +104,34 @@ __global__ void __launch_bounds__(NW * 32, 1) prefill_kernel(const __grid_consta
   }
   const int cols = n * p.g;
   const int col0 = blockIdx.x * C::COLS;
+  if (tid == 0 && blockIdx.x == 0 && kc == 0 && cols > static_cast<int>(gridDim.x) * C::COLS)
+    atomicOr(p.err, kErrBadLen);  // more new tokens than max_q_tokens
   if (col0 >= cols) return;
   const int cend = min(cols, col0 + C::COLS);
   const int lim_max = L - n + (cend - 1) / p.g;   // last position any column attends to
   const int lim_min = L - n + col0 / p.g;         // first column's position
-  const int nblk = lim_max / BS + 1;
+  const int nblk_all = lim_max / BS + 1;
   const int plain_blocks = (lim_min + 1) / BS;    // blocks no column needs masked
+  const int b_lo = p.nkv > 1 ? kc * p.kv_chunk : 0;
+  const int b_hi = p.nkv > 1 ? min(nblk_all, b_lo + p.kv_chunk) : nblk_all;
+  if (b_lo >= b_hi) return;                       // no keys of this chunk here
+  const int nblk = b_hi - b_lo;                    // blocks b_lo + j, j < nblk
 
   // warp 0: table entries of blocks 32w .. 32w + 31 (window w) and the next
-  int win = 0, tw_cur = 0, tw_nxt = 0;
+  int win = b_lo >> 5, tw_cur = 0, tw_nxt = 0;
   const int* trow = p.tables + s * p.t_s;
   if (warp == 0) {
-    tw_cur = lane < nblk ? __ldg(trow + lane) : 0;
-    tw_nxt = 32 + lane < nblk ? __ldg(trow + 32 + lane) : 0;
+    tw_cur = 32 * win + lane < nblk_all ? __ldg(trow + 32 * win + lane) : 0;
+    tw_nxt = 32 * (win + 1) + lane < nblk_all ? __ldg(trow + 32 * (win + 1) + lane) : 0;
   }
   const uint64_t policy = p.evict_first ? l2_policy_evict_first() : l2_policy_evict_normal();
-  auto issue = [&](int b) {  // warp 0, all lanes: block b into stage b % NS
+  auto issue = [&](int j) {  // warp 0, all lanes: block b_lo + j into stage j % NS
+    const int b = b_lo + j;
     if ((b >> 5) != win) {   // next window: shift, fetch the one after
       win = b >> 5;
       tw_cur = tw_nxt;
       const int nb2 = 32 * (win + 1) + lane;
-      tw_nxt = nb2 < nblk ? __ldg(trow + nb2) : 0;
+      tw_nxt = nb2 < nblk_all ? __ldg(trow + nb2) : 0;
     }
     int phys = __shfl_sync(0xffffffffu, tw_cur, b & 31);
     if (phys < 0 || phys >= p.NB) {
@@ -119,7 +139,7 @@ __global__ void __launch_bounds__(NW * 32, 1) prefill_kernel(const __grid_consta
       phys = 0;
     }
     if (lane == 0) {
-      const int stage = b % NS;
+      const int stage = j % NS;
       const uint32_t bar = full + stage * 8;
       const uint32_t dk = sbase + stage * C::STAGE, dv = dk + C::TILE;
       mbar_arrive_expect_tx(bar, C::STAGE);
@@ -175,12 +195,13 @@ __global__ void __launch_bounds__(NW * 32, 1) prefill_kernel(const __grid_consta
   const float sl = p.scale_log2;
   int jfail = nblk;
 
-  for (int b = 0; b < nblk; ++b) {
-    const int stage = b % NS;
-    const uint32_t parity = static_cast<uint32_t>((b / NS) & 1);
+  for (int j = 0; j < nblk; ++j) {
+    const int b = b_lo + j;
+    const int stage = j % NS;
+    const uint32_t parity = static_cast<uint32_t>((j / NS) & 1);
     if (!warp_wait(full + stage * 8, parity, kWaitNs)) {
       if (lane == 0) atomicOr(p.err, kErrWaitTimeout);
-      jfail = b;
+      jfail = j;
       break;
     }
     if (active) {
@@ -217,9 +238,12 @@ __global__ void __launch_bounds__(NW * 32, 1) prefill_kernel(const __grid_consta
             mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
             mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
           }
-          // finite from the first tile on: key 0 is every column's
+          // A column with no key yet (every key so far past its position, only
+          // in a later KV chunk) keeps m = -inf, l = 0, O = 0: the exponent
+          // base is then 0 instead of -inf.
           const float mn0 = fmaxf(mrun[jt][0], mx0), mn1 = fmaxf(mrun[jt][1], mx1);
-          const float al0 = exp2f(mrun[jt][0] - mn0), al1 = exp2f(mrun[jt][1] - mn1);
+          const float b0 = mn0 == -INFINITY ? 0.f : mn0, b1 = mn1 == -INFINITY ? 0.f : mn1;
+          const float al0 = exp2f(mrun[jt][0] - b0), al1 = exp2f(mrun[jt][1] - b1);
           lrun[jt][0] *= al0;
           lrun[jt][1] *= al1;
 #pragma unroll
@@ -231,8 +255,8 @@ __global__ void __launch_bounds__(NW * 32, 1) prefill_kernel(const __grid_consta
           }
           mrun[jt][0] = mn0;
           mrun[jt][1] = mn1;
-          const float p0 = exp2f(x0 - mn0), p1 = exp2f(x1 - mn1);
-          const float p2 = exp2f(x2 - mn0), p3 = exp2f(x3 - mn1);
+          const float p0 = exp2f(x0 - b0), p1 = exp2f(x1 - b1);
+          const float p2 = exp2f(x2 - b0), p3 = exp2f(x3 - b1);
           lrun[jt][0] += p0 + p2;
           lrun[jt][1] += p1 + p3;
           pb[jt][0] = movmatrix_t(pack2<QBF>(p0, p1));
@@ -259,7 +283,7 @@ __global__ void __launch_bounds__(NW * 32, 1) prefill_kernel(const __grid_consta
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(empty + stage * 8);
-    if (warp == 0 && b + NS < nblk) {
+    if (warp == 0 && j + NS < nblk) {
       // refill once every warp has read the stage
       bool ok = true;
       if (lane == 0) ok = lane_wait(empty + stage * 8, parity, kWaitNs);
@@ -267,7 +291,7 @@ __global__ void __launch_bounds__(NW * 32, 1) prefill_kernel(const __grid_consta
       if (!ok) {
         if (lane == 0) atomicOr(p.err, kErrWaitTimeout);
       } else {
-        issue(b + NS);
+        issue(j + NS);
         ++issued;
       }
     }
@@ -292,6 +316,26 @@ __global__ void __launch_bounds__(NW * 32, 1) prefill_kernel(const __grid_consta
     }
     const float i0 = l0 > 0.f ? 1.f / l0 : 0.f, i1 = l1 > 0.f ? 1.f / l1 : 0.f;
     const int cb0 = col0 + warp * 16 + jt * 8 + 2 * c;
+    if (p.nkv > 1) {  // partials of this KV chunk
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        if (!col_ok[jt][u]) continue;
+        const int col = cb0 + u;
+        const long long row = (static_cast<long long>(q0 + col / p.g) * (p.Hk * p.g) +
+                               static_cast<long long>(h) * p.g + col % p.g) * p.nkv + kc;
+        float* po = p.part_o + row * D;
+#pragma unroll
+        for (int mt = 0; mt < C::MT; ++mt) {
+          po[16 * mt + r] = acc[jt][mt][u];
+          po[16 * mt + r + 8] = acc[jt][mt][u + 2];
+        }
+        if (r == 0) {
+          p.part_ml[row * 2] = mrun[jt][u];
+          p.part_ml[row * 2 + 1] = u ? l1 : l0;
+        }
+      }
+      continue;
+    }
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       if (!col_ok[jt][u]) continue;
@@ -312,6 +356,88 @@ __global__ void __launch_bounds__(NW * 32, 1) prefill_kernel(const __grid_consta
         }
       }
     }
+  }
+}
+
+// One warp per (new token row, query head), grid (rows x heads of a
+// sequence, sequences): fold the row's KV-chunk partials (chunks whose keys
+// all lie past the row's position hold m = -inf and are skipped) and write
+// the normalised output.
+template <bool QBF, int D>
+__global__ void __launch_bounds__(128) prefill_merge_kernel(const __grid_constant__ PrefillParams p) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int lane = threadIdx.x & 31;
+  const long long wid = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int s = blockIdx.y;
+  const int Hq = p.Hk * p.g;
+  const int q0 = __ldg(p.q_start + s), q1 = __ldg(p.q_start + s + 1);
+  const int L = __ldg(p.lens + s);
+  const int n = q1 - q0;
+  if (n < 0 || L < n || L > p.MB * p.BS || q0 < 0 || q1 > p.T) return;  // flagged by the kernel
+  if (wid >= static_cast<long long>(n) * Hq) return;
+  const int j = static_cast<int>(wid / Hq), hq = static_cast<int>(wid % Hq);
+  const long long row = (static_cast<long long>(q0 + j) * Hq + hq) * p.nkv;
+  // chunks written for this row: those with keys before the last position of
+  // its column chunk (the kernel's CTA covers the whole column chunk)
+  const int cols = n * p.g, col = j * p.g + hq % p.g;
+  const int cend = min(cols, (col / p.ccols + 1) * p.ccols);
+  const int nblk_all = (L - n + (cend - 1) / p.g) / p.BS + 1;
+  const int nk = min(p.nkv, (nblk_all + p.kv_chunk - 1) / p.kv_chunk);
+  constexpr int V = D / 32;
+  float mx = -INFINITY, lsum = 0.f, a[V];
+#pragma unroll
+  for (int v = 0; v < V; ++v) a[v] = 0.f;
+  for (int base = 0; base < nk; base += 32) {
+    const int k = base + lane;
+    float m = -INFINITY, l = 0.f;
+    if (k < nk) {
+      m = p.part_ml[(row + k) * 2];
+      l = p.part_ml[(row + k) * 2 + 1];
+    }
+    float cm = m;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, o));
+    if (cm == -INFINITY) continue;
+    const float mn = fmaxf(mx, cm);
+    const float sa = mx == -INFINITY ? 0.f : exp2f(mx - mn);
+    lsum *= sa;
+#pragma unroll
+    for (int v = 0; v < V; ++v) a[v] *= sa;
+    mx = mn;
+    const float w = m == -INFINITY ? 0.f : exp2f(m - mn);
+    float lw = l * w;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, o);
+    lsum += lw;
+    const int cnt = min(32, nk - base);
+    for (int k0 = 0; k0 < cnt; k0 += 8) {
+      float x[8][V], wk[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        wk[u] = __shfl_sync(0xffffffffu, w, (k0 + u) & 31);
+        if (k0 + u < cnt && wk[u] != 0.f) {
+          const float* o = p.part_o + (row + base + k0 + u) * D;
+#pragma unroll
+          for (int v = 0; v < V; ++v) x[u][v] = o[lane * V + v];
+        } else {
+#pragma unroll
+          for (int v = 0; v < V; ++v) x[u][v] = 0.f;
+          wk[u] = 0.f;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+#pragma unroll
+        for (int v = 0; v < V; ++v) a[v] += x[u][v] * wk[u];
+    }
+  }
+  const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+  uint16_t* oh = static_cast<uint16_t*>(p.out) + (q0 + j) * p.o_t + hq * p.o_h + lane * V;
+#pragma unroll
+  for (int v = 0; v < V; ++v) {
+    if constexpr (QBF) oh[v] = __bfloat16_as_ushort(__float2bfloat16_rn(a[v] * inv));
+    else oh[v] = __half_as_ushort(__float2half_rn(a[v] * inv));
   }
 }
 
