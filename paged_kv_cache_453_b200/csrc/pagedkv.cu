@@ -18,6 +18,7 @@
 #include "cache_ops.cuh"
 #include "cascade.cuh"
 #include "prefill.cuh"
+#include "prefill_tc.cuh"
 #include "decode.cuh"
 
 namespace pkv {
@@ -640,6 +641,24 @@ PrefillLaunch* pick_prefill(bool qbf, int D, int BS, int cols) {
   return nullptr;
 }
 
+// Tensor-core (tcgen05) variant for 128-row query tiles, D = 128.
+struct PrefillTcLaunch {
+  void (*kernel)(PrefillParams);
+  int smem;
+  bool attr_set[kMaxDevices];
+};
+
+template <bool QBF, int BS>
+PrefillTcLaunch* prefill_tc_entry() {
+  static PrefillTcLaunch e = {&prefill_tc_kernel<QBF, BS>, PrefillTcCfg<BS>::SMEM, {false}};
+  return &e;
+}
+
+PrefillTcLaunch* pick_prefill_tc(bool qbf, int BS) {
+  if (qbf) return BS == 16 ? prefill_tc_entry<true, 16>() : prefill_tc_entry<true, 32>();
+  return BS == 16 ? prefill_tc_entry<false, 16>() : prefill_tc_entry<false, 32>();
+}
+
 int launch_prefill(const pkv_tensor* q, const pkv_tensor* kc, const pkv_tensor* vc,
                    const pkv_tensor* bt, const pkv_tensor* cl, const pkv_tensor* qs, int max_q,
                    int Hk, float scale, int BS, pkv_tensor* out, cudaStream_t stream) {
@@ -675,6 +694,11 @@ int launch_prefill(const pkv_tensor* q, const pkv_tensor* kc, const pkv_tensor* 
   if ((st = current_device(&dev)) != PKV_OK) return st;
   DeviceState* ds;
   if ((st = device_state(dev, &ds)) != PKV_OK) return st;
+  // 128-row tiles on the tensor cores when every (sequence, head) may have
+  // that many rows and q / out rows are 16-byte aligned (vector loads)
+  const bool rows16 = q->stride[0] % 8 == 0 && q->stride[1] % 8 == 0 && aligned(q->data, 16) &&
+                      out->stride[0] % 8 == 0 && out->stride[1] % 8 == 0 && aligned(out->data, 16);
+  const bool use_tc = D == 128 && cols >= 128 && rows16;
   {
     std::lock_guard<std::mutex> lk(g_mu);
     if (!e->attr_set[dev]) {
@@ -706,6 +730,31 @@ int launch_prefill(const pkv_tensor* q, const pkv_tensor* kc, const pkv_tensor* 
   p.NB = static_cast<int>(NB);
   p.MB = static_cast<int>(bt->shape[1]);
   p.BS = BS;
+  if (use_tc) {
+    PrefillTcLaunch* te = pick_prefill_tc(qdt == PKV_BF16, BS);
+    {
+      std::lock_guard<std::mutex> lk(g_mu);
+      if (!te->attr_set[dev]) {
+        if (cudaFuncSetAttribute(te->kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, te->smem) !=
+            cudaSuccess)
+          return PKV_ERR_CUDA;
+        te->attr_set[dev] = true;
+      }
+    }
+    p.err = ds->err;
+    p.nkv = 1;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t tc = {};
+    tc.gridDim = dim3(static_cast<unsigned>((cols + 127) / 128), 1, static_cast<unsigned>(S * Hk));
+    tc.blockDim = dim3(128);
+    tc.dynamicSmemBytes = static_cast<size_t>(te->smem);
+    tc.stream = stream;
+    tc.attrs = at;
+    tc.numAttrs = 1;
+    return cudaLaunchKernelEx(&tc, te->kernel, p) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+  }
   const int ncc = (cols + e->cols - 1) / e->cols;
   p.evict_first = ncc == 1;
   p.err = ds->err;

@@ -62,6 +62,13 @@ CASES = {
     "mixed_counts": (W.spec("llama3_8b").replace(num_seqs=6, lens=("fixed", [16, 17, 1, 500, 48, 2]),
                                                  table_width=None),
                      [16, 0, 1, 40, 33, 2]),
+    # 128-row tiles on the tensor cores (D = 128, at least 128 query rows)
+    "tc_chunk_g8_b32": (W.spec("llama3_70b").replace(num_seqs=2, block_size=32, lens=("fixed", [900, 601]),
+                                                     table_width=None),
+                        [300, 129]),
+    "tc_chunk_gqa_f16": (W.spec("llama3_8b").replace(num_seqs=3, cache_dtype="f16", q_dtype="f16",
+                                                     lens=("fixed", [333, 129, 700]), table_width=None),
+                         [333, 64, 250]),
 }
 
 
@@ -94,6 +101,20 @@ def test_full_size_verification_sampled():
     out = _run(s, lay, t, q, q_start, max_q)
     check_no_device_error()
     seqs = [0, 17, 40, 63]
+    ref = _oracle(s, lay, t, q, q_start, seqs=seqs)
+    rows = [r for sq in seqs for r in range(int(q_start[sq]), int(q_start[sq + 1]))]
+    assert max_err(out, ref, rows) <= TOL[s.cache_dtype]
+    assert torch.isfinite(out).all()
+
+
+def test_full_size_chunk_sampled():
+    # llama3_8b-shaped batch with a 64-token chunk per sequence (256 query rows
+    # per kv head: tensor-core tiles)
+    spec = W.spec("llama3_8b")
+    s, lay, t, q, q_start, max_q = _case(spec, [64] * spec.num_seqs)
+    out = _run(s, lay, t, q, q_start, max_q)
+    check_no_device_error()
+    seqs = [3, 31, 62]
     ref = _oracle(s, lay, t, q, q_start, seqs=seqs)
     rows = [r for sq in seqs for r in range(int(q_start[sq]), int(q_start[sq + 1]))]
     assert max_err(out, ref, rows) <= TOL[s.cache_dtype]
