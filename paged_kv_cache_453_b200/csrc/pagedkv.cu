@@ -748,7 +748,7 @@ int launch_prefill(const pkv_tensor* q, const pkv_tensor* kc, const pkv_tensor* 
     at[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t tc = {};
     tc.gridDim = dim3(static_cast<unsigned>((cols + 127) / 128), 1, static_cast<unsigned>(S * Hk));
-    tc.blockDim = dim3(128);
+    tc.blockDim = dim3(256);
     tc.dynamicSmemBytes = static_cast<size_t>(te->smem);
     tc.stream = stream;
     tc.attrs = at;

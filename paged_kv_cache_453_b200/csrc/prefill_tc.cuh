@@ -6,23 +6,27 @@
 // rule); this kernel is used when a (sequence, kv head) has at least 128
 // query rows (new tokens x query heads of the group).
 //
-// CTA = 4 warps, one (sequence, kv head, 128 query rows); a row is one query
-// head of one new token (token-major), and thread r owns row r (tensor
-// memory lane r). Per step of 128 keys (128 / B blocks through the block
-// table):
+// CTA = 8 warps, one (sequence, kv head, 128 query rows); a row is one query
+// head of one new token (token-major). Threads r and r + 128 share row r
+// (tensor-memory lane r; warps w and w + 4 read the same lane quarter), each
+// owning 64 of the 128 columns of S and of O. Per step of 128 keys (128 / B
+// blocks through the block table):
 //   TMA: the blocks' K and V tiles into a two-stage ring, laid out as two
 //        64-column halves of [128 keys x 128 B], 128-byte swizzled
 //   S = Q K^T   8 MMAs (K = 16 each) into tensor-memory columns [0, 128)
-//   softmax     each thread loads its row of S (32 columns at a time), masks
-//               keys past its position, runs the online max / sum in the
-//               exp2 domain, rescales its row of O in tensor memory and
-//               writes P (16-bit) to shared memory in the MMA's layout
+//   softmax     each thread loads its 64 columns of S once (kept in
+//               registers), masks keys past its position, exchanges its
+//               max with the row's other thread, runs the online max / sum
+//               in the exp2 domain (sums kept per half, added at the end),
+//               rescales its half of O in tensor memory and writes its half
+//               of P (16-bit) to shared memory in the MMA's layout
 //   O += P V    8 MMAs into tensor-memory columns [128, 256), V read as an
 //               MN-major operand straight from the TMA tiles
-// The next step's loads are issued as soon as the MMAs of the step before
-// have released their stage. Q rows are loaded once into shared memory.
-// Shared memory: Q 32 KB, K 2 x 32 KB, V 2 x 32 KB, P 32 KB (one CTA per SM);
-// tensor memory: 256 columns.
+// Loads run two steps ahead; S of the next step is issued as soon as this
+// step's S is complete (it runs while this step is reduced: two S buffers in
+// tensor memory), and O += P V overlaps the next step's max. Q rows are
+// loaded once into shared memory. Shared memory: Q 32 KB, K 2 x 32 KB,
+// V 2 x 32 KB, P 32 KB (one CTA per SM); tensor memory: 512 columns.
 #pragma once
 
 #include "prefill.cuh"
@@ -118,33 +122,43 @@ struct PrefillTcCfg {
   // layout from the 1024-aligned base: Q | K0 K1 | V0 V1 | P | barriers | tmem slot
   static constexpr int OFF_Q = 0, OFF_K = TILE, OFF_V = 3 * TILE, OFF_P = 5 * TILE;
   static constexpr int OFF_BAR = 6 * TILE;
-  static constexpr int SMEM = 1024 + 6 * TILE + 64;
+  static constexpr int OFF_X = OFF_BAR + 128;  // [256] floats: row max / sum exchange
+  static constexpr int OFF_PH = OFF_X + 256 * 4;  // [4][BPS] physical blocks, steps mod 4
+  static constexpr int SMEM = 1024 + 6 * TILE + 128 + 256 * 4 + 4 * BPS * 4;
 };
 
 template <bool QBF, int BS>
-__global__ void __launch_bounds__(128, 1) prefill_tc_kernel(const __grid_constant__ PrefillParams p) {
+__global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constant__ PrefillParams p) {
   using C = PrefillTcCfg<BS>;
   constexpr uint64_t kWaitNs = 2000000000ull;
-  constexpr uint32_t kCols = 256;  // tensor-memory columns: S [0, 128), O [128, 256)
+  // tensor-memory columns: S of even steps [0, 128), of odd steps [128, 256),
+  // O [256, 384)
+  constexpr uint32_t kCols = 512;
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t sraw = smem_addr(smem_raw);
   const uint32_t sbase = (sraw + 1023u) & ~1023u;
   uint8_t* sgen = smem_raw + (sbase - sraw);
   const uint32_t sQ = sbase + C::OFF_Q, sP = sbase + C::OFF_P;
-  const uint32_t bar_kv = sbase + C::OFF_BAR;  // [2]: K and V of stage landed
-  const uint32_t bar_s = bar_kv + 16;          // S complete
-  const uint32_t bar_o = bar_kv + 24;          // O += P V complete
-  const uint32_t tslot = bar_kv + 32;          // tensor-memory base address
-  uint32_t* tslot_gen = reinterpret_cast<uint32_t*>(sgen + C::OFF_BAR + 32);
+  const uint32_t bar_k = sbase + C::OFF_BAR;  // [2]: K tile of the stage landed
+  const uint32_t bar_v = bar_k + 16;          // [2]: V tile of the stage landed
+  const uint32_t bar_s = bar_k + 32;          // S of the next step complete
+  const uint32_t bar_o = bar_k + 40;          // O += P V complete
+  const uint32_t tslot = bar_k + 48;          // tensor-memory base address
+  uint32_t* tslot_gen = reinterpret_cast<uint32_t*>(sgen + C::OFF_BAR + 48);
+  float* xch = reinterpret_cast<float*>(sgen + C::OFF_X);
+  int* s_phys = reinterpret_cast<int*>(sgen + C::OFF_PH);
 
   const int tid = threadIdx.x, warp = tid >> 5;
+  const int rl = tid & 127, half = tid >> 7;  // row in the tile, column half
   const int s = static_cast<int>(blockIdx.z / p.Hk), h = static_cast<int>(blockIdx.z % p.Hk);
 
   pdl_launch_dependents();
   if (tid == 0) {
-    mbar_init(bar_kv, 1);
-    mbar_init(bar_kv + 8, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_k + i * 8, 1);
+      mbar_init(bar_v + i * 8, 1);
+    }
     mbar_init(bar_s, 1);
     mbar_init(bar_o, 1);
     tma_prefetch_desc(&p.tmk);
@@ -159,8 +173,9 @@ __global__ void __launch_bounds__(128, 1) prefill_tc_kernel(const __grid_constan
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tslot_gen);
-  const uint32_t tS = tmem, tO = tmem + 128;
-  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;  // this warp's lane quarter
+  const uint32_t tO = tmem + 256;
+  const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;  // this warp's lane quarter
+  const uint32_t col_off = static_cast<uint32_t>(half * 64);               // this thread's columns
 
   pdl_wait();
   bool ok = s < p.S;
@@ -191,7 +206,7 @@ __global__ void __launch_bounds__(128, 1) prefill_tc_kernel(const __grid_constan
   const int nsteps = (nblk + C::BPS - 1) / C::BPS;
 
   // this thread's row: its position, or the CTA's last for padding rows
-  const int row = r0 + tid;
+  const int row = r0 + rl;
   const bool row_ok = row < rows_all;
   const int pos = row_ok ? L - n + row / p.g : lim_max;
 
@@ -201,165 +216,217 @@ __global__ void __launch_bounds__(128, 1) prefill_tc_kernel(const __grid_constan
         static_cast<const uint16_t*>(p.q) + (q0 + (row_ok ? row / p.g : 0)) * p.q_t +
         (static_cast<long long>(h) * p.g + (row_ok ? row % p.g : 0)) * p.q_h);
 #pragma unroll
-    for (int c = 0; c < 16; ++c) {
+    for (int cc = 0; cc < 8; ++cc) {  // this thread's half of the row: chunks 8 half ..
+      const int c = half * 8 + cc;
       const uint4 v = row_ok ? __ldg(qp + c) : make_uint4(0u, 0u, 0u, 0u);
-      const uint32_t a = sQ + (c >> 3) * C::HALF + (tid >> 3) * 1024 + (tid & 7) * 128 +
-                         (((c & 7) ^ (tid & 7)) << 4);
+      const uint32_t a = sQ + (c >> 3) * C::HALF + (rl >> 3) * 1024 + (rl & 7) * 128 +
+                         (((c & 7) ^ (rl & 7)) << 4);
       asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z),
                    "r"(v.w)
                    : "memory");
     }
   }
 
-  // ---- K / V loads of step i into stage i & 1 (thread 0) ----
+  // ---- K or V tiles of step i into stage i & 1 (thread 0) ----
   const int* trow = p.tables + s * p.t_s;
   const uint64_t policy = l2_policy_evict_normal();
-  auto issue = [&](int i) {
-    const int st = i & 1;
-    const uint32_t bar = bar_kv + st * 8;
-    const uint32_t dk = sbase + C::OFF_K + st * C::TILE, dv = sbase + C::OFF_V + st * C::TILE;
-    mbar_arrive_expect_tx(bar, 2 * C::TILE);
-    for (int ib = 0; ib < C::BPS; ++ib) {
-      // blocks past the ones needed repeat the last needed one (finite data,
-      // masked by position)
+  // Physical blocks of step i, checked, into s_phys[i % 4] (threads 32 ..
+  // 32 + BPS - 1, three steps ahead of their use). Blocks past the ones
+  // needed repeat the last needed one (finite data, masked by position).
+  auto stage_phys = [&](int i) {
+    const int ib = tid - 32;
+    if (ib >= 0 && ib < C::BPS && i < nsteps) {
       const int b = min(i * C::BPS + ib, nblk - 1);
       int phys = __ldg(trow + b);
       if (phys < 0 || phys >= p.NB) {
         atomicOr(p.err, kErrBadBlock);
         phys = 0;
       }
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        tma_load_4d(dk + hh * C::HALF + ib * BS * 128, &p.tmk, bar, hh * 64, 0, h, phys, policy);
-        tma_load_4d(dv + hh * C::HALF + ib * BS * 128, &p.tmv, bar, hh * 64, 0, h, phys, policy);
-      }
+      s_phys[(i & 3) * C::BPS + ib] = phys;
     }
   };
-  int kv_issued = 0, s_issued = 0, o_issued = 0;  // thread 0's counts (drain on failure)
+  auto issue = [&](int i, bool v_tile) {
+    const int st = i & 1;
+    const uint32_t bar = (v_tile ? bar_v : bar_k) + st * 8;
+    const uint32_t dst = sbase + (v_tile ? C::OFF_V : C::OFF_K) + st * C::TILE;
+    const CUtensorMap* map = v_tile ? &p.tmv : &p.tmk;
+    mbar_arrive_expect_tx(bar, C::TILE);
+#pragma unroll
+    for (int ib = 0; ib < C::BPS; ++ib) {
+      const int phys = s_phys[(i & 3) * C::BPS + ib];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh)
+        tma_load_4d(dst + hh * C::HALF + ib * BS * 128, map, bar, hh * 64, 0, h, phys, policy);
+    }
+  };
+  constexpr uint32_t kIdS = idesc_f16<QBF>(false);  // B = K tile, K-major
+  constexpr uint32_t kIdO = idesc_f16<QBF>(true);   // B = V tile, MN-major
+  // S of step i = Q K_i^T into its tensor-memory buffer (thread 0)
+  auto issue_s = [&](int i) {
+    const uint32_t dk = sbase + C::OFF_K + (i & 1) * C::TILE;
+    const uint32_t tS = tmem + (i & 1) * 128;
+    tc_fence_after();
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const uint32_t off = (ks >> 2) * C::HALF + (ks & 3) * 32;
+      tc_mma(tS, smem_desc_sw128(sQ + off, 16, 1024), smem_desc_sw128(dk + off, 16, 1024), kIdS, ks > 0);
+    }
+    tc_commit(bar_s);
+  };
+
+  // Loads run two steps ahead, S one step ahead of the softmax, and O += P V
+  // of a step overlaps the next step's first pass. Thread 0's counts let a
+  // failed wait drain what is in flight.
+  int k_issued = 0, v_issued = 0, s_issued = 0, o_issued = 0;
+  bool failed = false;
+  stage_phys(0);
+  stage_phys(1);
+  stage_phys(2);
+  __syncthreads();
   if (tid == 0) {
-    issue(0);
-    kv_issued = 1;
+    issue(0, false);
+    issue(0, true);
+    k_issued = v_issued = 1;
     if (nsteps > 1) {
-      issue(1);
-      kv_issued = 2;
+      issue(1, false);
+      issue(1, true);
+      k_issued = v_issued = 2;
     }
   }
   fence_async_smem();  // Q written by the threads, read by the tensor cores
   tc_fence_before();
   __syncthreads();
+  if (tid == 0) {
+    if (lane_wait(bar_k, 0, kWaitNs)) {
+      issue_s(0);
+      s_issued = 1;
+    } else {
+      failed = true;
+    }
+  }
+  failed = __syncthreads_or(failed);
 
-  constexpr uint32_t kIdS = idesc_f16<QBF>(false);  // B = K tile, K-major
-  constexpr uint32_t kIdO = idesc_f16<QBF>(true);   // B = V tile, MN-major
   const float sl = p.scale_log2;
   float m_run = -INFINITY, l_run = 0.f;
-  bool failed = false;
 
-  // Every wait's outcome is made CTA-wide (__syncthreads_or) so that a wait
-  // that gives up sends every thread to the drain together.
-  int i_fail = nsteps;
+  // `failed` is only acted on after a CTA-wide OR, and every warp_wait (whose
+  // __all_sync needs all 32 lanes) runs unconditionally; after each block only
+  // thread 0 runs, __syncwarp reconverges warp 0 before the warp-collective
+  // tensor-memory loads.
   for (int i = 0; i < nsteps; ++i) {
     const int st = i & 1;
-    if (__syncthreads_or(!warp_wait(bar_kv + st * 8, static_cast<uint32_t>((i >> 1) & 1), kWaitNs))) {
-      failed = true;
-      i_fail = i;
-      break;
-    }
     const int key0 = i * C::KEYS;
-    // V rows at or past the sequence's length may hold anything (a partly
-    // filled last block): zero them, their P is 0 but 0 * NaN is not
-    if (key0 + C::KEYS > L) {
-      const uint32_t dv = sbase + C::OFF_V + st * C::TILE;
-      for (int k = max(L - key0, 0) * 16 + tid; k < C::KEYS * 16; k += 128) {
-        const int key = k >> 4, c = k & 15;  // 16-byte chunk c of key row `key`
-        const uint32_t a = dv + (c >> 3) * C::HALF + (key >> 3) * 1024 + (key & 7) * 128 + ((c & 7) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0u) : "memory");
+    const uint32_t tS = tmem + st * 128;
+    {
+      const bool w_ok = warp_wait(bar_s, static_cast<uint32_t>(i & 1), kWaitNs);
+      if (__syncthreads_or(failed || !w_ok)) {
+        failed = true;
+        break;
       }
-      fence_async_smem();
-      __syncthreads();
-    }
-    if (tid == 0) {  // S = Q K^T
-      tc_fence_after();
-      const uint32_t dk = sbase + C::OFF_K + st * C::TILE;
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        const uint32_t off = (ks >> 2) * C::HALF + (ks & 3) * 32;
-        tc_mma(tS, smem_desc_sw128(sQ + off, 16, 1024), smem_desc_sw128(dk + off, 16, 1024), kIdS,
-               ks > 0);
-      }
-      tc_commit(bar_s);
-      ++s_issued;
-    }
-    if (__syncthreads_or(!warp_wait(bar_s, static_cast<uint32_t>(i & 1), kWaitNs))) {
-      failed = true;
-      i_fail = i + 1;  // step i's K / V landed
-      break;
     }
     tc_fence_after();
-    // pass 1: this row's max over the step's keys it may see
-    float mx = -INFINITY;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      uint32_t v[32];
-      tmem_ld32(tS + lane_off + j * 32, v);
+    stage_phys(i + 3);  // read from step i + 1 on, after this step's barriers
+    // S of the next step while this one is reduced: its K tile has landed
+    // (loaded two steps ahead) and its buffer was read one step ago
+    if (tid == 0 && i + 1 < nsteps) {
+      if (lane_wait(bar_k + ((i + 1) & 1) * 8, static_cast<uint32_t>(((i + 1) >> 1) & 1), kWaitNs)) {
+        issue_s(i + 1);
+        ++s_issued;
+        // this step's K stage is free now (its S is complete): step i + 2's K
+        if (i + 2 < nsteps) {
+          issue(i + 2, false);
+          ++k_issued;
+        }
+      } else {
+        failed = true;
+      }
+    }
+    __syncwarp();
+    // this thread's 64 columns of S, once, into registers (masked, scaled)
+    float x[64];
+    {
+      uint32_t v0[32], v1[32];
+      tmem_ld32(tS + lane_off + col_off, v0);
+      tmem_ld32(tS + lane_off + col_off + 32, v1);
       tmem_wait_ld();
 #pragma unroll
       for (int u = 0; u < 32; ++u) {
-        const int key = key0 + j * 32 + u;
-        const float x = key <= pos ? __uint_as_float(v[u]) * sl : -INFINITY;
-        mx = fmaxf(mx, x);
+        const int k0 = key0 + half * 64 + u;
+        x[u] = k0 <= pos ? __uint_as_float(v0[u]) * sl : -INFINITY;
+        x[32 + u] = k0 + 32 <= pos ? __uint_as_float(v1[u]) * sl : -INFINITY;
       }
     }
+    float mx = -INFINITY;
+#pragma unroll
+    for (int u = 0; u < 64; ++u) mx = fmaxf(mx, x[u]);
+    xch[tid] = mx;  // the row's other thread takes the max of both halves
+    __syncthreads();
+    mx = fmaxf(mx, xch[tid ^ 128]);
     const float m_new = fmaxf(m_run, mx);
     const float base = m_new == -INFINITY ? 0.f : m_new;
     const float alpha = exp2f(m_run - base);
-    // the previous step's O += P V must be done: O is rescaled, P rewritten,
-    // and its K / V stage refilled
+    // the previous step's O += P V must be done before O is rescaled and P
+    // rewritten; its V stage then takes step i + 1's V
     if (i > 0) {
-      if (__syncthreads_or(!warp_wait(bar_o, static_cast<uint32_t>((i - 1) & 1), kWaitNs))) {
+      const bool w_ok = warp_wait(bar_o, static_cast<uint32_t>((i - 1) & 1), kWaitNs);
+      if (__syncthreads_or(failed || !w_ok)) {
         failed = true;
-        i_fail = i + 1;
         break;
       }
       tc_fence_after();
       if (tid == 0 && i + 1 < nsteps) {
-        issue(i + 1);
-        kv_issued = i + 2;
+        issue(i + 1, true);
+        ++v_issued;
       }
+      __syncwarp();
       // tcgen05.ld / st are warp-collective: rescale when any row of the warp
       // needs it (alpha is 1 for the others)
       if (__any_sync(0xffffffffu, alpha != 1.f)) {
+        uint32_t v0[32], v1[32];
+        tmem_ld32(tO + lane_off + col_off, v0);
+        tmem_ld32(tO + lane_off + col_off + 32, v1);
+        tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint32_t v[32];
-          tmem_ld32(tO + lane_off + j * 32, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int u = 0; u < 32; ++u) v[u] = __float_as_uint(__uint_as_float(v[u]) * alpha);
-          tmem_st32(tO + lane_off + j * 32, v);
+        for (int u = 0; u < 32; ++u) {
+          v0[u] = __float_as_uint(__uint_as_float(v0[u]) * alpha);
+          v1[u] = __float_as_uint(__uint_as_float(v1[u]) * alpha);
         }
+        tmem_st32(tO + lane_off + col_off, v0);
+        tmem_st32(tO + lane_off + col_off + 32, v1);
       }
     }
-    // pass 2: P = exp2(x - m) as 16-bit into shared memory, row sum
+    // V rows at or past the sequence's length may hold anything (a partly
+    // filled last block): zero them, their P is 0 but 0 * NaN is not
+    if (key0 + C::KEYS > L) {
+      const bool w_ok = warp_wait(bar_v + st * 8, static_cast<uint32_t>((i >> 1) & 1), kWaitNs);
+      if (__syncthreads_or(failed || !w_ok)) {
+        failed = true;
+        break;
+      }
+      const uint32_t dv = sbase + C::OFF_V + st * C::TILE;
+      for (int k = max(L - key0, 0) * 16 + tid; k < C::KEYS * 16; k += 256) {
+        const int key = k >> 4, c = k & 15;  // 16-byte chunk c of key row `key`
+        const uint32_t a = dv + (c >> 3) * C::HALF + (key >> 3) * 1024 + (key & 7) * 128 + ((c & 7) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0u) : "memory");
+      }
+    }
+    // P = exp2(x - m) as 16-bit into shared memory (this thread's 64 keys),
+    // this half's sum
     float lsum = 0.f;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      uint32_t v[32];
-      tmem_ld32(tS + lane_off + j * 32, v);
-      tmem_wait_ld();
+    for (int j = 0; j < 2; ++j) {
       uint32_t pk[16];
 #pragma unroll
       for (int u = 0; u < 32; u += 2) {
-        const int key = key0 + j * 32 + u;
-        const float p0 = key <= pos ? exp2f(__uint_as_float(v[u]) * sl - base) : 0.f;
-        const float p1 = key + 1 <= pos ? exp2f(__uint_as_float(v[u + 1]) * sl - base) : 0.f;
+        const float p0 = exp2f(x[32 * j + u] - base), p1 = exp2f(x[32 * j + u + 1] - base);
         lsum += p0 + p1;
         pk[u >> 1] = pack2<QBF>(p0, p1);
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {  // 16-byte chunk kc = 4 j + u of the row's keys
+      for (int u = 0; u < 4; ++u) {  // 16-byte chunk 4 j + u of this half of the keys
         const int kc = 4 * j + u;
-        const uint32_t a = sP + (kc >> 3) * C::HALF + (tid >> 3) * 1024 + (tid & 7) * 128 +
-                           (((kc & 7) ^ (tid & 7)) << 4);
+        const uint32_t a = sP + half * C::HALF + (rl >> 3) * 1024 + (rl & 7) * 128 +
+                           (((kc & 7) ^ (rl & 7)) << 4);
         asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(pk[4 * u]),
                      "r"(pk[4 * u + 1]), "r"(pk[4 * u + 2]), "r"(pk[4 * u + 3])
                      : "memory");
@@ -370,49 +437,63 @@ __global__ void __launch_bounds__(128, 1) prefill_tc_kernel(const __grid_constan
     tmem_wait_st();
     fence_async_smem();
     tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {  // O += P V
-      tc_fence_after();
-      const uint32_t dv = sbase + C::OFF_V + st * C::TILE;
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        const uint32_t a_off = (ks >> 2) * C::HALF + (ks & 3) * 32;  // keys 16 ks .. of P
-        tc_mma(tO, smem_desc_sw128(sP + a_off, 16, 1024),
-               smem_desc_sw128(dv + ks * 2048, C::HALF, 1024), kIdO, (i > 0 || ks > 0) ? 1u : 0u);
-      }
-      tc_commit(bar_o);
-      ++o_issued;
+    if (__syncthreads_or(failed)) {
+      failed = true;
+      break;
     }
+    if (tid == 0) {  // O += P V, once this step's V tile has landed
+      if (lane_wait(bar_v + st * 8, static_cast<uint32_t>((i >> 1) & 1), kWaitNs)) {
+        tc_fence_after();
+        const uint32_t dv = sbase + C::OFF_V + st * C::TILE;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t a_off = (ks >> 2) * C::HALF + (ks & 3) * 32;  // keys 16 ks .. of P
+          tc_mma(tO, smem_desc_sw128(sP + a_off, 16, 1024),
+                 smem_desc_sw128(dv + ks * 2048, C::HALF, 1024), kIdO, (i > 0 || ks > 0) ? 1u : 0u);
+        }
+        tc_commit(bar_o);
+        ++o_issued;
+      } else {
+        failed = true;
+      }
+    }
+    __syncwarp();
   }
 
-  if (!failed &&
-      __syncthreads_or(!warp_wait(bar_o, static_cast<uint32_t>((nsteps - 1) & 1), kWaitNs))) {
-    failed = true;
-    i_fail = nsteps;
+  failed = __syncthreads_or(failed);
+  if (!failed) {
+    const bool w_ok = warp_wait(bar_o, static_cast<uint32_t>((nsteps - 1) & 1), kWaitNs);
+    failed = __syncthreads_or(!w_ok);
   }
   if (failed) {
     if (tid == 0) {
       atomicOr(p.err, kErrWaitTimeout);
       // let what is still in flight finish (bounded) before the CTA's shared
-      // and tensor memory go: loads of steps not yet consumed, the last
-      // issued products
+      // and tensor memory go: every issued load and the last products
       constexpr uint64_t kDrainNs = 100000000ull;
-      for (int k = i_fail; k < kv_issued; ++k)
-        lane_wait(bar_kv + (k & 1) * 8, static_cast<uint32_t>((k >> 1) & 1), kDrainNs);
+      // loads into one stage complete in order: wait for each stage's last
+      for (int k = max(k_issued - 2, 0); k < k_issued; ++k)
+        lane_wait(bar_k + (k & 1) * 8, static_cast<uint32_t>((k >> 1) & 1), kDrainNs);
+      for (int k = max(v_issued - 2, 0); k < v_issued; ++k)
+        lane_wait(bar_v + (k & 1) * 8, static_cast<uint32_t>((k >> 1) & 1), kDrainNs);
       if (s_issued > 0) lane_wait(bar_s, static_cast<uint32_t>((s_issued - 1) & 1), kDrainNs);
       if (o_issued > 0) lane_wait(bar_o, static_cast<uint32_t>((o_issued - 1) & 1), kDrainNs);
     }
   } else {
     tc_fence_after();
-    // epilogue: O row / l, 16-bit, to the output row
-    const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+    // epilogue: O row / l (both halves' sums), 16-bit, to the output row
+    xch[tid] = l_run;
+    __syncthreads();
+    const float lt = l_run + xch[tid ^ 128];
+    const float inv = lt > 0.f ? 1.f / lt : 0.f;
     uint4* orow = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) +
                                            (q0 + (row_ok ? row / p.g : 0)) * p.o_t +
-                                           (static_cast<long long>(h) * p.g + (row_ok ? row % p.g : 0)) * p.o_h);
+                                           (static_cast<long long>(h) * p.g + (row_ok ? row % p.g : 0)) * p.o_h +
+                                           half * 64);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+    for (int j = 0; j < 2; ++j) {
       uint32_t v[32];
-      tmem_ld32(tO + lane_off + j * 32, v);
+      tmem_ld32(tO + lane_off + col_off + j * 32, v);
       tmem_wait_ld();
       if (row_ok) {
 #pragma unroll
