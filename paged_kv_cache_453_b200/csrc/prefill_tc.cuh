@@ -362,9 +362,14 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
     xch[tid] = mx;  // the row's other thread takes the max of both halves
     __syncthreads();
     mx = fmaxf(mx, xch[tid ^ 128]);
+    // The exponent base moves only when the row's max grows by more than 8
+    // (P then stays below 2^8, exact enough in 16 bits and far from fp32
+    // overflow in O and l); otherwise O needs no rescale this step.
     const float m_new = fmaxf(m_run, mx);
-    const float base = m_new == -INFINITY ? 0.f : m_new;
-    const float alpha = exp2f(m_run - base);
+    const bool grow = m_new > m_run + 8.f || m_run == -INFINITY;
+    const float m_use = grow ? m_new : m_run;
+    const float base = m_use == -INFINITY ? 0.f : m_use;
+    const float alpha = grow ? exp2f(m_run - base) : 1.f;
     // the previous step's O += P V must be done before O is rescaled and P
     // rewritten; its V stage then takes step i + 1's V
     if (i > 0) {
@@ -433,7 +438,7 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
       }
     }
     l_run = l_run * alpha + lsum;
-    m_run = m_new;
+    m_run = m_use;
     tmem_wait_st();
     fence_async_smem();
     tc_fence_before();
