@@ -695,10 +695,11 @@ int launch_prefill(const pkv_tensor* q, const pkv_tensor* kc, const pkv_tensor* 
   DeviceState* ds;
   if ((st = device_state(dev, &ds)) != PKV_OK) return st;
   // 128-row tiles on the tensor cores when every (sequence, head) may have
-  // that many rows and q / out rows are 16-byte aligned (vector loads)
+  // that many rows, q / out rows are 16-byte aligned (vector loads) and the
+  // scale is positive (that kernel takes row maxima of the unscaled scores)
   const bool rows16 = q->stride[0] % 8 == 0 && q->stride[1] % 8 == 0 && aligned(q->data, 16) &&
                       out->stride[0] % 8 == 0 && out->stride[1] % 8 == 0 && aligned(out->data, 16);
-  const bool use_tc = D == 128 && cols >= 128 && rows16;
+  const bool use_tc = D == 128 && cols >= 128 && rows16 && scale > 0.f;
   {
     std::lock_guard<std::mutex> lk(g_mu);
     if (!e->attr_set[dev]) {
@@ -748,7 +749,7 @@ int launch_prefill(const pkv_tensor* q, const pkv_tensor* kc, const pkv_tensor* 
     at[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t tc = {};
     tc.gridDim = dim3(static_cast<unsigned>((cols + 127) / 128), 1, static_cast<unsigned>(S * Hk));
-    tc.blockDim = dim3(256);
+    tc.blockDim = dim3(PrefillTcCfg<16>::THREADS);  // the same for every block size
     tc.dynamicSmemBytes = static_cast<size_t>(te->smem);
     tc.stream = stream;
     tc.attrs = at;
