@@ -6,13 +6,13 @@
 // rule); this kernel is used when a (sequence, kv head) has at least 128
 // query rows (new tokens x query heads of the group).
 //
-// CTA = 8 softmax warps + 3 producer warps, one (sequence, kv head, 128 query
+// CTA = 8 softmax warps + 4 producer warps, one (sequence, kv head, 128 query
 // rows); a row is one query head of one new token (token-major). Threads r
 // and r + 128 share row r (tensor-memory lane r; warps w and w + 4 read the
 // same lane quarter), each owning 64 of the 128 columns of S and of O. One
-// producer warp issues the MMAs, one the K loads, one the V loads (issuing a
+// producer warp issues the MMAs, two the K loads, one the V loads (issuing a
 // paged load or an MMA costs far more than its few instructions suggest, so
-// the three proceed side by side); they and the softmax warps meet only at
+// they proceed side by side); they and the softmax warps meet only at
 // mbarriers (S ready, P ready, O done, stage landed), never at a CTA-wide
 // barrier inside the loop. Per step of 128 keys (128 / B blocks through the
 // block table):
@@ -159,7 +159,10 @@ struct PrefillTcCfg {
   static constexpr int TILE = 2 * HALF;   // Q, K, V or P tile: 32 KB
   static constexpr int BPS = KEYS / BS;   // blocks per step
   static constexpr int SOFT = 256;        // softmax threads (8 warps)
-  static constexpr int THREADS = SOFT + 96;  // warp 8 issues the MMAs, 9 loads K, 10 loads V
+  static constexpr int LWK = 2, LWV = 1;  // warps loading the K / V tile of a step
+  static_assert(BPS % LWK == 0 && BPS % LWV == 0, "a loading warp takes whole blocks");
+  // warp 8 issues the MMAs, the next LWK warps load K, the LWV after them V
+  static constexpr int THREADS = SOFT + 32 * (1 + LWK + LWV);
   // layout from the (1024-aligned) base:
   //   Q | K0 K1 | V0 V1 | P0 P1 | barriers | exchange | flags
   static constexpr int OFF_Q = 0, OFF_K = TILE, OFF_V = 3 * TILE, OFF_P = 5 * TILE;
@@ -217,8 +220,8 @@ __global__ void __launch_bounds__(PrefillTcCfg<BS>::THREADS, 1) prefill_tc_kerne
   pdl_launch_dependents();
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
-      mbar_init(bar_k + i * 8, 1);
-      mbar_init(bar_v + i * 8, 1);
+      mbar_init(bar_k + i * 8, C::LWK);
+      mbar_init(bar_v + i * 8, C::LWV);
     }
     mbar_init(bar_s, 1);
     mbar_init(bar_s + 8, 1);
@@ -294,26 +297,34 @@ __global__ void __launch_bounds__(PrefillTcCfg<BS>::THREADS, 1) prefill_tc_kerne
       // ---- MMA issue: S of step i + 1 before O += P V of step i ----
       constexpr uint32_t kIdS = idesc_f16<QBF>(false);  // B = K tile, K-major
       constexpr uint32_t kIdO = idesc_f16<QBF>(true);   // B = V tile, MN-major
+      // descriptors of each operand's stage 0; a stage or a K step moves the
+      // start address field (16-byte units, no carry: shared addresses are
+      // below 256 KB)
+      const uint64_t d_q = smem_desc_sw128(sQ, 16, 1024);
+      const uint64_t d_k = smem_desc_sw128(sbase + C::OFF_K, 16, 1024);
+      const uint64_t d_p = smem_desc_sw128(sP, 16, 1024);
+      const uint64_t d_v = smem_desc_sw128(sbase + C::OFF_V, C::HALF, 1024);
       auto issue_s = [&](int i) {  // lane 0: S of step i into its buffer
-        const uint32_t dk = sbase + C::OFF_K + (i & 1) * C::TILE;
+        const uint64_t dk = d_k + static_cast<uint64_t>((i & 1) * (C::TILE >> 4));
         const uint32_t tS = tmem + (i & 1) * 128;
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t off = (ks >> 2) * C::HALF + (ks & 3) * 32;
-          tc_mma(tS, smem_desc_sw128(sQ + off, 16, 1024), smem_desc_sw128(dk + off, 16, 1024), kIdS, ks > 0);
+          constexpr int kHalf16 = C::HALF >> 4;
+          const uint64_t off = static_cast<uint64_t>((ks >> 2) * kHalf16 + (ks & 3) * 2);
+          tc_mma(tS, d_q + off, dk + off, kIdS, ks > 0);
         }
         tc_commit(bar_s + (i & 1) * 8);
       };
       auto issue_pv = [&](int i) {  // lane 0: O += P V of step i
-        const uint32_t dv = sbase + C::OFF_V + (i & 1) * C::TILE;
-        const uint32_t dp = sP + (i & 1) * C::TILE;
+        const uint64_t dv = d_v + static_cast<uint64_t>((i & 1) * (C::TILE >> 4));
+        const uint64_t dp = d_p + static_cast<uint64_t>((i & 1) * (C::TILE >> 4));
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t a_off = (ks >> 2) * C::HALF + (ks & 3) * 32;  // keys 16 ks .. of P
-          tc_mma(tO, smem_desc_sw128(dp + a_off, 16, 1024), smem_desc_sw128(dv + ks * 2048, C::HALF, 1024),
-                 kIdO, (i > 0 || ks > 0) ? 1u : 0u);
+          constexpr int kHalf16 = C::HALF >> 4;
+          const uint64_t a_off = static_cast<uint64_t>((ks >> 2) * kHalf16 + (ks & 3) * 2);  // keys 16 ks ..
+          tc_mma(tO, dp + a_off, dv + static_cast<uint64_t>(ks * (2048 >> 4)), kIdO, (i > 0 || ks > 0) ? 1u : 0u);
         }
         tc_commit(bar_o + (i & 1) * 8);
       };
@@ -348,12 +359,17 @@ __global__ void __launch_bounds__(PrefillTcCfg<BS>::THREADS, 1) prefill_tc_kerne
           lane_wait(bar_o + (k & 1) * 8, static_cast<uint32_t>((k >> 1) & 1), kDrainNs);
       }
     } else {
-      // ---- K (warp 9) or V (warp 10) tiles of each step, two stages ----
+      // ---- K or V tiles of each step, two stages; LWK (LWV) warps per tile,
+      // each loading an equal share of the step's blocks ----
       // A stage is free again once the product that read it (S, or O += P V,
       // of two steps before) is complete. Lanes 0 .. BPS - 1 hold the step's
       // physical blocks (read a step ahead); blocks past the ones needed
       // repeat the last needed one (finite data, masked).
-      const bool vt = warp == C::SOFT / 32 + 2;
+      const int lw = warp - C::SOFT / 32 - 1;  // 0 .. LWK + LWV - 1
+      const bool vt = lw >= C::LWK;
+      const int nlw = vt ? C::LWV : C::LWK;
+      const int nb = C::BPS / nlw;  // blocks this warp loads
+      const int ib0 = (vt ? lw - C::LWK : lw) * nb;
       const int* trow = p.tables + s * p.t_s;
       const uint64_t policy = l2_policy_evict_normal();
       const uint32_t full = vt ? bar_v : bar_k;
@@ -373,15 +389,18 @@ __global__ void __launch_bounds__(PrefillTcCfg<BS>::THREADS, 1) prefill_tc_kerne
         }
         if (j >= 2 && !wait1(done + (j & 1) * 8, static_cast<uint32_t>(((j - 2) >> 1) & 1))) break;
         const uint32_t bar = full + (j & 1) * 8, dst = dst0 + (j & 1) * C::TILE;
-        if (lane == 0) mbar_arrive_expect_tx(bar, C::TILE);
+        int pb[C::BPS];
 #pragma unroll
-        for (int ib = 0; ib < C::BPS; ++ib) {
-          const int pb = __shfl_sync(0xffffffffu, phys, ib);
-          if (lane == 0) {
+        for (int u = 0; u < C::BPS; ++u) pb[u] = __shfl_sync(0xffffffffu, phys, min(ib0 + u, C::BPS - 1));
+        if (lane == 0) {
+          mbar_arrive_expect_tx(bar, C::TILE / nlw);
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh)
-              tma_load_4d(dst + hh * C::HALF + ib * BS * 128, map, bar, hh * 64, 0, h, pb, policy);
-          }
+          for (int u = 0; u < C::BPS; ++u)
+            if (u < nb) {
+#pragma unroll
+              for (int hh = 0; hh < 2; ++hh)
+                tma_load_4d(dst + hh * C::HALF + (ib0 + u) * BS * 128, map, bar, hh * 64, 0, h, pb[u], policy);
+            }
         }
         ++issued;
         phys = phys_next;
