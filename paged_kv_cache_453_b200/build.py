@@ -19,7 +19,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libpagedkv.so")
 SOURCES = [os.path.join(CSRC, "pagedkv.cu"), os.path.join(CSRC, "allocator.cpp")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("decode.cuh", "cascade.cuh", "prefill.cuh", "prefill_tc.cuh", "cache_ops.cuh", "ptx.cuh")] + [
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("decode.cuh", "cascade.cuh", "prefill.cuh", "prefill_tc.cuh", "prefill_tc2.cuh", "cache_ops.cuh", "ptx.cuh")] + [
     os.path.join(ROOT, "include", "pagedkv.h"), os.path.abspath(__file__)]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

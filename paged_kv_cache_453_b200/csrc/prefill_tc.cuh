@@ -3,8 +3,8 @@
 // prompt chunk of many new tokens is a dense contraction, so both products
 // run as 128 x 128 x 16 tcgen05.mma instructions issued by one thread.
 // The result is the one prefill_kernel computes (same positions, same causal
-// rule); this kernel is used when a (sequence, kv head) has at least 128
-// query rows (new tokens x query heads of the group).
+// rule); this kernel is used when a (sequence, kv head) may have at least
+// 64 query rows (new tokens x query heads of the group).
 //
 // CTA = 8 softmax warps + 4 producer warps, one (sequence, kv head, 128 query
 // rows); a row is one query head of one new token (token-major). Threads r

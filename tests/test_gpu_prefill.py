@@ -69,6 +69,10 @@ CASES = {
     "tc_chunk_gqa_f16": (W.spec("llama3_8b").replace(num_seqs=3, cache_dtype="f16", q_dtype="f16",
                                                      lens=("fixed", [333, 129, 700]), table_width=None),
                          [333, 64, 250]),
+    # 64 rows at most: one half-filled tensor-core tile per (sequence, head)
+    "tc_half_tile": (W.spec("llama3_8b").replace(num_seqs=4, lens=("fixed", [200, 16, 77, 1000]),
+                                                 table_width=None),
+                     [16, 9, 1, 16]),
 }
 
 
