@@ -332,22 +332,19 @@ __global__ void __launch_bounds__(PrefillTc2Cfg<BS>::THREADS, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, v[c]);
         tmem_wait_ld();
-        float x[128];
-        const bool masked = __any_sync(0xffffffffu, key0 + 127 > pos);
-        if (masked) {
+        if (__any_sync(0xffffffffu, key0 + 127 > pos)) {  // masked in place (bits of -inf)
 #pragma unroll
-          for (int u = 0; u < 128; ++u) x[u] = key0 + u <= pos ? __uint_as_float(v[u >> 5][u & 31]) : -INFINITY;
-        } else {
-#pragma unroll
-          for (int u = 0; u < 128; ++u) x[u] = __uint_as_float(v[u >> 5][u & 31]);
+          for (int u = 0; u < 128; ++u)
+            if (key0 + u > pos) v[u >> 5][u & 31] = 0xff800000u;
         }
+        auto x = [&](int u) { return __uint_as_float(v[u >> 5][u & 31]); };
         float mm[4];  // independent chains of 32
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          mm[c] = x[32 * c];
+          mm[c] = x(32 * c);
 #pragma unroll
-          for (int u = 1; u < 31; u += 2) mm[c] = fmax3(mm[c], x[32 * c + u], x[32 * c + u + 1]);
-          mm[c] = fmaxf(mm[c], x[32 * c + 31]);
+          for (int u = 1; u < 31; u += 2) mm[c] = fmax3(mm[c], x(32 * c + u), x(32 * c + u + 1));
+          mm[c] = fmaxf(mm[c], x(32 * c + 31));
         }
         const float mx = fmaxf(fmax3(mm[0], mm[1], mm[2]), mm[3]) * sl;
         // The exponent base moves only when the row's max grows by more than
@@ -358,17 +355,6 @@ __global__ void __launch_bounds__(PrefillTc2Cfg<BS>::THREADS, 1)
         const float m_use = grow ? m_new : m_run;
         const float base = m_use == -INFINITY ? 0.f : m_use;
         const float alpha = grow ? exp2f(m_run - base) : 1.f;
-        if (i > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {  // warp-collective loads / stores
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            uint32_t o[16];
-            tmem_ld16(tO + 16 * c, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int u = 0; u < 16; ++u) o[u] = __float_as_uint(__uint_as_float(o[u]) * alpha);
-            tmem_st16(tO + 16 * c, o);
-          }
-        }
         // V rows at or past the sequence's length may hold anything (a
         // partly filled last block): tile A zeroes them (their P is 0 but
         // 0 * NaN is not); both products of the step are issued after P_A
@@ -394,12 +380,25 @@ __global__ void __launch_bounds__(PrefillTc2Cfg<BS>::THREADS, 1)
 #pragma unroll
           for (int u = 0; u < 32; u += 2) {
             float t0, t1;
-            f2_unpack(f2_fma(f2_pack(x[32 * c + u], x[32 * c + u + 1]), sl2, nb2), t0, t1);
+            f2_unpack(f2_fma(f2_pack(x(32 * c + u), x(32 * c + u + 1)), sl2, nb2), t0, t1);
             const float p0 = ex2_fast(t0), p1 = ex2_fast(t1);
             acc[(u >> 1) & 3] = f2_add(acc[(u >> 1) & 3], f2_pack(p0, p1));
             pk[u >> 1] = pack2<QBF>(p0, p1);
           }
           tmem_st16(tS + 16 * c, pk);
+        }
+        // O rescaled after P, when the scores' registers are free again (the
+        // product that adds P V is issued only after this thread's arrival)
+        if (i > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {  // warp-collective loads / stores
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            uint32_t o[16];
+            tmem_ld16(tO + 16 * c, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int u = 0; u < 16; ++u) o[u] = __float_as_uint(__uint_as_float(o[u]) * alpha);
+            tmem_st16(tO + 16 * c, o);
+          }
         }
         float lsum0, lsum1;
         f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), lsum0, lsum1);
