@@ -455,12 +455,14 @@ def run_prefill(a, s: W.Spec):
     if st != P.PKV_OK:
         raise SystemExit(f"device check failed: {P.status_string(st)}")
     sec = e0.elapsed_time(e1) / K / 1e3
-    # 128-row tiles of (new tokens x group heads) run on the tensor cores:
+    # tiles of 128 rows (new tokens x group heads) run on the tensor cores
+    # from 64 rows (one tile per CTA up to 128 rows, two beyond):
     # that launch is bound by the MMAs, the others by the KV bytes
     g = s.num_q_heads // s.num_kv_heads
-    if s.head_dim == 128 and max(nq) * g >= 128:
+    if s.head_dim == 128 and max(nq) * g >= 64 and s.scale > 0:
         peak, src = measured_peak_bf16()
-        roof = {"kernel": "prefill_tc_kernel", "bound": "tensor", "achieved": flops / sec / 1e12, "peak": peak,
+        kern = "prefill_tc2_kernel" if max(nq) * g > 128 else "prefill_tc_kernel"
+        roof = {"kernel": kern, "bound": "tensor", "achieved": flops / sec / 1e12, "peak": peak,
                 "unit": "TFLOP/s", "frac": flops / sec / 1e12 / peak, "peak_source": src + " (bf16 burst)",
                 "traffic": None, "alg_bytes_per_launch": alg, "flops_per_launch": flops}
     else:
