@@ -459,9 +459,21 @@ def run_prefill(a, s: W.Spec):
     # from 64 rows (one tile per CTA up to 128 rows, two beyond):
     # that launch is bound by the MMAs, the others by the KV bytes
     g = s.num_q_heads // s.num_kv_heads
-    if s.head_dim == 128 and max(nq) * g >= 64 and s.scale > 0:
+    cols = max(nq) * g
+    tc = s.head_dim == 128 and cols >= 64 and s.scale > 0
+    # kernels one call launches: the tensor-core kernel (after the one-CTA
+    # longest-first ordering pass when 1 < S <= 1024), or the warp-MMA
+    # kernel (plus its merge when the KV is cut into chunks)
+    if tc:
+        per_call = 1 + (1 if 1 < s.num_seqs <= 1024 else 0)
+    else:
+        ecols = 16 if cols <= 16 else 32 if cols <= 32 else 64
+        ncc = -(-cols // ecols)
+        sms = torch.cuda.get_device_properties(0).multi_processor_count
+        per_call = 1 + (1 if s.num_seqs * s.num_kv_heads * ncc < 4 * sms and lay.tables.shape[1] > 32 else 0)
+    if tc:
         peak, src = measured_peak_bf16()
-        kern = "prefill_tc2_kernel" if max(nq) * g > 128 else "prefill_tc_kernel"
+        kern = "prefill_tc2_kernel" if cols > 128 else "prefill_tc_kernel"
         roof = {"kernel": kern, "bound": "tensor", "achieved": flops / sec / 1e12, "peak": peak,
                 "unit": "TFLOP/s", "frac": flops / sec / 1e12 / peak, "peak_source": src + " (bf16 burst)",
                 "traffic": None, "alg_bytes_per_launch": alg, "flops_per_launch": flops}
@@ -479,7 +491,7 @@ def run_prefill(a, s: W.Spec):
                    "kv_bytes": kv, "l2": "inputs larger than L2 (K/V pool > 126 MB), no flush"},
         "tflops": flops / sec / 1e12,
         "roofline": roof,
-        "clocks": clk, "gpu_launches": K,
+        "clocks": clk, "gpu_launches": per_call * K,
     }))
 
 

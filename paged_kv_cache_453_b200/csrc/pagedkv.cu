@@ -41,6 +41,7 @@ struct DeviceState {
   size_t cas_bytes = 0;
   void* pre = nullptr;  // library-owned multi-token partials
   size_t pre_bytes = 0;
+  int* ord = nullptr;   // library-owned sequence order for the tensor-core multi-token kernels
 };
 DeviceState g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -762,6 +763,19 @@ int launch_prefill(const pkv_tensor* q, const pkv_tensor* kc, const pkv_tensor* 
     }
     p.err = ds->err;
     p.nkv = 1;
+    // longest contexts first, so the last wave of CTAs is short ones
+    if (S > 1 && S <= kOrderMaxSeqs) {
+      {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!ds->ord && cudaMalloc(reinterpret_cast<void**>(&ds->ord), kOrderMaxSeqs * sizeof(int)) != cudaSuccess) {
+          ds->ord = nullptr;
+          return PKV_ERR_CUDA;
+        }
+      }
+      order_by_len_kernel<<<1, kOrderMaxSeqs, 0, stream>>>(p.lens, static_cast<int>(S), ds->ord);
+      if (cudaGetLastError() != cudaSuccess) return PKV_ERR_CUDA;
+      p.order = ds->ord;
+    }
     cudaLaunchAttribute at[1];
     at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     at[0].val.programmaticStreamSerializationAllowed = 1;

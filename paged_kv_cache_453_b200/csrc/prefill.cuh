@@ -48,7 +48,31 @@ struct PrefillParams {
   int kv_chunk;     // blocks per KV chunk (split only)
   float* part_o;    // [T * Hq * nkv][D] (split only)
   float* part_ml;   // [T * Hq * nkv][2]
+  const int* order;  // [S] sequences by decreasing context length, or null (tensor-core kernels)
 };
+
+// order[r] = the sequence with the r-th longest context (ties: lower index
+// first); one CTA of 1024 threads, S <= 1024 (each thread counts its
+// sequence's rank over the lengths staged in shared memory). Its dependents
+// may start their prologue at once; they read order only after their
+// grid-dependency wait.
+constexpr int kOrderMaxSeqs = 1024;
+__global__ void __launch_bounds__(kOrderMaxSeqs) order_by_len_kernel(const int* lens, int S, int* order) {
+  __shared__ int sl[kOrderMaxSeqs];
+  pdl_launch_dependents();
+  const int i = threadIdx.x;
+  const int li = i < S ? lens[i] : 0;
+  sl[i] = li;
+  __syncthreads();
+  if (i < S) {
+    int rank = 0;
+    for (int j = 0; j < S; ++j) {
+      const int lj = sl[j];
+      rank += (lj > li || (lj == li && j < i)) ? 1 : 0;
+    }
+    order[rank] = i;
+  }
+}
 
 template <bool QBF, int D, int BS, int NS, int NW>
 struct PrefillCfg {

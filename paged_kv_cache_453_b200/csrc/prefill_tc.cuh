@@ -215,7 +215,7 @@ __global__ void __launch_bounds__(PrefillTcCfg<BS>::THREADS, 1) prefill_tc_kerne
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int rl = tid & 127, half = (tid >> 7) & 1;  // softmax: row in the tile, column half
-  const int s = static_cast<int>(blockIdx.z / p.Hk), h = static_cast<int>(blockIdx.z % p.Hk);
+  const int zs = static_cast<int>(blockIdx.z / p.Hk), h = static_cast<int>(blockIdx.z % p.Hk);
 
   pdl_launch_dependents();
   if (tid == 0) {
@@ -250,7 +250,10 @@ __global__ void __launch_bounds__(PrefillTcCfg<BS>::THREADS, 1) prefill_tc_kerne
   const uint32_t col_off = static_cast<uint32_t>(half * 64);               // this thread's columns
 
   pdl_wait();
-  bool ok = s < p.S;
+  // the sequence: in launch order, or longest context first when an order
+  // was computed (it shortens the tail of the last wave)
+  const int s = p.order ? p.order[zs] : zs;
+  bool ok = s >= 0 && s < p.S;
   if (tmem_got != tmem) {
     if (tid == 0) atomicOr(p.err, kErrTcSetup);
     ok = false;

@@ -104,7 +104,7 @@ __global__ void __launch_bounds__(PrefillTc2Cfg<BS>::THREADS, 1)
   uint32_t* tslot_gen = reinterpret_cast<uint32_t*>(smem_raw + C::OFF_BAR + 128);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int s = static_cast<int>(blockIdx.z / p.Hk), h = static_cast<int>(blockIdx.z % p.Hk);
+  const int zs = static_cast<int>(blockIdx.z / p.Hk), h = static_cast<int>(blockIdx.z % p.Hk);
 
   pdl_launch_dependents();
   if (tid == 0) {
@@ -136,7 +136,10 @@ __global__ void __launch_bounds__(PrefillTc2Cfg<BS>::THREADS, 1)
   constexpr uint32_t tmem = 0;
 
   pdl_wait();
-  bool ok = s < p.S;
+  // the sequence: in launch order, or longest context first when an order
+  // was computed (it shortens the tail of the last wave)
+  const int s = p.order ? p.order[zs] : zs;
+  bool ok = s >= 0 && s < p.S;
   if (tmem_got != tmem) {
     if (tid == 0) atomicOr(p.err, kErrTcSetup);
     ok = false;
