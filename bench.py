@@ -464,14 +464,17 @@ def run_prefill(a, s: W.Spec):
     # kernels one call launches: the tensor-core kernel (after the one-CTA
     # longest-first ordering pass when 1 < S <= 1024), or the warp-MMA
     # kernel (plus its merge when the KV is cut into chunks)
-    if tc:
+    decode_step = max(nq) == 1 and T == s.num_seqs  # served by the decode kernels
+    if decode_step:
+        per_call = 2
+    elif tc:
         per_call = 1 + (1 if 1 < s.num_seqs <= 1024 else 0)
     else:
         ecols = 16 if cols <= 16 else 32 if cols <= 32 else 64
         ncc = -(-cols // ecols)
         sms = torch.cuda.get_device_properties(0).multi_processor_count
         per_call = 1 + (1 if s.num_seqs * s.num_kv_heads * ncc < 4 * sms and lay.tables.shape[1] > 32 else 0)
-    if tc:
+    if tc and not decode_step:
         peak, src = measured_peak_bf16()
         kern = "prefill_tc2_kernel" if cols > 128 else "prefill_tc_kernel"
         roof = {"kernel": kern, "bound": "tensor", "achieved": flops / sec / 1e12, "peak": peak,
@@ -479,7 +482,8 @@ def run_prefill(a, s: W.Spec):
                 "traffic": None, "alg_bytes_per_launch": alg, "flops_per_launch": flops}
     else:
         peak, src = measured_peak_hbm()
-        roof = {"kernel": "prefill_kernel", "bound": "hbm", "achieved": alg / sec / 1e9, "peak": peak,
+        roof = {"kernel": "decode_kernel + decode_merge_kernel" if decode_step else "prefill_kernel",
+                "bound": "hbm", "achieved": alg / sec / 1e9, "peak": peak,
                 "unit": "GB/s", "frac": alg / sec / 1e9 / peak, "peak_source": src, "traffic": None,
                 "alg_bytes_per_launch": alg, "flops_per_launch": flops}
     print(json.dumps({

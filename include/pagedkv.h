@@ -182,11 +182,17 @@ int paged_attn_decode_ex(const pkv_tensor* q, const pkv_tensor* k_cache,
  *   max_q_tokens  host int >= every n_s (sizes the launch)
  *   out           device [T, Hq, D] like q; rows of tokens in no sequence
  *                 are left untouched
- * One CTA per (sequence, kv head, 16 / 32 / 64 query columns), a column being
- * one query head of one new token: the chunk's columns share every K/V tile
- * read, so the cache is read once per chunk. Asynchronous on `stream`; an
- * inconsistent q_start / context_lens row or block id is flagged
- * (PKV_ERR_DEVICE_CHECK) and that row skipped.
+ * Kernels, by query rows per (sequence, kv head) (new tokens x group heads):
+ * up to 64, one CTA per (sequence, kv head, 16 / 32 / 64 query columns) with
+ * warp MMAs, a column being one query head of one new token (the chunk's
+ * columns share every K/V tile read); from 64 (D = 128, scale > 0), 128-row
+ * tiles on the tensor cores, one or two per CTA, sequences taken longest
+ * context first (a one-CTA ordering pass runs before them, S <= 1024).
+ * With max_q_tokens = 1 and T = S (one new token per sequence) the call is
+ * the decode step and runs the decode kernels; q_start, which can then only
+ * be 0, 1, ..., S, is not read. Asynchronous on `stream`; an inconsistent
+ * q_start / context_lens row or block id is flagged (PKV_ERR_DEVICE_CHECK)
+ * and that row skipped.
  */
 int paged_attn_prefill(const pkv_tensor* q, const pkv_tensor* k_cache, const pkv_tensor* v_cache,
                        const pkv_tensor* block_tables, const pkv_tensor* context_lens,

@@ -1175,6 +1175,17 @@ int paged_attn_prefill(const pkv_tensor* q, const pkv_tensor* k_cache, const pkv
                        const pkv_tensor* block_tables, const pkv_tensor* context_lens,
                        const pkv_tensor* q_start, int max_q_tokens, int num_kv_heads, float scale,
                        int block_size, pkv_tensor* out, void* stream) {
+  // One new token per sequence (max_q_tokens 1 and as many query rows as
+  // sequences) is the decode step: the decode kernel serves it (q_start can
+  // then only be 0, 1, ..., S and is not read). Shapes the decode does not
+  // take go to the multi-token kernels.
+  if (q && block_tables && max_q_tokens == 1 && q->ndim == 3 && block_tables->ndim == 2 &&
+      q->shape[0] == block_tables->shape[0]) {
+    DecodeArgs a{q, k_cache, v_cache, nullptr, nullptr, block_tables, context_lens,
+                 num_kv_heads, scale, block_size, out};
+    const int st = launch_decode(a, false, nullptr, 0, true, static_cast<cudaStream_t>(stream));
+    if (st != PKV_ERR_UNSUPPORTED) return st;
+  }
   return launch_prefill(q, k_cache, v_cache, block_tables, context_lens, q_start, max_q_tokens,
                         num_kv_heads, scale, block_size, out, static_cast<cudaStream_t>(stream));
 }

@@ -87,6 +87,7 @@ def test_prefill_matches_oracle(name):
 
 
 def test_one_token_per_sequence_is_the_decode_step():
+    # T = S and max_q_tokens = 1: served by the decode kernels
     spec = W.scaled_down(W.spec("llama3_8b"), 8, 700)
     s, lay, t, q, q_start, max_q = _case(spec, [1] * 8)
     out = _run(s, lay, t, q, q_start, max_q)
@@ -94,8 +95,18 @@ def test_one_token_per_sequence_is_the_decode_step():
     P.paged_attn_decode(q, t.k_cache, t.v_cache, lay.tables.cuda(), lay.lens.cuda(), s.num_kv_heads, s.scale,
                         s.block_size, dec)
     torch.cuda.synchronize()
-    assert (out.float() - dec.float()).abs().max().item() <= TOL[s.cache_dtype]
     check_no_device_error()
+    assert torch.equal(out, dec)
+    assert max_err(out, _oracle(s, lay, t, q, q_start)) <= TOL[s.cache_dtype]
+
+
+def test_one_token_for_some_sequences_uses_the_multi_token_path():
+    # max_q_tokens = 1 but fewer rows than sequences: the multi-token kernel
+    spec = W.scaled_down(W.spec("llama3_8b"), 6, 500)
+    s, lay, t, q, q_start, max_q = _case(spec, [1, 0, 1, 1, 0, 1])
+    out = _run(s, lay, t, q, q_start, max_q)
+    check_no_device_error()
+    assert max_err(out, _oracle(s, lay, t, q, q_start)) <= TOL[s.cache_dtype]
 
 
 def test_full_size_verification_sampled():
