@@ -33,6 +33,13 @@
  *     safe values. pkv_device_error() reads and clears that flag.
  *   - Supported shapes: head_dim 64 or 128 (128 for fp8), block_size 16 or
  *     32, num_q_heads = g * num_kv_heads with 1 <= g <= 8.
+ *   - Scratch: the attention calls keep their intermediate state (split-KV
+ *     partials and claim words, prefix partials, multi-token partials, the
+ *     longest-first sequence order) in device buffers the library owns, one
+ *     set per device, grown with cudaMalloc when a call needs more. Calls
+ *     that overlap on the GPU (different streams with nothing ordering
+ *     them) race on those buffers: serialise them (or give each stream its
+ *     own workspace through paged_attn_decode_noalloc).
  *
  * The host allocator calls touch no device memory and are not thread-safe
  * per handle (one handle per scheduler thread).
