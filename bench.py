@@ -462,13 +462,17 @@ def run_prefill(a, s: W.Spec):
     cols = max(nq) * g
     tc = s.head_dim == 128 and cols >= 64 and s.scale > 0
     # kernels one call launches: the tensor-core kernel (after the one-CTA
-    # longest-first ordering pass when 1 < S <= 1024), or the warp-MMA
+    # longest-first ordering pass when 1 < S <= 1024 and the grid is more
+    # than one wave), or the warp-MMA
     # kernel (plus its merge when the KV is cut into chunks)
     decode_step = max(nq) == 1 and T == s.num_seqs  # served by the decode kernels
     if decode_step:
         per_call = 2
     elif tc:
-        per_call = 1 + (1 if 1 < s.num_seqs <= 1024 else 0)
+        rows = 256 if cols > 128 else 128  # query rows per CTA
+        ctas = s.num_seqs * s.num_kv_heads * -(-cols // rows)
+        sms = torch.cuda.get_device_properties(0).multi_processor_count
+        per_call = 1 + (1 if 1 < s.num_seqs <= 1024 and ctas > sms else 0)
     else:
         ecols = 16 if cols <= 16 else 32 if cols <= 32 else 64
         ncc = -(-cols // ecols)

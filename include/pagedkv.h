@@ -194,7 +194,8 @@ int paged_attn_decode_ex(const pkv_tensor* q, const pkv_tensor* k_cache,
  * warp MMAs, a column being one query head of one new token (the chunk's
  * columns share every K/V tile read); from 64 (D = 128, scale > 0), 128-row
  * tiles on the tensor cores, one or two per CTA, sequences taken longest
- * context first (a one-CTA ordering pass runs before them, S <= 1024).
+ * context first (a one-CTA ordering pass runs before them when S <= 1024
+ * and the grid is more than one wave).
  * With max_q_tokens = 1 and T = S (one new token per sequence) the call is
  * the decode step and runs the decode kernels; q_start, which can then only
  * be 0, 1, ..., S, is not read. Asynchronous on `stream`; an inconsistent

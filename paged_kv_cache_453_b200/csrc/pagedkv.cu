@@ -763,8 +763,10 @@ int launch_prefill(const pkv_tensor* q, const pkv_tensor* kc, const pkv_tensor* 
     }
     p.err = ds->err;
     p.nkv = 1;
-    // longest contexts first, so the last wave of CTAs is short ones
-    if (S > 1 && S <= kOrderMaxSeqs) {
+    // longest contexts first, so the last wave of CTAs is short ones (only
+    // when there is more than one wave)
+    const long long tc_ctas = S * Hk * ((cols + te->rows - 1) / te->rows);
+    if (S > 1 && S <= kOrderMaxSeqs && tc_ctas > ds->sms) {
       {
         std::lock_guard<std::mutex> lk(g_mu);
         if (!ds->ord && cudaMalloc(reinterpret_cast<void**>(&ds->ord), kOrderMaxSeqs * sizeof(int)) != cudaSuccess) {
