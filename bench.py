@@ -239,6 +239,25 @@ def profiled_traffic(s: W.Spec):
     return e.get("dram_bytes_per_launch")
 
 
+def prefill_traffic(s: W.Spec, q_tokens: int, kernel: str):
+    """DRAM bytes per tensor-core multi-token launch from the committed ncu
+    summary, if it was taken on the current kernel source, this workload
+    and this kernel."""
+    p = os.path.join(ROOT, "profiles", "prefill_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    h = hashlib.sha256()
+    for name in ("prefill.cuh", "prefill_tc.cuh", "prefill_tc2.cuh", "ptx.cuh"):
+        with open(os.path.join(ROOT, "paged_kv_cache_453_b200", "csrc", name), "rb") as fh:
+            h.update(fh.read())
+    e = d.get(f"{s.name}/{s.cache_dtype}/B{s.block_size}/q{q_tokens}")
+    if not e or e.get("kernel_sha") != h.hexdigest()[:16] or e.get("kernel") != kernel:
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
 # ---------------------------------------------------------------------------
 # CPU oracle timing (cpu_baseline leg and the reference arm)
 # ---------------------------------------------------------------------------
@@ -483,7 +502,8 @@ def run_prefill(a, s: W.Spec):
         kern = "prefill_tc2_kernel" if cols > 128 else "prefill_tc_kernel"
         roof = {"kernel": kern, "bound": "tensor", "achieved": flops / sec / 1e12, "peak": peak,
                 "unit": "TFLOP/s", "frac": flops / sec / 1e12 / peak, "peak_source": src + " (bf16 burst)",
-                "traffic": None, "alg_bytes_per_launch": alg, "flops_per_launch": flops}
+                "traffic": prefill_traffic(s, a.q_tokens, kern), "alg_bytes_per_launch": alg,
+                "flops_per_launch": flops}
     else:
         peak, src = measured_peak_hbm()
         roof = {"kernel": "decode_kernel + decode_merge_kernel" if decode_step else "prefill_kernel",
