@@ -96,7 +96,9 @@ def test_one_token_per_sequence_is_the_decode_step():
                         s.block_size, dec)
     torch.cuda.synchronize()
     check_no_device_error()
-    assert torch.equal(out, dec)
+    # same kernels; work stealing may cut units differently between calls,
+    # so the merge order (and the last bit) can differ
+    assert (out.float() - dec.float()).abs().max().item() <= TOL[s.cache_dtype]
     assert max_err(out, _oracle(s, lay, t, q, q_start)) <= TOL[s.cache_dtype]
 
 
