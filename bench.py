@@ -323,6 +323,16 @@ def dist_setup(a):
     return ws, rank, local, pg
 
 
+def max_over_ranks(vals, dist, device):
+    """Each value's maximum over all ranks (a timing: the slowest rank sets
+    the job's time). Without a process group the values come back as they are."""
+    if not dist:
+        return [float(v) for v in vals]
+    tt = torch.tensor([float(v) for v in vals], device=device, dtype=torch.float64)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return [float(x) for x in tt]
+
+
 def run_reference(a, s: W.Spec, ws: int, rank: int):
     if rank != 0:
         return
@@ -614,10 +624,7 @@ def main():
     clk = clocks.stop()
     elapsed_ms = start.elapsed_time(stop)
     dec_ms = sum(e0.elapsed_time(e1) for e0, e1 in ev) / K
-    if dist:
-        tt = torch.tensor([elapsed_ms, dec_ms], device=f"cuda:{dev}", dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        elapsed_ms, dec_ms = float(tt[0]), float(tt[1])
+    elapsed_ms, dec_ms = max_over_ranks([elapsed_ms, dec_ms], dist, f"cuda:{dev}")
     st = P.device_error(dev)
     if st != P.PKV_OK:
         raise SystemExit(f"device check failed: {P.status_string(st)}")
@@ -653,10 +660,7 @@ def main():
     e1.record()
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
-    if dist:
-        tt = torch.tensor([e2e_ms], device=f"cuda:{dev}", dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt[0])
+    (e2e_ms,) = max_over_ranks([e2e_ms], dist, f"cuda:{dev}")
     e2e_value = ws * kv_bytes / (e2e_ms / 1e3 / Ke) / 1e9
 
     if rank != 0:
