@@ -28,9 +28,11 @@
  *     PKV_ERR_UNSUPPORTED for a valid but unimplemented shape) and launches
  *     nothing. A failed launch returns PKV_ERR_CUDA.
  *   - Device-side checks (a block id outside the pool, a context length
- *     beyond the table row, a bounded wait that ran out) never fault: the
- *     kernel records the problem in a per-device flag and carries on with
- *     safe values. pkv_device_error() reads and clears that flag.
+ *     beyond the table row, a bounded wait that ran out, a tensor-core
+ *     kernel finding its shared or tensor memory placed otherwise than it
+ *     assumes) never fault: the kernel records the problem in a per-device
+ *     flag and carries on with safe values (or skips the work).
+ *     pkv_device_error() reads and clears that flag.
  *   - Supported shapes: head_dim 64 or 128 (128 for fp8), block_size 16 or
  *     32, num_q_heads = g * num_kv_heads with 1 <= g <= 8.
  *   - Scratch: the attention calls keep their intermediate state (split-KV
