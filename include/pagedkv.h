@@ -122,9 +122,14 @@ int pkv_version(void);
  *   out          [S, Hq, D], same dtype as q, written
  *
  * Uses a per-device workspace owned by the library: the first call on a
- * device (or one needing more) allocates it with cudaMalloc, which
- * synchronises; later calls reuse it. Calls that share a device and overlap
- * on the GPU must use paged_attn_decode_ex with separate workspaces.
+ * device (or one needing more) allocates it with cudaMalloc and zeroes it
+ * on `stream`; a larger one replaces the old buffer, which is released with
+ * cudaFree (that waits for all work on the device, so no stream still uses
+ * it). Either makes that call synchronise the device and keeps it out of
+ * stream capture: make a first call of the largest shape before capturing.
+ * Later calls reuse the buffer and do not synchronise. Calls that share a
+ * device and overlap on the GPU must use paged_attn_decode_ex with separate
+ * workspaces.
  */
 int paged_attn_decode(const pkv_tensor* q, const pkv_tensor* k_cache, const pkv_tensor* v_cache,
                       const pkv_tensor* block_tables, const pkv_tensor* context_lens,
@@ -139,7 +144,10 @@ int paged_attn_decode(const pkv_tensor* q, const pkv_tensor* k_cache, const pkv_
  *
  *   k_cache, v_cache  [NB, Hk, B, D] PKV_FP8_E4M3 codes
  *   k_scale, v_scale  [Hk] f32 device: element value = decode(code) * scale[h]
- *   q, out            f16 | bf16 (q is rounded to f16 for the dot products)
+ *   q, out            f16 | bf16 (q is rounded to f16 for the dot products;
+ *                     a bf16 row of one head whose largest magnitude is 2^16
+ *                     or more is first scaled by a power of two, which its
+ *                     logit scale takes back, so it does not overflow)
  */
 int paged_attn_decode_fp8(const pkv_tensor* q, const pkv_tensor* k_cache,
                           const pkv_tensor* v_cache, const pkv_tensor* k_scale,
@@ -164,13 +172,24 @@ size_t paged_attn_decode_workspace_bytes(int num_q_heads, int num_kv_heads, int 
  * call leaves zeroed again. The workspace must not be used by another call
  * until this one has finished on the GPU; after a PKV_ERR_DEVICE_CHECK from
  * a call that used it, zero it again.
+ *
+ * flags: 0, or PKV_DECODE_DETERMINISTIC. By default a warp that runs out of
+ * work takes over part of another warp's remaining blocks, so where a
+ * sequence's context is cut between warps (and so the order in which its
+ * partial sums are added) changes from call to call with the timing: results
+ * agree to rounding, not bit for bit. PKV_DECODE_DETERMINISTIC cuts the
+ * work only where the static split puts the cuts and merges the pieces in a
+ * fixed order, so identical calls on the same device give identical bits
+ * (the slowest SMs then set the time: usually a little slower). Other bits:
+ * PKV_ERR_INVALID_ARG.
  */
+#define PKV_DECODE_DETERMINISTIC 1u
 int paged_attn_decode_ex(const pkv_tensor* q, const pkv_tensor* k_cache,
                          const pkv_tensor* v_cache, const pkv_tensor* k_scale,
                          const pkv_tensor* v_scale, const pkv_tensor* block_tables,
                          const pkv_tensor* context_lens, int num_kv_heads, float scale,
                          int block_size, pkv_tensor* out, void* workspace,
-                         size_t workspace_bytes, void* stream);
+                         size_t workspace_bytes, unsigned flags, void* stream);
 
 /*
  * paged_attn_prefill - causal attention of several new tokens per sequence
@@ -362,7 +381,12 @@ int reshape_and_cache_fp8(const pkv_tensor* k, const pkv_tensor* v, pkv_tensor* 
  *   k_cache, v_cache [NB, Hk, B, D] any element type (same for both)
  *   pairs         [n, 2] int32 device; every dst distinct and no dst also a
  *                 src in the same call (the allocator's copy-on-write pairs
- *                 satisfy this); ids outside the pool are skipped and flagged.
+ *                 satisfy this), so that every copy reads the pool as it was
+ *                 before the call whatever order they run in. A pair whose
+ *                 dst is another pair's src or dst, or whose src is another
+ *                 pair's dst, is not copied and is flagged
+ *                 (PKV_ERR_DEVICE_CHECK); the other pairs are copied. Ids
+ *                 outside the pool are skipped and flagged.
  */
 int copy_blocks(pkv_tensor* k_cache, pkv_tensor* v_cache, const pkv_tensor* pairs,
                 void* stream);

@@ -10,7 +10,7 @@ Device calls (names and argument order follow include/pagedkv.h):
                       num_kv_heads, scale, block_size, out)
     paged_attn_decode_fp8(q, k_cache, v_cache, k_scale, v_scale, block_tables,
                           context_lens, num_kv_heads, scale, block_size, out)
-    paged_attn_decode_ex(..., workspace=<uint8 cuda tensor>)
+    paged_attn_decode_ex(..., workspace=<uint8 cuda tensor>, flags=0 | PKV_DECODE_DETERMINISTIC)
     reshape_and_cache(k, v, k_cache, v_cache, slot_mapping)
     reshape_and_cache_fp8(k, v, k_cache, v_cache, slot_mapping, k_scale, v_scale)
     copy_blocks(k_cache, v_cache, pairs)
@@ -39,6 +39,9 @@ PKV_ERR_CUDA = -7
 PKV_ERR_DEVICE_CHECK = -8
 PKV_ERR_WORKSPACE = -9
 PKV_ERR_SCRATCH_LIMIT = -10
+
+NOALLOC_SCRATCH_BYTES = 16 << 20  # PKV_NOALLOC_SCRATCH_BYTES of include/pagedkv.h
+PKV_DECODE_DETERMINISTIC = 1  # paged_attn_decode_ex flag: static split, identical bits per call
 
 # Every symbol include/pagedkv.h declares.
 EXPORTED = (
@@ -87,7 +90,8 @@ def lib() -> ctypes.CDLL:
                                                      ctypes.c_int, P, vp]),
             "paged_attn_decode_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int] * 6),
             "paged_attn_decode_ex": (ctypes.c_int, [P, P, P, P, P, P, P, ctypes.c_int, f32,
-                                                    ctypes.c_int, P, vp, ctypes.c_size_t, vp]),
+                                                    ctypes.c_int, P, vp, ctypes.c_size_t, ctypes.c_uint,
+                                                    vp]),
             "paged_attn_decode_noalloc": (ctypes.c_int, [P, P, P, P, P, P, P, ctypes.c_int, f32,
                                                          ctypes.c_int, P, vp]),
             "reshape_and_cache": (ctypes.c_int, [P, P, P, P, P, vp]),
@@ -216,6 +220,17 @@ class PrefixGroups:
         self.members = mem.to(dev) if mem.numel() else torch.zeros(0, dtype=torch.int32, device=dev)
         self.prefix_blocks = pb.to(dev)
 
+    @classmethod
+    def on_device(cls, prefix_blocks, group_start, members, num_groups: int, max_group_size: int,
+                  max_prefix_blocks: int) -> "PrefixGroups":
+        """A grouping whose arrays already live on the device (for instance
+        views into a caller's staging buffer)."""
+        g = cls.__new__(cls)
+        g.prefix_blocks, g.group_start, g.members = prefix_blocks, group_start, members
+        g.num_groups, g.max_group_size = int(num_groups), int(max_group_size)
+        g.max_prefix_blocks = int(max_prefix_blocks)
+        return g
+
 
 def paged_attn_decode_cascade(q, k_cache, v_cache, block_tables, context_lens, groups: PrefixGroups,
                               num_kv_heads: int, scale: float, block_size: int, out, stream=None) -> None:
@@ -297,7 +312,7 @@ def workspace_bytes(num_q_heads: int, num_kv_heads: int, head_dim: int, block_si
 
 def paged_attn_decode_ex(q, k_cache, v_cache, block_tables, context_lens, num_kv_heads: int,
                          scale: float, block_size: int, out, workspace, k_scale=None, v_scale=None,
-                         stream=None) -> None:
+                         stream=None, flags: int = 0) -> None:
     fp8 = k_scale is not None
     ks = _desc(k_scale) if fp8 else None
     vs = _desc(v_scale) if fp8 else None
@@ -308,7 +323,7 @@ def paged_attn_decode_ex(q, k_cache, v_cache, block_tables, context_lens, num_kv
                                       _ref(ds[3]), _ref(ds[4]), int(num_kv_heads), float(scale),
                                       int(block_size), _ref(ds[5]),
                                       ctypes.c_void_p(workspace.data_ptr()),
-                                      workspace.numel() * workspace.element_size(),
+                                      workspace.numel() * workspace.element_size(), int(flags),
                                       _stream(stream)), "paged_attn_decode_ex")
 
 
@@ -577,7 +592,7 @@ class Prepared:
 
 def prepare_decode(q, k_cache, v_cache, block_tables, context_lens, num_kv_heads: int, scale: float,
                    block_size: int, out, k_scale=None, v_scale=None, workspace=None,
-                   stream=None) -> Prepared:
+                   stream=None, flags: int = 0) -> Prepared:
     fp8 = k_scale is not None
     ds = [_desc(q), _desc(k_cache, fp8), _desc(v_cache, fp8), _desc(block_tables), _desc(context_lens),
           _desc(out)]
@@ -594,7 +609,7 @@ def prepare_decode(q, k_cache, v_cache, block_tables, context_lens, num_kv_heads
                 ctypes.byref(ks) if fp8 else None, ctypes.byref(vs) if fp8 else None,
                 ctypes.byref(ds[3]), ctypes.byref(ds[4]), int(num_kv_heads), float(scale),
                 int(block_size), ctypes.byref(ds[5]), ctypes.c_void_p(workspace.data_ptr()),
-                workspace.numel() * workspace.element_size())
+                workspace.numel() * workspace.element_size(), int(flags))
         return Prepared("paged_attn_decode_ex", L.paged_attn_decode_ex, args, (ds, ks, vs, workspace),
                         stream)
     args = (ctypes.byref(ds[0]), ctypes.byref(ds[1]), ctypes.byref(ds[2]), ctypes.byref(ds[3]),

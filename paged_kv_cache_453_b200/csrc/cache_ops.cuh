@@ -9,7 +9,8 @@
 //
 // copy_blocks: the device half of copy-on-write ("Parallel Sampling & Beam
 // Search via Copy-on-Write"): block dst := block src in both pools, bit-exact,
-// 16-byte vectors.
+// 16-byte vectors; pairs that would make the result depend on the order of
+// the copies are refused (flagged).
 //
 // swap_blocks_kernel: the device half of preemption by swapping ("Preemption
 // and eviction", "Preemption & GPU Swapping"): record i of a page-locked host
@@ -145,12 +146,28 @@ struct CopyParams {
   int row_vecs;                // 16-byte vectors per token row
 };
 
-// grid.x = pair, grid.y = chunk of the block's vectors
+// grid.x = pair, grid.y = chunk of the block's vectors. Every copy of a call
+// reads the pool as it was before the call; that holds whatever order the
+// CTAs run in as long as no block is written by one pair and read or written
+// by another. Each CTA checks its own pair against all the others: a pair
+// that shares its destination with another pair's source or destination, or
+// whose source is another pair's destination, is not copied and is flagged
+// (the other pairs are still copied).
 __global__ void copy_blocks_kernel(const __grid_constant__ CopyParams p, int* err) {
   const int pi = blockIdx.x;
   const int src = p.pairs[pi * p.pr_s], dst = p.pairs[pi * p.pr_s + 1];
   if (src < 0 || src >= p.NB || dst < 0 || dst >= p.NB) {
     if (threadIdx.x == 0 && blockIdx.y == 0) atomicOr(err, kErrBadBlock);
+    return;
+  }
+  int clash = 0;
+  for (int j = threadIdx.x; j < p.n; j += blockDim.x) {
+    if (j == pi) continue;
+    const int sj = p.pairs[j * p.pr_s], dj = p.pairs[j * p.pr_s + 1];
+    clash |= (sj == dst) | (dj == dst) | (dj == src);
+  }
+  if (__syncthreads_or(clash)) {
+    if (threadIdx.x == 0 && blockIdx.y == 0) atomicOr(err, kErrBadCopy);
     return;
   }
   const int per_head = p.B * p.row_vecs;

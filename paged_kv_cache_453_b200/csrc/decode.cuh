@@ -38,8 +38,10 @@
 // movmatrix per 8x8 tile. Slots past the context length are masked by
 // predicate: their logits become -inf and their V entries 0, so NaN there
 // never reaches the result. fp8-e4m3 tiles are widened to f16 in registers
-// (exact); q is rounded to f16 for that path and the per-head scales are
-// folded into the logit scale and the output.
+// (exact); q is rounded to f16 for that path (a bf16 row beyond the f16 range
+// is first scaled by a power of two, folded back into that head's logit
+// scale) and the per-head scales are folded into the logit scale and the
+// output.
 #pragma once
 
 #include <type_traits>
@@ -71,6 +73,7 @@ struct DecodeParams {
   int S, Hk, g, MB, NB;
   int nwt;                    // consumer warps in the grid
   int tag;                    // per-call tag of steal records (never 0)
+  int steal;                  // 1: warps that run out of work steal; 0: static split only
   int pool_slots;             // partial slots available to steals
   long long* hdr;             // workspace header: [0] total items W
   int* err;                   // device-check flag (OR of error bits)
@@ -250,6 +253,12 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
   // memory; everything below may.
   pdl_wait();
 
+  // The owner's first claim on its range word (NS items, see run_range) goes
+  // out now so its round trip overlaps the length scan below.
+  const int gw = blockIdx.x * NC + warp;
+  unsigned long long first_claim = 0;
+  if (p.steal && lane == 0) first_claim = atomicAdd(p.words + gw, static_cast<unsigned long long>(NS));
+
   // ---- total work and each thread's chunk prefix (every CTA, redundantly) ----
   {
     const int s0 = static_cast<int>((static_cast<long long>(tid) * p.S) / C::NT);
@@ -283,7 +292,6 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
   const long long W = *total;
   if (blockIdx.x == 0 && tid == 0) p.hdr[0] = W;
 
-  const int gw = blockIdx.x * NC + warp;
   const long long my_lo = range_lo(gw, W, p.nwt);
   const long long my_len = range_lo(gw + 1, W, p.nwt) - my_lo;
   if (my_len >= (1ll << 23)) {  // range words hold 24-bit counts
@@ -351,7 +359,7 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
   uint32_t qb[C::KS][2];
   float acc[C::MT][4];
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-  float sl = p.scale_log2;
+  float sl0 = p.scale_log2, sl1 = p.scale_log2;  // logit scales of head columns 2c and 2c + 1
   const bool h0_ok = (2 * c) < p.g;
   const bool h1_ok = (2 * c + 1) < p.g;
 
@@ -372,7 +380,12 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
     unsigned long long* wp = p.words + owner;
     const unsigned own_len = static_cast<unsigned>(hi - a);
     bool claiming = claim;
-    unsigned long long pend = 0;  // lane 0: pending claim of the item at pc
+    // Claims: lane 0's `pend` is the range word as the latest claim found
+    // it; that claim covers pend_n items, pend_off of them issued so far. The
+    // first claim (NS items) was made at the kernel's start, later ones take
+    // one item each.
+    unsigned long long pend = first_claim;
+    int pend_off = 0, pend_n = NS;
 
     auto issue = [&](int stage) {
       const uint32_t bar = my_bars + stage * 8;
@@ -422,7 +435,8 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
     auto try_issue = [&]() -> bool {
       if (pc.k >= hi) return false;
       if (claiming) {
-        const unsigned long long w = __shfl_sync(0xffffffffu, pend, 0);
+        const unsigned long long w =
+            __shfl_sync(0xffffffffu, pend, 0) + static_cast<unsigned long long>(pend_off);
         if (rw_front(w) + rw_back(w) >= own_len) {
           claiming = false;
           hi = pc.k;  // everything from here on belongs to thieves
@@ -432,12 +446,15 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
       issue(static_cast<int>(issued % NS));
       pc.advance(p, max_len);
       ++issued;
-      if (claiming && lane == 0) pend = atomicAdd(wp, 1ull);  // claim the following item
+      if (claiming && ++pend_off == pend_n) {  // claim the following item
+        pend_off = 0;
+        pend_n = 1;
+        if (lane == 0) pend = atomicAdd(wp, 1ull);
+      }
       return true;
     };
 
     if (lane == 0) p.desc[owner * (1 + kMaxSteals) + sub] = make_int4(-1, 0, 0, 0);
-    if (claiming && lane == 0) pend = atomicAdd(wp, 1ull);
     for (int i = 0; i < NS; ++i)
       if (!try_issue()) break;
 
@@ -446,8 +463,9 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
       for (int mt = 0; mt < C::MT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
       m0 = m1 = -INFINITY;
       l0 = l1 = 0.f;
-      sl = p.scale_log2;
+      float sl = p.scale_log2;
       if constexpr (FP8) sl *= __ldg(p.k_scale + cur.h);
+      sl0 = sl1 = sl;
       const bool row_ok = r < p.g;
       const long long qoff = cur.s * p.q_s + (static_cast<long long>(cur.h) * p.g + r) * p.q_h;
       if constexpr (!FP8) {
@@ -463,25 +481,45 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
         // and slots 2c+8, 2c+9 <- dims 4c+2, 4c+3 of each 16-dim step.
         const uint2* qp =
             reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(p.q) + qoff);
+        float f[C::KS][4];
+        float amax = 0.f;
 #pragma unroll
         for (int ks = 0; ks < C::KS; ++ks) {
           uint2 v = row_ok ? __ldg(qp + (ks * 16 + 4 * c) / 4) : make_uint2(0u, 0u);
-          float f0, f1, f2, f3;
           if constexpr (QBF) {
-            f0 = __uint_as_float(v.x << 16);
-            f1 = __uint_as_float(v.x & 0xffff0000u);
-            f2 = __uint_as_float(v.y << 16);
-            f3 = __uint_as_float(v.y & 0xffff0000u);
+            f[ks][0] = __uint_as_float(v.x << 16);
+            f[ks][1] = __uint_as_float(v.x & 0xffff0000u);
+            f[ks][2] = __uint_as_float(v.y << 16);
+            f[ks][3] = __uint_as_float(v.y & 0xffff0000u);
+            amax = fmaxf(amax, fmaxf(fmaxf(fabsf(f[ks][0]), fabsf(f[ks][1])),
+                                     fmaxf(fabsf(f[ks][2]), fabsf(f[ks][3]))));
           } else {
             __half2 a2 = *reinterpret_cast<__half2*>(&v.x);
             __half2 b2 = *reinterpret_cast<__half2*>(&v.y);
-            f0 = __low2float(a2);
-            f1 = __high2float(a2);
-            f2 = __low2float(b2);
-            f3 = __high2float(b2);
+            f[ks][0] = __low2float(a2);
+            f[ks][1] = __high2float(a2);
+            f[ks][2] = __low2float(b2);
+            f[ks][3] = __high2float(b2);
           }
-          qb[ks][0] = pack2<false>(f0, f1);
-          qb[ks][1] = pack2<false>(f2, f3);
+        }
+        // A bf16 row may exceed the f16 range (2^16 and up): it is scaled by
+        // a power of two 2^-e (exact) and its logit scale by 2^e. Rows below
+        // 2^16 keep e = 0. The row of head r is held by the 4 lanes 4r .. 4r+3.
+        float qs = 1.f;
+        if constexpr (QBF) {
+          amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+          amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+          const int ex = static_cast<int>((__float_as_uint(amax) >> 23) & 0xffu) - 127;
+          const int e = ex >= 16 ? ex - 15 : 0;
+          qs = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+          const int e0 = __shfl_sync(0xffffffffu, e, 8 * c), e1 = __shfl_sync(0xffffffffu, e, 8 * c + 4);
+          sl0 = sl * __uint_as_float(static_cast<uint32_t>(127 + e0) << 23);
+          sl1 = sl * __uint_as_float(static_cast<uint32_t>(127 + e1) << 23);
+        }
+#pragma unroll
+        for (int ks = 0; ks < C::KS; ++ks) {
+          qb[ks][0] = pack2<false>(f[ks][0] * qs, f[ks][1] * qs);
+          qb[ks][1] = pack2<false>(f[ks][2] * qs, f[ks][3] * qs);
         }
       }
     };
@@ -695,10 +733,10 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
 #pragma unroll
         for (int tt = 0; tt < C::TT; ++tt) {
           const int t0 = tt * 16 + r, t1 = t0 + 8;
-          sacc[tt][0] = t0 < nvalid ? sacc[tt][0] * sl : -INFINITY;
-          sacc[tt][1] = t0 < nvalid ? sacc[tt][1] * sl : -INFINITY;
-          sacc[tt][2] = t1 < nvalid ? sacc[tt][2] * sl : -INFINITY;
-          sacc[tt][3] = t1 < nvalid ? sacc[tt][3] * sl : -INFINITY;
+          sacc[tt][0] = t0 < nvalid ? sacc[tt][0] * sl0 : -INFINITY;
+          sacc[tt][1] = t0 < nvalid ? sacc[tt][1] * sl1 : -INFINITY;
+          sacc[tt][2] = t1 < nvalid ? sacc[tt][2] * sl0 : -INFINITY;
+          sacc[tt][3] = t1 < nvalid ? sacc[tt][3] * sl1 : -INFINITY;
           mx0 = fmaxf(mx0, fmaxf(sacc[tt][0], sacc[tt][2]));
           mx1 = fmaxf(mx1, fmaxf(sacc[tt][1], sacc[tt][3]));
         }
@@ -764,7 +802,8 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
   };
 
   // ---- own range, then steal until no remainder is worth splitting ----
-  if (my_len > 0 && !run_range(my_lo, my_lo + my_len, true, gw, 0, 2ll * gw)) return;
+  if (my_len > 0 && !run_range(my_lo, my_lo + my_len, p.steal != 0, gw, 0, 2ll * gw)) return;
+  if (!p.steal) return;  // static split: every unit is cut at the same places in every call
 
   const long long nominal = W / p.nwt;  // every static range is nominal or nominal + 1 long
   for (int attempt = 0; attempt < 4 * kStealTries; ++attempt) {
@@ -844,24 +883,31 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
 // together; (2) for each of its sub-ranges whose last piece starts a cut
 // unit, the steal records of the following static ranges, one range per
 // thread (the next 128, and so on), listing the piece slots of every
-// sub-range that starts before the unit's end (order does not matter to the
-// merge); (3) the pieces' running maxima per head; (4) the rescaled sums.
+// sub-range that starts before the unit's end; (3) the pieces' running
+// maxima per head; (4) the rescaled sums. A piece's place in the list comes
+// from a block-wide scan (range order, then item order inside a range), so
+// the list is the same every time it is built: a unit with more pieces than
+// the list holds is folded in several passes over it, and a call without
+// steals folds every unit's pieces in one fixed order.
 template <bool QBF, int D>
 __global__ void __launch_bounds__(128, 8) decode_merge_kernel(const __grid_constant__ DecodeParams p) {
   pdl_wait();  // the decode grid has finished
   pdl_launch_dependents();
   constexpr int NT = 128;
-  constexpr int kCap = 2048;  // pieces of one cut unit
+  constexpr int kCap = 1024;  // pieces folded per pass
   constexpr int ND = 1 + kMaxSteals;
   __shared__ int s_slot[kCap];
+  __shared__ float s_red[NT * 10];
+  __shared__ int s_wsum[NT / 32];
   __shared__ int4 s_desc[ND];
   __shared__ int4 s_rec[kMaxSteals];
   __shared__ long long s_own_start[kMaxSteals];
   __shared__ int s_own_slot[kMaxSteals];
   __shared__ long long s_W;
-  __shared__ int s_n, s_m_own;
+  __shared__ int s_m_own;
 
   const int tid = threadIdx.x;
+  const int lane = tid & 31;
   const int w0 = blockIdx.x;
   const int g = p.g;
   const int E = g * D;
@@ -902,6 +948,36 @@ __global__ void __launch_bounds__(128, 8) decode_merge_kernel(const __grid_const
   __syncthreads();
   const int m_own = s_m_own;
 
+  // Piece slots of the sub-ranges of warp range v that start before U1, in
+  // item order from its sub-range `from` on (0 = the owner's own part,
+  // i >= 1 = steal m - i).
+  auto list_range = [&](int v, int from, long long U1, int* out) -> int {
+    long long st_v[kMaxSteals];
+    int sl_v[kMaxSteals];
+    int m;
+    if (v == w0) {
+      m = m_own;
+      for (int j = 0; j < m; ++j) {
+        st_v[j] = s_own_start[j];
+        sl_v[j] = s_own_slot[j];
+      }
+    } else {
+      int4 rec[kMaxSteals];
+#pragma unroll
+      for (int j = 0; j < kMaxSteals; ++j) rec[j] = p.steal_info[v * kMaxSteals + j];
+      m = valid_steals(v, rec, st_v, sl_v);
+    }
+    const long long vlo = range_lo(v, W, p.nwt), vhi = range_lo(v + 1, W, p.nwt);
+    int cnt = 0;
+    for (int pos = from; pos <= m; ++pos) {
+      const long long st = pos == 0 ? vlo : st_v[m - pos];
+      const long long en = pos < m ? st_v[m - pos - 1] : vhi;
+      if (st >= U1) break;
+      if (en > st) out[cnt++] = pos == 0 ? 2 * v : sl_v[m - pos];
+    }
+    return cnt;
+  };
+
   for (int k = 0; k <= m_own; ++k) {
     const int4 d = s_desc[k];
     if (d.x < 0) continue;
@@ -915,55 +991,12 @@ __global__ void __launch_bounds__(128, 8) decode_merge_kernel(const __grid_const
     // item-order position of this sub-range in w0's list: 0 = owner part,
     // i >= 1 = steal (m - i)
     const int pos0 = (k == 0) ? 0 : m_own - (k - 1);
-    if (tid == 0) {
-      s_n = 1;
-      s_slot[0] = ((k == 0) ? 2 * w0 : s_own_slot[k - 1]) + 1;
-    }
-    __syncthreads();
-    // round 2: the pieces of the sub-ranges after this one that start before U1
-    for (int chunk = 0;; ++chunk) {
-      const int v = w0 + chunk * NT + tid;
-      if (v < p.nwt && range_lo(v, W, p.nwt) < U1) {
-        long long st_v[kMaxSteals];
-        int sl_v[kMaxSteals];
-        int m;
-        if (v == w0) {
-          m = m_own;
-          for (int j = 0; j < m; ++j) {
-            st_v[j] = s_own_start[j];
-            sl_v[j] = s_own_slot[j];
-          }
-        } else {
-          int4 rec[kMaxSteals];
-#pragma unroll
-          for (int j = 0; j < kMaxSteals; ++j) rec[j] = p.steal_info[v * kMaxSteals + j];
-          m = valid_steals(v, rec, st_v, sl_v);
-        }
-        const long long vlo = range_lo(v, W, p.nwt), vhi = range_lo(v + 1, W, p.nwt);
-        for (int pos = (v == w0) ? pos0 + 1 : 0; pos <= m; ++pos) {
-          const long long st = pos == 0 ? vlo : st_v[m - pos];
-          const long long en = pos < m ? st_v[m - pos - 1] : vhi;
-          if (st >= U1) break;
-          if (en > st) {
-            const int idx = atomicAdd(&s_n, 1);
-            if (idx < kCap) s_slot[idx] = pos == 0 ? 2 * v : sl_v[m - pos];
-          }
-        }
-      }
-      const long long next = w0 + static_cast<long long>(chunk + 1) * NT;
-      if (next >= p.nwt || range_lo(next, W, p.nwt) >= U1) break;
-    }
-    __syncthreads();
-    const int n = s_n;
-    if (n > kCap) {
-      if (tid == 0) atomicOr(p.err, kErrBadMerge);
-      __syncthreads();
-      continue;
-    }
-    // round 3: fold the pieces in. Thread t owns an 8-element chunk of one
-    // head (chunk t % NC8) and the pieces q = t / NC8 (mod PG); it loads four
-    // pieces at a time (m, l and two float4 of O each) before folding them
-    // with an online max / rescale, then the piece groups are combined.
+    const int first = ((k == 0) ? 2 * w0 : s_own_slot[k - 1]) + 1;  // the unit's first piece
+
+    // Thread t owns an 8-element chunk of one head (chunk t % NC8) and the
+    // pieces q = t / NC8 (mod PG) of each pass; it loads four pieces at a
+    // time (m, l and two float4 of O each) before folding them with an
+    // online max / rescale, then the piece groups are combined.
     const int NC8 = E / 8;                // chunks of 8 elements (D is a multiple of 8)
     const int PG = NT / NC8;              // piece groups (1 at g = 8, D = 128)
     const int c8 = tid % NC8, pg = tid / NC8;
@@ -971,47 +1004,84 @@ __global__ void __launch_bounds__(128, 8) decode_merge_kernel(const __grid_const
     float rm = -INFINITY, rl = 0.f, ra[8];
 #pragma unroll
     for (int x = 0; x < 8; ++x) ra[x] = 0.f;
-    if (pg < PG) {
-      for (int q0 = pg; q0 < n; q0 += 4 * PG) {
-        float mv[4], lv[4];
-        float4 o0[4], o1[4];
+
+    for (int pass = 0;; ++pass) {
+      // round 2: list the pieces; this pass keeps positions [wlo, wlo + kCap)
+      const int wlo = pass * kCap;
+      if (pass == 0 && tid == 0) s_slot[0] = first;
+      int run = 1;  // positions taken so far (position 0: the first piece)
+      for (int chunk = 0;; ++chunk) {
+        const int v = w0 + chunk * NT + tid;
+        int sl[ND];
+        int cnt = 0;
+        if (v < p.nwt && range_lo(v, W, p.nwt) < U1) cnt = list_range(v, v == w0 ? pos0 + 1 : 0, U1, sl);
+        int incl = cnt;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int q = q0 + u * PG;
-          mv[u] = -INFINITY;
-          lv[u] = 0.f;
-          o0[u] = o1[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (q < n) {
-            const long long base = static_cast<long long>(s_slot[q]) * g + hi8;
-            mv[u] = p.part_ml[base * 2];
-            lv[u] = p.part_ml[base * 2 + 1];
-            const float4* op = reinterpret_cast<const float4*>(p.part_o + base * D + d8);
-            o0[u] = op[0];
-            o1[u] = op[1];
+        for (int o = 1; o < 32; o <<= 1) {
+          const int u = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += u;
+        }
+        if (lane == 31) s_wsum[tid >> 5] = incl;
+        __syncthreads();
+        int at = run + incl - cnt, tot = 0;
+#pragma unroll
+        for (int w = 0; w < NT / 32; ++w) {
+          const int x = s_wsum[w];
+          if (w < (tid >> 5)) at += x;
+          tot += x;
+        }
+        for (int i = 0; i < cnt; ++i, ++at)
+          if (at >= wlo && at < wlo + kCap) s_slot[at - wlo] = sl[i];
+        run += tot;
+        __syncthreads();
+        const long long next = w0 + static_cast<long long>(chunk + 1) * NT;
+        if (next >= p.nwt || range_lo(next, W, p.nwt) >= U1) break;
+      }
+      const int n = min(run - wlo, kCap);
+      // rounds 3 and 4: fold this pass's pieces in
+      if (pg < PG) {
+        for (int q0 = pg; q0 < n; q0 += 4 * PG) {
+          float mv[4], lv[4];
+          float4 o0[4], o1[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int q = q0 + u * PG;
+            mv[u] = -INFINITY;
+            lv[u] = 0.f;
+            o0[u] = o1[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (q < n) {
+              const long long base = static_cast<long long>(s_slot[q]) * g + hi8;
+              mv[u] = p.part_ml[base * 2];
+              lv[u] = p.part_ml[base * 2 + 1];
+              const float4* op = reinterpret_cast<const float4*>(p.part_o + base * D + d8);
+              o0[u] = op[0];
+              o1[u] = op[1];
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            if (mv[u] == -INFINITY) continue;
+            const float mn = fmaxf(rm, mv[u]);
+            const float sa = (rm == -INFINITY) ? 0.f : exp2f(rm - mn), sb = exp2f(mv[u] - mn);
+            rl = rl * sa + lv[u] * sb;
+            ra[0] = ra[0] * sa + o0[u].x * sb;
+            ra[1] = ra[1] * sa + o0[u].y * sb;
+            ra[2] = ra[2] * sa + o0[u].z * sb;
+            ra[3] = ra[3] * sa + o0[u].w * sb;
+            ra[4] = ra[4] * sa + o1[u].x * sb;
+            ra[5] = ra[5] * sa + o1[u].y * sb;
+            ra[6] = ra[6] * sa + o1[u].z * sb;
+            ra[7] = ra[7] * sa + o1[u].w * sb;
+            rm = mn;
           }
         }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          if (mv[u] == -INFINITY) continue;
-          const float mn = fmaxf(rm, mv[u]);
-          const float sa = (rm == -INFINITY) ? 0.f : exp2f(rm - mn), sb = exp2f(mv[u] - mn);
-          rl = rl * sa + lv[u] * sb;
-          ra[0] = ra[0] * sa + o0[u].x * sb;
-          ra[1] = ra[1] * sa + o0[u].y * sb;
-          ra[2] = ra[2] * sa + o0[u].z * sb;
-          ra[3] = ra[3] * sa + o0[u].w * sb;
-          ra[4] = ra[4] * sa + o1[u].x * sb;
-          ra[5] = ra[5] * sa + o1[u].y * sb;
-          ra[6] = ra[6] * sa + o1[u].z * sb;
-          ra[7] = ra[7] * sa + o1[u].w * sb;
-          rm = mn;
-        }
       }
+      __syncthreads();  // the list is rebuilt by the next pass or unit
+      if (run <= wlo + kCap) break;
     }
-    // combine the piece groups of each chunk (through the now unused list)
+    // combine the piece groups of each chunk
     if (PG > 1) {
-      float* red = reinterpret_cast<float*>(s_slot);  // [NT][10]
-      __syncthreads();
+      float* red = s_red;  // [NT][10]
       red[tid * 10 + 0] = rm;
       red[tid * 10 + 1] = rl;
 #pragma unroll
@@ -1066,7 +1136,7 @@ __global__ void __launch_bounds__(128, 8) decode_merge_kernel(const __grid_const
         }
       }
     }
-    __syncthreads();  // s_slot / s_n are reused by the next cut unit
+    __syncthreads();  // s_red is reused by the next cut unit
   }
 }
 

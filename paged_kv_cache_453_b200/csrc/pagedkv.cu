@@ -351,10 +351,11 @@ struct CascadeTail {
 // Launch decode + merge. lib_ws: use (and grow) the library's workspace for
 // this device; otherwise `ws` is the caller's. fit: shrink the steal-slot pool
 // to fit ws_bytes; clear: zero the claim state first (callers that cannot
-// vouch for it).
+// vouch for it); fixed_split: no work stealing (identical calls give
+// identical bits).
 int launch_decode(const DecodeArgs& a, bool fp8, void* ws, size_t ws_bytes, bool lib_ws,
                   cudaStream_t stream, bool fit = false, bool clear = false,
-                  const CascadeTail* tail = nullptr) {
+                  const CascadeTail* tail = nullptr, bool fixed_split = false) {
   int ck = 0;
   DecodeLaunch* e = nullptr;
   int st = check_decode(a, fp8, &ck, &e);
@@ -377,12 +378,14 @@ int launch_decode(const DecodeArgs& a, bool fp8, void* ws, size_t ws_bytes, bool
       ds->ws = nullptr;
       ds->ws_bytes = 0;
       if (cudaMalloc(&ds->ws, L.total) != cudaSuccess) return PKV_ERR_CUDA;
-      if (cudaMemset(ds->ws, 0, L.total) != cudaSuccess) return PKV_ERR_CUDA;
+      // zeroed on the call's stream, so this launch sees it zeroed
+      if (cudaMemsetAsync(ds->ws, 0, L.total, stream) != cudaSuccess) return PKV_ERR_CUDA;
       ds->ws_bytes = L.total;
     }
     ws = ds->ws;
     ws_bytes = ds->ws_bytes;
   }
+  if (fit && L.total > ws_bytes) return PKV_ERR_SCRATCH_LIMIT;  // even with no steal slots
   if (!ws || ws_bytes < L.total || !aligned(ws, 16)) return PKV_ERR_WORKSPACE;
   if (clear && cudaMemsetAsync(ws, 0, L.steal, stream) != cudaSuccess) return PKV_ERR_CUDA;
 
@@ -410,6 +413,7 @@ int launch_decode(const DecodeArgs& a, bool fp8, void* ws, size_t ws_bytes, bool
   p.NB = static_cast<int>(a.kc->shape[0]);
   p.nwt = nwt;
   p.tag = next_tag();
+  p.steal = fixed_split ? 0 : 1;
   p.pool_slots = L.pool_slots;
   uint8_t* w = static_cast<uint8_t*>(ws);
   p.hdr = reinterpret_cast<long long*>(w + L.hdr);
@@ -1078,12 +1082,14 @@ int paged_attn_decode_ex(const pkv_tensor* q, const pkv_tensor* k_cache,
                          const pkv_tensor* v_scale, const pkv_tensor* block_tables,
                          const pkv_tensor* context_lens, int num_kv_heads, float scale,
                          int block_size, pkv_tensor* out, void* workspace,
-                         size_t workspace_bytes, void* stream) {
+                         size_t workspace_bytes, unsigned flags, void* stream) {
+  if (flags & ~static_cast<unsigned>(PKV_DECODE_DETERMINISTIC)) return PKV_ERR_INVALID_ARG;
   const bool fp8 = k_cache && k_cache->dtype == PKV_FP8_E4M3;
   DecodeArgs a{q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
                num_kv_heads, scale, block_size, out};
   return launch_decode(a, fp8, workspace, workspace_bytes, false,
-                       static_cast<cudaStream_t>(stream));
+                       static_cast<cudaStream_t>(stream), false, false, nullptr,
+                       (flags & PKV_DECODE_DETERMINISTIC) != 0);
 }
 
 // Decode for callers that cannot allocate: the scratch is the static
@@ -1096,24 +1102,13 @@ int paged_attn_decode_noalloc(const pkv_tensor* q, const pkv_tensor* k_cache,
   const bool fp8 = k_cache && k_cache->dtype == PKV_FP8_E4M3;
   DecodeArgs a{q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
                num_kv_heads, scale, block_size, out};
-  int ck = 0;
-  DecodeLaunch* e = nullptr;
-  int st = check_decode(a, fp8, &ck, &e);
-  if (st != PKV_OK || !e) return st;
-  int dev;
+  int dev, st;
   if ((st = current_device(&dev)) != PKV_OK) return st;
-  DeviceState* ds;
-  if ((st = device_state(dev, &ds)) != PKV_OK) return st;
-  int grid;
-  if ((st = decode_grid(e, dev, ds->sms, &grid)) != PKV_OK) return st;
-  const int g = static_cast<int>(q->shape[1] / num_kv_heads);
-  const size_t need =
-      ws_fit(ds->sms, grid * e->nc, g, static_cast<int>(q->shape[2]), PKV_NOALLOC_SCRATCH_BYTES)
-          .total;
-  if (need > PKV_NOALLOC_SCRATCH_BYTES) return PKV_ERR_SCRATCH_LIMIT;
   void* scratch = nullptr;
   if ((st = noalloc_scratch(dev, &scratch)) != PKV_OK) return st;
-  // The scratch keeps the previous call's contents: clear the claim state.
+  // launch_decode fits the layout to the array (fewer steal slots when the
+  // default does not fit; PKV_ERR_SCRATCH_LIMIT when nothing fits) and, the
+  // array keeping the previous call's contents, clears the claim state.
   return launch_decode(a, fp8, scratch, PKV_NOALLOC_SCRATCH_BYTES, false,
                        static_cast<cudaStream_t>(stream), true, true);
 }

@@ -14,6 +14,7 @@ constexpr int kErrBadBlock = 1;     // block id outside the pool
 constexpr int kErrBadLen = 2;       // context length < 0 or beyond the table row
 constexpr int kErrWaitTimeout = 4;  // a bounded mbarrier wait ran out
 constexpr int kErrBadSlot = 8;      // cache slot outside the pool
+constexpr int kErrBadCopy = 64;     // a block-copy pair overlapping another pair (not copied)
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -1,0 +1,30 @@
+"""The bench's packed step inputs (host side): one buffer holds every input of
+a step at 16-byte aligned offsets, and the views read back exactly what was
+packed (so one copy moves a whole step's inputs)."""
+import os
+import sys
+
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def test_step_buffers_round_trip_and_alignment():
+    g = torch.Generator().manual_seed(3)
+    parts = {"q": torch.randn(3, 5, 8, generator=g).to(torch.bfloat16),
+             "slots": torch.randint(-5, 1000, (3,), generator=g, dtype=torch.int64),
+             "tables": torch.randint(-1, 100, (3, 7), generator=g, dtype=torch.int32),
+             "lens": torch.randint(0, 90, (3,), generator=g, dtype=torch.int32),
+             "empty": torch.zeros((0, 2), dtype=torch.int32),
+             "codes": torch.randint(0, 256, (3, 2, 5), generator=g, dtype=torch.uint8)}
+    b = bench.StepBuffers(parts, "cpu", pin=False)
+    used = sum(x.numel() * x.element_size() for x in parts.values())
+    assert used <= b.nbytes < used + bench.StepBuffers.ALIGN * len(parts)
+    for k, x in parts.items():
+        v = b.d(k)
+        assert v.dtype == x.dtype and tuple(v.shape) == tuple(x.shape)
+        assert torch.equal(v, x), k
+        assert (v.data_ptr() - b.dev.data_ptr()) % bench.StepBuffers.ALIGN == 0, k

@@ -82,6 +82,24 @@ def test_copy_blocks_bit_exact(dtype):
     check_no_device_error()
 
 
+def test_copy_blocks_overlapping_pairs_refused():
+    # A pair whose destination another pair reads (or also writes), or whose
+    # source another pair writes, would make the result depend on the order
+    # of the copies: it is not copied and the call is flagged; the other
+    # pairs are copied bit for bit (as the oracle copies them).
+    gen = torch.Generator().manual_seed(9)
+    kc, vc = _pools(12, 4, 16, 64, torch.float16, gen)
+    k0, v0 = kc.clone(), vc.clone()
+    pairs = torch.tensor([[0, 2], [2, 1], [3, 4], [5, 5], [6, 7], [8, 7], [9, 10]], dtype=torch.int32)
+    P.copy_blocks(kc, vc, pairs.cuda())
+    assert P.device_error(torch.cuda.current_device()) == P.PKV_ERR_DEVICE_CHECK
+    ek, ev = copy_blocks(raw(k0), raw(v0), np.array([[3, 4], [5, 5], [9, 10]]))
+    assert np.array_equal(raw(kc), ek) and np.array_equal(raw(vc), ev)
+    for blk in (1, 2, 7):                  # chained (0 -> 2 -> 1) and shared destination (7): untouched
+        assert torch.equal(kc[blk], k0[blk]) and torch.equal(vc[blk], v0[blk])
+    check_no_device_error()
+
+
 def test_bad_slot_is_flagged_and_skipped():
     gen = torch.Generator().manual_seed(3)
     kc, vc = _pools(4, 2, 16, 64, torch.float16, gen)

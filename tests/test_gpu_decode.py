@@ -189,3 +189,61 @@ def test_one_workspace_shared_by_configurations():
             torch.cuda.synchronize()
             assert max_err(out, ref) <= TOL[s.cache_dtype], (rnd, s.name)
     check_no_device_error()
+
+
+def test_cut_unit_with_more_pieces_than_one_merge_pass():
+    # One (sequence, kv head) unit spread over the whole persistent grid: at
+    # D = 64 and 16-token blocks a B200 runs 2 CTAs of 4 warps per SM (1184
+    # warps), and 40000 tokens give every warp part of the unit, so the merge
+    # folds more pieces than its list holds (1024) in more than one pass.
+    for g, cd in ((1, "f16"), (8, "bf16")):
+        s = W.spec("tiny").replace(num_seqs=1, num_q_heads=g, num_kv_heads=1, cache_dtype=cd, q_dtype=cd,
+                                   lens=("fixed", [40000]), pool_blocks=None, table_width=None)
+        s, lay, t = decode_case(s)
+        out = run_decode(s, lay, t)
+        torch.cuda.synchronize()
+        check_no_device_error()
+        assert max_err(out, oracle_decode(s, lay, t)) <= TOL[cd], (g, cd)
+
+
+def test_fp8_bf16_q_rows_beyond_f16_range():
+    # bf16 q rows up to ~1e5 (past the f16 maximum 65504) on an fp8 cache: the
+    # row is scaled by a power of two before its f16 rounding, so the output
+    # stays finite and within tolerance; ordinary rows of the same batch are
+    # unaffected.
+    s, lay, t = decode_case(W.scaled_down(W.spec("long_skewed"), 8, 1500, cache_dtype="fp8_e4m3"))
+    q = t.q.float()
+    q[::2] *= 2.5e4                       # every other sequence: |q| up to about 1e5
+    q[1, 3] = 0.0
+    q[1, 3, 5] = -1.2e5                   # one element far past 65504, rest of that row 0
+    t.q.copy_(q.to(t.q.dtype))
+    assert t.q.float().abs().max() > 65504
+    out = run_decode(s, lay, t)
+    torch.cuda.synchronize()
+    check_no_device_error()
+    assert max_err(out, oracle_decode(s, lay, t)) <= TOL["fp8_e4m3"]
+
+
+@pytest.mark.parametrize("name", ["skewed_b16", "skewed_fp8_b16", "one_long", "d64_f16_b16_g1"])
+def test_deterministic_flag_gives_identical_bits(name):
+    s, lay, t = decode_case(SMALL[name], seed=SMALL[name].seed + 5)
+    code = {"bf16": P.PKV_BF16, "f16": P.PKV_F16, "fp8_e4m3": P.PKV_FP8_E4M3}[s.cache_dtype]
+    nbytes = P.workspace_bytes(s.num_q_heads, s.num_kv_heads, s.head_dim, s.block_size, code,
+                               torch.cuda.current_device())
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    tables, lens = lay.tables.cuda(), lay.lens.cuda()
+    outs = []
+    for _ in range(5):
+        out = torch.full_like(t.q, float("nan"))
+        P.paged_attn_decode_ex(t.q, t.k_cache, t.v_cache, tables, lens, s.num_kv_heads, s.scale, s.block_size,
+                               out, ws, t.k_scale, t.v_scale, flags=P.PKV_DECODE_DETERMINISTIC)
+        outs.append(out)
+    torch.cuda.synchronize()
+    check_no_device_error()
+    for o in outs[1:]:
+        assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16)), name
+    assert max_err(outs[0], oracle_decode(s, lay, t)) <= TOL[s.cache_dtype], name
+    with pytest.raises(P.PkvError) as e:
+        P.paged_attn_decode_ex(t.q, t.k_cache, t.v_cache, tables, lens, s.num_kv_heads, s.scale, s.block_size,
+                               outs[0], ws, t.k_scale, t.v_scale, flags=2)
+    assert e.value.status == P.PKV_ERR_INVALID_ARG
