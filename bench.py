@@ -293,7 +293,16 @@ def prefill_traffic(s: W.Spec, q_tokens: int, kernel: str):
 # CPU oracle timing (cpu_baseline leg and the reference arm)
 # ---------------------------------------------------------------------------
 
+def _host_cores() -> int:
+    """Cores this process may run on (the host's usable cores)."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        return os.cpu_count() or 1
+
+
 def _blas_threads() -> int:
+    """Threads the oracle's BLAS calls run on (the cores it actually uses)."""
     try:
         from threadpoolctl import threadpool_info
         n = [d["num_threads"] for d in threadpool_info() if d.get("user_api") == "blas"]
@@ -331,7 +340,8 @@ def cpu_baseline(s: W.Spec, host, budget_s: float) -> dict:
         tot_t += dt
         tot_b += nb
         done += 1
-    return {"value": tot_b / tot_t / 1e9, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+    return {"value": tot_b / tot_t / 1e9, "unit": UNIT, "cores": _blas_threads(), "host_cores": _host_cores(),
+            "kind": "oracle",
             "sample": f"fp64 numpy oracle, one sequence per call, cycling over the workload's {S} "
                       f"sequences: {done} sequence decodes ({tot_b} K/V bytes) in {tot_t:.1f} s",
             "seqs_per_s": done / tot_t}
@@ -408,8 +418,8 @@ def run_reference(a, s: W.Spec, ws: int, rank: int):
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * tot_t / max(1, a.steps),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": config_of(s, lay, kv_bytes_of(s, lay.lens.tolist())),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
-                         "sample": sample},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": _blas_threads(), "host_cores": _host_cores(),
+                         "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }))
 

@@ -56,11 +56,6 @@ constexpr int kMaxSteals = 6;     // steals from one warp's range per call
 constexpr int kMinStealable = 8;  // a remainder worth splitting (items)
 constexpr int kStealTries = 8;
 constexpr int kErrBadMerge = 16;  // a merge record out of range (skipped)
-// e4m3 terms of q against an fp8 K: two hold every bf16 value of a row
-// exactly (4 + 4 significant bits; elements 2^13 times below the row's
-// largest lose low bits), three every f16 value. 0: widen K to f16 instead.
-constexpr int kFp8QTermsBF16 = 2;
-constexpr int kFp8QTermsF16 = 3;
 
 struct DecodeParams {
   CUtensorMap tmk;  // K pool viewed as {D, B, Hk, NB}
@@ -200,10 +195,6 @@ struct DecodeCfg {
   static constexpr int KT = IB * TILE;            // K (or V) tiles of one item
   static constexpr int STAGE = 2 * KT;
   static constexpr int KS = D / 16;               // k-steps of the QK^T product
-  // fp8 caches: K goes to the tensor cores as e4m3 (m16n8k32) against q
-  // written as a sum of QT e4m3 terms (0: K widened to f16 instead).
-  static constexpr int QT = kFp8 ? (QBF ? kFp8QTermsBF16 : kFp8QTermsF16) : 0;
-  static constexpr int QREGS = QT > 0 ? QT * (KS / 2) : KS;  // q B-fragment register pairs
   static constexpr int MT = D / 16;               // m-tiles of the PV product
   static constexpr int TT = TOK / 16;             // 16-token tiles per item
   static constexpr int NT = NC * 32;
@@ -365,7 +356,7 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
   long long it = 0;      // items consumed by this warp (ring position)
   long long issued = 0;  // items issued into the ring
 
-  uint32_t qb[C::QREGS][2];
+  uint32_t qb[C::KS][2];
   float acc[C::MT][4];
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
   float sl0 = p.scale_log2, sl1 = p.scale_log2;  // logit scales of head columns 2c and 2c + 1
@@ -508,63 +499,29 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
             f[ks][2] = __low2float(b2);
             f[ks][3] = __high2float(b2);
           }
-          amax = fmaxf(amax, fmaxf(fmaxf(fabsf(f[ks][0]), fabsf(f[ks][1])),
-                                   fmaxf(fabsf(f[ks][2]), fabsf(f[ks][3]))));
+          if constexpr (QBF)
+            amax = fmaxf(amax, fmaxf(fmaxf(fabsf(f[ks][0]), fabsf(f[ks][1])),
+                                     fmaxf(fabsf(f[ks][2]), fabsf(f[ks][3]))));
         }
-        // largest magnitude of the row of head r (held by lanes 4r .. 4r + 3)
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-        const int ex = static_cast<int>((__float_as_uint(amax) >> 23) & 0xffu) - 127;
-        if constexpr (C::QT == 0) {
-          // q rounded to f16. A bf16 row may exceed the f16 range (2^16 and
-          // up): it is scaled by a power of two 2^-e (exact) and its logit
-          // scale by 2^e. Rows below 2^16 keep e = 0.
-          float qs = 1.f;
-          if constexpr (QBF) {
-            const int e = ex >= 16 ? ex - 15 : 0;
-            qs = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
-            const int e0 = __shfl_sync(0xffffffffu, e, 8 * c), e1 = __shfl_sync(0xffffffffu, e, 8 * c + 4);
-            sl0 = sl * __uint_as_float(static_cast<uint32_t>(127 + e0) << 23);
-            sl1 = sl * __uint_as_float(static_cast<uint32_t>(127 + e1) << 23);
-          }
+        // q rounded to f16. A bf16 row may exceed the f16 range (2^16 and
+        // up): it is scaled by a power of two 2^-e (exact) and its logit
+        // scale by 2^e. Rows below 2^16 keep e = 0. The row of head r is held
+        // by lanes 4r .. 4r + 3.
+        float qs = 1.f;
+        if constexpr (QBF) {
+          amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+          amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+          const int ex = static_cast<int>((__float_as_uint(amax) >> 23) & 0xffu) - 127;
+          const int e = ex >= 16 ? ex - 15 : 0;
+          qs = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+          const int e0 = __shfl_sync(0xffffffffu, e, 8 * c), e1 = __shfl_sync(0xffffffffu, e, 8 * c + 4);
+          sl0 = sl * __uint_as_float(static_cast<uint32_t>(127 + e0) << 23);
+          sl1 = sl * __uint_as_float(static_cast<uint32_t>(127 + e1) << 23);
+        }
 #pragma unroll
-          for (int ks = 0; ks < C::KS; ++ks) {
-            qb[ks][0] = pack2<false>(f[ks][0] * qs, f[ks][1] * qs);
-            qb[ks][1] = pack2<false>(f[ks][2] * qs, f[ks][3] * qs);
-          }
-        } else {
-          // q row scaled by 2^sh (exact) into [128, 256) at its largest
-          // element, then written as e4m3 terms: t0 = e4m3(x), t1 =
-          // e4m3(x - t0), ... (each rounding to nearest even; the residual
-          // shrinks 16-fold per term). The logit scale takes 2^-sh back.
-          // B fragment of k-step kp (32 dims): [0] = dims 32kp + 4c .. +3,
-          // [1] = dims 32kp + 16 + 4c .. +3, one byte each, first dim lowest.
-          // zero or non-finite rows: no shift; tiny rows: at most 2^127
-          const int sh = (amax > 0.f && ex < 128) ? min(7 - ex, 127) : 0;
-          const float up = __uint_as_float(static_cast<uint32_t>(127 + sh) << 23);
-          const int sh0 = __shfl_sync(0xffffffffu, sh, 8 * c), sh1 = __shfl_sync(0xffffffffu, sh, 8 * c + 4);
-          sl0 = sl * __uint_as_float(static_cast<uint32_t>(127 - sh0) << 23);
-          sl1 = sl * __uint_as_float(static_cast<uint32_t>(127 - sh1) << 23);
-#pragma unroll
-          for (int ks = 0; ks < C::KS; ++ks) {
-            float x[4] = {f[ks][0] * up, f[ks][1] * up, f[ks][2] * up, f[ks][3] * up};
-#pragma unroll
-            for (int qt = 0; qt < C::QT; ++qt) {
-              const uint32_t lo2 = __nv_cvt_float2_to_fp8x2(make_float2(x[0], x[1]), __NV_NOSAT, __NV_E4M3);
-              const uint32_t hi2 = __nv_cvt_float2_to_fp8x2(make_float2(x[2], x[3]), __NV_NOSAT, __NV_E4M3);
-              qb[qt * (C::KS / 2) + ks / 2][ks & 1] = lo2 | (hi2 << 16);
-              if (qt + 1 < C::QT) {  // residual for the next term
-                uint32_t w01 = e4m3x2_to_f16x2(static_cast<uint16_t>(lo2));
-                uint32_t w23 = e4m3x2_to_f16x2(static_cast<uint16_t>(hi2));
-                const __half2 d01 = *reinterpret_cast<__half2*>(&w01);
-                const __half2 d23 = *reinterpret_cast<__half2*>(&w23);
-                x[0] -= __low2float(d01);
-                x[1] -= __high2float(d01);
-                x[2] -= __low2float(d23);
-                x[3] -= __high2float(d23);
-              }
-            }
-          }
+        for (int ks = 0; ks < C::KS; ++ks) {
+          qb[ks][0] = pack2<false>(f[ks][0] * qs, f[ks][1] * qs);
+          qb[ks][1] = pack2<false>(f[ks][2] * qs, f[ks][3] * qs);
         }
       }
     };
@@ -715,18 +672,6 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
               uint32_t a0, a1, a2, a3;
               ldsm_x4(kt + swz<BS>(trow, ks * 32 + (lane >> 4) * 16), a0, a1, a2, a3);
               mma16816<MBF>(sacc[tt], a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
-            }
-          } else if constexpr (C::QT > 0) {
-            // the K tile's bytes are the e4m3 A fragment of m16n8k32 as
-            // ldmatrix leaves them: rows r / r + 8, bytes 4c .. 4c + 3 / + 16
-#pragma unroll
-            for (int kp = 0; kp < C::KS / 2; ++kp) {
-              uint32_t x0, x1, x2, x3;
-              ldsm_x4(kt + swz<BS>(trow, kp * 32 + (lane >> 4) * 16), x0, x1, x2, x3);
-#pragma unroll
-              for (int qt = 0; qt < C::QT; ++qt)
-                mma16832_e4m3(sacc[tt], x0, x1, x2, x3, qb[qt * (C::KS / 2) + kp][0],
-                              qb[qt * (C::KS / 2) + kp][1]);
             }
           } else {
 #pragma unroll

@@ -118,18 +118,6 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
   }
 }
 
-// D(16x8 f32) += A(16x32 e4m3) * B(32x8 e4m3). A: rows r / r + 8 (a0, a2 /
-// a1, a3), bytes 4c .. 4c + 3 (a0, a1) and 16 + 4c .. (a2, a3); B: rows
-// 4c .. 4c + 3 (b0) and 16 + 4c .. (b1) of column r; r = lane / 4, c = lane % 4.
-__device__ __forceinline__ void mma16832_e4m3(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                              uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0, %1, %2, %3}, "
-      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
 // ---- conversions ---------------------------------------------------------------
 // Two e4m3 codes (low byte = first element) to an f16x2 (exact: every e4m3
 // value is an f16 value).
