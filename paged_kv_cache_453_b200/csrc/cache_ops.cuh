@@ -41,9 +41,15 @@ struct CacheParams {
   int in_bytes;  // bytes of one input row of k / v
 };
 
+// The cache writes and block copies are launched as programmatic dependents
+// of the kernel before them: they may be resident before it ends, and wait
+// for it (griddepcontrol.wait) before touching memory; then they let the
+// kernel after them (a decode) start its prologue.
+
 // 16-bit pools: a plain 16-byte copy per thread.
 __global__ void reshape_and_cache_kernel(const __grid_constant__ CacheParams p, int* err) {
-  pdl_launch_dependents();  // a decode launched after this may start its prologue
+  pdl_wait();
+  pdl_launch_dependents();
   const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const long long per_tok = static_cast<long long>(p.Hk) * p.row_vecs;
   if (i >= per_tok * p.T) return;
@@ -112,6 +118,7 @@ __device__ __forceinline__ uint4 quantise16(const int4& a, const int4& b, float 
 
 template <bool BF16>
 __global__ void reshape_and_cache_fp8_kernel(const __grid_constant__ CacheParams p, int* err) {
+  pdl_wait();
   pdl_launch_dependents();
   const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const long long per_tok = static_cast<long long>(p.Hk) * p.row_vecs;
@@ -154,6 +161,8 @@ struct CopyParams {
 // whose source is another pair's destination, is not copied and is flagged
 // (the other pairs are still copied).
 __global__ void copy_blocks_kernel(const __grid_constant__ CopyParams p, int* err) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int pi = blockIdx.x;
   const int src = p.pairs[pi * p.pr_s], dst = p.pairs[pi * p.pr_s + 1];
   if (src < 0 || src >= p.NB || dst < 0 || dst >= p.NB) {

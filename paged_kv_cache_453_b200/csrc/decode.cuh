@@ -53,8 +53,10 @@ namespace pkv {
 enum CacheKind : int { kCacheF16 = 0, kCacheBF16 = 1, kCacheE4M3 = 2 };
 
 constexpr int kMaxSteals = 6;     // steals from one warp's range per call
-constexpr int kMinStealable = 8;  // a remainder worth splitting (items)
+constexpr int kMinStealable = 4;  // a remainder worth splitting (items)
 constexpr int kStealTries = 8;
+constexpr int kScanBatch = 16;    // range words each lane loads at once when choosing a victim
+constexpr int kMergeAhead = 8;    // ranges whose steal records the merge reads in its first round
 constexpr int kErrBadMerge = 16;  // a merge record out of range (skipped)
 
 struct DecodeParams {
@@ -678,12 +680,13 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
             for (int kp = 0; kp < C::KS / 2; ++kp) {
               uint32_t x0, x1, x2, x3;
               ldsm_x4(kt + swz<BS>(trow, kp * 32 + (lane >> 4) * 16), x0, x1, x2, x3);
-              mma16816<false>(sacc[tt], e4m3x2_to_f16x2(x0 & 0xffff),
-                              e4m3x2_to_f16x2(x1 & 0xffff), e4m3x2_to_f16x2(x0 >> 16),
-                              e4m3x2_to_f16x2(x1 >> 16), qb[2 * kp][0], qb[2 * kp][1]);
-              mma16816<false>(sacc[tt], e4m3x2_to_f16x2(x2 & 0xffff),
-                              e4m3x2_to_f16x2(x3 & 0xffff), e4m3x2_to_f16x2(x2 >> 16),
-                              e4m3x2_to_f16x2(x3 >> 16), qb[2 * kp + 1][0], qb[2 * kp + 1][1]);
+              uint32_t a0, a2, a1, a3, b0, b2, b1, b3;
+              e4m3x4_to_f16x2x2(x0, a0, a2);
+              e4m3x4_to_f16x2x2(x1, a1, a3);
+              e4m3x4_to_f16x2x2(x2, b0, b2);
+              e4m3x4_to_f16x2x2(x3, b1, b3);
+              mma16816<false>(sacc[tt], a0, a1, a2, a3, qb[2 * kp][0], qb[2 * kp][1]);
+              mma16816<false>(sacc[tt], b0, b1, b2, b3, qb[2 * kp + 1][0], qb[2 * kp + 1][1]);
             }
           }
         }
@@ -704,25 +707,33 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
             const int vrow = (tt * 16) % BS + (lane & 7) + ((lane >> 4) & 1) * 8;
             ldsm_x4_t(tv + ((tt * 16) / BS) * C::TILE + swz<BS>(vrow, i * 32 + ((lane >> 3) & 1) * 16),
                       f[0], f[1], f[2], f[3]);
-            f[0] &= keep01;
-            f[1] &= keep01;
-            f[2] &= keep23;
-            f[3] &= keep23;
+            if constexpr (kMask) {
+              f[0] &= keep01;
+              f[1] &= keep01;
+              f[2] &= keep23;
+              f[3] &= keep23;
+            }
           } else {
             const int vrow = (tt * 16) % BS + (lane & 7) + ((lane >> 3) & 1) * 8;
             uint32_t x0, x1, x2, x3;
             ldsm_x4_t(tv + ((tt * 16) / BS) * C::TILE + swz<BS>(vrow, i * 32 + (lane >> 4) * 16), x0,
                       x1, x2, x3);
-            const uint32_t e0 = prmt(x0, 0, 0x3120), e1 = prmt(x1, 0, 0x3120);
-            const uint32_t e2 = prmt(x2, 0, 0x3120), e3 = prmt(x3, 0, 0x3120);
-            f[0] = e4m3x2_to_f16x2(e0 & 0xffff) & keep01;
-            f[1] = e4m3x2_to_f16x2(e0 >> 16) & keep01;
-            f[2] = e4m3x2_to_f16x2(e1 & 0xffff) & keep23;
-            f[3] = e4m3x2_to_f16x2(e1 >> 16) & keep23;
-            f[4] = e4m3x2_to_f16x2(e2 & 0xffff) & keep01;
-            f[5] = e4m3x2_to_f16x2(e2 >> 16) & keep01;
-            f[6] = e4m3x2_to_f16x2(e3 & 0xffff) & keep23;
-            f[7] = e4m3x2_to_f16x2(e3 >> 16) & keep23;
+            // bytes (d, t), (d + 1, t), (d, t + 1), (d + 1, t + 1) -> token
+            // pairs (d, t | t + 1) and (d + 1, t | t + 1)
+            e4m3x4_to_f16x2x2(prmt(x0, 0, 0x3120), f[0], f[1]);
+            e4m3x4_to_f16x2x2(prmt(x1, 0, 0x3120), f[2], f[3]);
+            e4m3x4_to_f16x2x2(prmt(x2, 0, 0x3120), f[4], f[5]);
+            e4m3x4_to_f16x2x2(prmt(x3, 0, 0x3120), f[6], f[7]);
+            if constexpr (kMask) {
+              f[0] &= keep01;
+              f[1] &= keep01;
+              f[2] &= keep23;
+              f[3] &= keep23;
+              f[4] &= keep01;
+              f[5] &= keep01;
+              f[6] &= keep23;
+              f[7] &= keep23;
+            }
           }
         };
         if constexpr (kEarly) {
@@ -820,30 +831,51 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
   if (!p.steal) return;  // static split: every unit is cut at the same places in every call
 
   const long long nominal = W / p.nwt;  // every static range is nominal or nominal + 1 long
+  // Two partial slots from the pool per steal, reserved only once a victim
+  // is in sight and kept across failed attempts (a reservation made for
+  // nothing would use up the pool: every warp ends with a failed search).
+  unsigned slot0 = 0;
+  bool have_slots = false;
   for (int attempt = 0; attempt < 4 * kStealTries; ++attempt) {
-    // reserve two partial slots from the pool
-    unsigned slot0 = 0;
-    if (lane == 0) slot0 = atomicAdd(p.pool, 2u);
-    slot0 = __shfl_sync(0xffffffffu, slot0, 0);
-    if (slot0 + 2 > static_cast<unsigned>(p.pool_slots)) break;
-
     // find the victim with the largest unclaimed remainder, steal its back half
     int stolen = 0;
+    bool pool_empty = false;
     long long sa = 0, sb = 0;
     int victim = -1, sj = 0;
     for (int tries = 0; tries < kStealTries && !stolen; ++tries) {
       long long best = 0;
       int bv = -1;
       unsigned long long bw = 0;
-      for (int v = lane; v < p.nwt; v += 32) {
-        const unsigned long long w = ld_relaxed(p.words + v);
-        const long long rem = rw_steals(w) >= kMaxSteals
-                                  ? 0
-                                  : nominal - static_cast<long long>(rw_front(w)) - rw_back(w);
-        if (rem > best) {
-          best = rem;
-          bv = v;
-          bw = w;
+      // range words 16 per lane at a time: every load of a batch is issued
+      // before the first is used (one round trip per batch, not per word)
+      for (int v0 = lane; v0 < p.nwt; v0 += 32 * kScanBatch) {
+        unsigned long long wb[kScanBatch];
+#pragma unroll
+        for (int j = 0; j < kScanBatch; ++j)
+          wb[j] = v0 + 32 * j < p.nwt ? ld_relaxed(p.words + v0 + 32 * j) : 0ull;
+#pragma unroll
+        for (int j = 0; j < kScanBatch; ++j) {
+          const unsigned long long w = wb[j];
+          const int v = v0 + 32 * j;
+          long long rem = (v >= p.nwt || rw_steals(w) >= kMaxSteals)
+                              ? 0
+                              : nominal - static_cast<long long>(rw_front(w)) - rw_back(w);
+          // Thieves that finish together would all pick the same largest
+          // remainder and collide on one word: each scores a victim at its
+          // remainder plus up to a quarter of it, by a hash of (thief,
+          // victim), so they spread over the victims near the largest.
+          if (rem >= kMinStealable) {
+            const unsigned hsh = (static_cast<unsigned>(v) * 2654435761u) ^
+                                 (static_cast<unsigned>(gw + 1) * 2246822519u);
+            rem = rem * 4 + ((rem * static_cast<long long>((hsh >> 24) & 0xffu)) >> 8);
+          } else {
+            rem = 0;
+          }
+          if (rem > best) {
+            best = rem;
+            bv = v;
+            bw = w;
+          }
         }
       }
 #pragma unroll
@@ -857,16 +889,31 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
           bw = ow;
         }
       }
-      if (best < kMinStealable) break;
+      if (best < 4 * kMinStealable) break;  // (scores are 4x the remainder or more)
+      if (!have_slots) {
+        if (lane == 0) slot0 = atomicAdd(p.pool, 2u);
+        slot0 = __shfl_sync(0xffffffffu, slot0, 0);
+        if (slot0 + 2 > static_cast<unsigned>(p.pool_slots)) {
+          pool_empty = true;
+          break;
+        }
+        have_slots = true;
+      }
       if (lane == 0) {
+        // The owner claims an item every microsecond or so, so the word read
+        // by the scan is usually stale by now: a failed CAS returns the
+        // current word, which the next attempt takes as its expectation.
         const long long vlo = range_lo(bv, W, p.nwt);
         const long long vlen = range_lo(bv + 1, W, p.nwt) - vlo;
-        const unsigned f = rw_front(bw), b = rw_back(bw), ns = rw_steals(bw);
-        const long long rem = vlen - static_cast<long long>(f) - b;
-        if (rem >= kMinStealable && ns < kMaxSteals) {
+        unsigned long long cur = bw;
+        for (int c = 0; c < kStealTries; ++c) {
+          const unsigned f = rw_front(cur), b = rw_back(cur), ns = rw_steals(cur);
+          const long long rem = vlen - static_cast<long long>(f) - b;
+          if (rem < kMinStealable || ns >= kMaxSteals) break;
           const unsigned take = static_cast<unsigned>(rem / 2);
           const unsigned long long want = rw_make(f, b + take, ns + 1);
-          if (atomicCAS(p.words + bv, bw, want) == bw) {
+          const unsigned long long prev = atomicCAS(p.words + bv, cur, want);
+          if (prev == cur) {
             stolen = 1;
             sb = vlo + vlen - b;
             sa = sb - take;
@@ -875,12 +922,15 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
             p.steal_info[bv * kMaxSteals + sj] =
                 make_int4(static_cast<int>(sa & 0xffffffffll), 2 * p.nwt + static_cast<int>(slot0),
                           p.tag, static_cast<int>(sa >> 32));
+            break;
           }
+          cur = prev;
         }
       }
       stolen = __shfl_sync(0xffffffffu, stolen, 0);
     }
-    if (!stolen) break;
+    if (!stolen || pool_empty) break;
+    have_slots = false;  // this steal's partials use them
     sa = __shfl_sync(0xffffffffu, sa, 0);
     sb = __shfl_sync(0xffffffffu, sb, 0);
     victim = __shfl_sync(0xffffffffu, victim, 0);
@@ -914,7 +964,7 @@ __global__ void __launch_bounds__(128, 8) decode_merge_kernel(const __grid_const
   __shared__ float s_red[NT * 10];
   __shared__ int s_wsum[NT / 32];
   __shared__ int4 s_desc[ND];
-  __shared__ int4 s_rec[kMaxSteals];
+  __shared__ int4 s_rec[kMergeAhead][kMaxSteals];  // steal records of ranges w0 .. w0 + kMergeAhead - 1
   __shared__ long long s_own_start[kMaxSteals];
   __shared__ int s_own_slot[kMaxSteals];
   __shared__ long long s_W;
@@ -926,11 +976,15 @@ __global__ void __launch_bounds__(128, 8) decode_merge_kernel(const __grid_const
   const int g = p.g;
   const int E = g * D;
 
-  // round 1: descriptors, own steal records, item count
+  // round 1: descriptors, the steal records of this range and the next
+  // few (a cut unit rarely reaches further), item count
   if (tid < ND) s_desc[tid] = p.desc[w0 * ND + tid];
-  else if (tid >= 32 && tid < 32 + kMaxSteals) s_rec[tid - 32] = p.steal_info[w0 * kMaxSteals + tid - 32];
-  else if (tid == 64) s_W = p.hdr[0];
-  else if (tid == 96) {
+  else if (tid >= 32 && tid < 32 + kMergeAhead * kMaxSteals) {
+    const int j = tid - 32, v = w0 + j / kMaxSteals;
+    if (v < p.nwt) s_rec[j / kMaxSteals][j % kMaxSteals] = p.steal_info[v * kMaxSteals + j % kMaxSteals];
+  } else if (tid == 32 + kMergeAhead * kMaxSteals) {
+    s_W = p.hdr[0];
+  } else if (tid == 33 + kMergeAhead * kMaxSteals) {
     p.words[w0] = 0ull;  // leave the claim state zeroed for the next call
     if (w0 == 0) *p.pool = 0u;
   }
@@ -958,7 +1012,7 @@ __global__ void __launch_bounds__(128, 8) decode_merge_kernel(const __grid_const
     return m;
   };
 
-  if (tid == 0) s_m_own = valid_steals(w0, s_rec, s_own_start, s_own_slot);
+  if (tid == 0) s_m_own = valid_steals(w0, s_rec[0], s_own_start, s_own_slot);
   __syncthreads();
   const int m_own = s_m_own;
 
@@ -975,6 +1029,8 @@ __global__ void __launch_bounds__(128, 8) decode_merge_kernel(const __grid_const
         st_v[j] = s_own_start[j];
         sl_v[j] = s_own_slot[j];
       }
+    } else if (v < w0 + kMergeAhead) {
+      m = valid_steals(v, s_rec[v - w0], st_v, sl_v);
     } else {
       int4 rec[kMaxSteals];
 #pragma unroll

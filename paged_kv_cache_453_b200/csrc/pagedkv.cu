@@ -228,6 +228,24 @@ int decode_grid(DecodeLaunch* e, int dev, int sms, int* grid) {
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Launch as a programmatic dependent of the kernel before it in the stream
+// (the kernel waits for it with griddepcontrol.wait before touching memory).
+template <typename P>
+int launch_dependent(void (*kern)(P, int*), dim3 grid, dim3 block, cudaStream_t stream, const P& p,
+                     int* err) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, p, err) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
 // Decode workspace: header (total items, steal-slot pool counter), range
 // words, steal records, last-piece descriptors, and fp32 partial slots (two
 // per warp for its own range, `pool` more for steals). The range words and
@@ -263,9 +281,9 @@ WsLayout ws_layout(int sms, int nwt, int g, int D, int pool_slots) {
   return l;
 }
 
-// Default: room for one steal per warp.
+// Default: room for two steals per warp on average.
 WsLayout ws_default(int sms, int nwt, int g, int D) {
-  return ws_layout(sms, nwt, g, D, 2 * nwt);
+  return ws_layout(sms, nwt, g, D, 4 * nwt);
 }
 
 // The largest layout that fits in `bytes` (fewer steal slots), or one whose
@@ -963,12 +981,10 @@ int launch_reshape(const pkv_tensor* k, const pkv_tensor* v, pkv_tensor* kc, pkv
   const int tpb = 128;
   const long long blocks = (threads + tpb - 1) / tpb;
   if (blocks > INT32_MAX) return PKV_ERR_UNSUPPORTED;
-  if (!fp8) reshape_and_cache_kernel<<<static_cast<int>(blocks), tpb, 0, stream>>>(p, ds->err);
-  else if (xdt == PKV_BF16)
-    reshape_and_cache_fp8_kernel<true><<<static_cast<int>(blocks), tpb, 0, stream>>>(p, ds->err);
-  else
-    reshape_and_cache_fp8_kernel<false><<<static_cast<int>(blocks), tpb, 0, stream>>>(p, ds->err);
-  return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+  void (*kern)(CacheParams, int*) = !fp8                ? reshape_and_cache_kernel
+                                    : xdt == PKV_BF16 ? reshape_and_cache_fp8_kernel<true>
+                                                      : reshape_and_cache_fp8_kernel<false>;
+  return launch_dependent(kern, dim3(static_cast<unsigned>(blocks)), dim3(tpb), stream, p, ds->err);
 }
 
 }  // namespace
@@ -1164,8 +1180,7 @@ int copy_blocks(pkv_tensor* k_cache, pkv_tensor* v_cache, const pkv_tensor* pair
   int chunks = (total + tpb - 1) / tpb;
   if (chunks > 65535) chunks = 65535;
   dim3 grid(static_cast<unsigned>(n), static_cast<unsigned>(chunks));
-  copy_blocks_kernel<<<grid, tpb, 0, static_cast<cudaStream_t>(stream)>>>(p, ds->err);
-  return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+  return launch_dependent(copy_blocks_kernel, grid, dim3(tpb), static_cast<cudaStream_t>(stream), p, ds->err);
 }
 
 int paged_attn_prefill(const pkv_tensor* q, const pkv_tensor* k_cache, const pkv_tensor* v_cache,

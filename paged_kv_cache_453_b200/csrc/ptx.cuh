@@ -119,12 +119,16 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
 }
 
 // ---- conversions ---------------------------------------------------------------
-// Two e4m3 codes (low byte = first element) to an f16x2 (exact: every e4m3
-// value is an f16 value).
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t v) {
-  uint32_t d;
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(d) : "h"(v));
-  return d;
+// Four e4m3 codes (bytes 0..3) to two f16x2 (exact: every e4m3 value is an
+// f16 value): lo = (byte 0, byte 1), hi = (byte 2, byte 3), the lower byte
+// the first element; the register's halves feed the conversions directly.
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t v, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 l, h;\n\t"
+      "mov.b32 {l, h}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, l;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(v));
 }
 template <bool BF16>
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
