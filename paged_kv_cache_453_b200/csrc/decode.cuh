@@ -55,7 +55,7 @@ enum CacheKind : int { kCacheF16 = 0, kCacheBF16 = 1, kCacheE4M3 = 2 };
 constexpr int kMaxSteals = 6;     // steals from one warp's range per call
 constexpr int kMinStealable = 4;  // a remainder worth splitting (items)
 constexpr int kStealTries = 8;
-constexpr int kScanBatch = 16;    // range words each lane loads at once when choosing a victim
+constexpr int kScanBatch = 4;     // range words each lane loads when choosing a victim (a window of 128)
 constexpr int kMergeAhead = 8;    // ranges whose steal records the merge reads in its first round
 constexpr int kErrBadMerge = 16;  // a merge record out of range (skipped)
 
@@ -843,21 +843,29 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
     long long sa = 0, sb = 0;
     int victim = -1, sj = 0;
     for (int tries = 0; tries < kStealTries && !stolen; ++tries) {
+      const int win0 = static_cast<int>(
+          ((static_cast<unsigned>(gw) * 2654435761u) >> 7) +
+          static_cast<unsigned>((attempt * kStealTries + tries) * 32 * kScanBatch)) % p.nwt;
       long long best = 0;
       int bv = -1;
       unsigned long long bw = 0;
-      // range words 16 per lane at a time: every load of a batch is issued
-      // before the first is used (one round trip per batch, not per word)
-      for (int v0 = lane; v0 < p.nwt; v0 += 32 * kScanBatch) {
+      // A window of 32 x kScanBatch range words, from an offset that differs
+      // per thief and per try: every load is issued before the first is used
+      // (one round trip), and a window without a candidate ends the search,
+      // so a warp with nothing to steal leaves after one round trip.
+      {
         unsigned long long wb[kScanBatch];
 #pragma unroll
-        for (int j = 0; j < kScanBatch; ++j)
-          wb[j] = v0 + 32 * j < p.nwt ? ld_relaxed(p.words + v0 + 32 * j) : 0ull;
+        for (int j = 0; j < kScanBatch; ++j) {
+          const int off = lane + 32 * j;
+          wb[j] = off < p.nwt ? ld_relaxed(p.words + (win0 + off) % p.nwt) : 0ull;
+        }
 #pragma unroll
         for (int j = 0; j < kScanBatch; ++j) {
           const unsigned long long w = wb[j];
-          const int v = v0 + 32 * j;
-          long long rem = (v >= p.nwt || rw_steals(w) >= kMaxSteals)
+          const int off = lane + 32 * j;
+          const int v = (win0 + off) % p.nwt;
+          long long rem = (off >= p.nwt || rw_steals(w) >= kMaxSteals)
                               ? 0
                               : nominal - static_cast<long long>(rw_front(w)) - rw_back(w);
           // Thieves that finish together would all pick the same largest
@@ -969,15 +977,45 @@ __global__ void __launch_bounds__(128, 8) decode_merge_kernel(const __grid_const
   __shared__ int s_own_slot[kMaxSteals];
   __shared__ long long s_W;
   __shared__ int s_m_own;
+  constexpr int kSpec = 3;  // pieces loaded speculatively in the first round
+  __shared__ float2 s_sp_ml[kSpec][NT];
+  __shared__ float4 s_sp_o[kSpec][NT][2];
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int w0 = blockIdx.x;
   const int g = p.g;
   const int E = g * D;
+  // Thread t owns an 8-element chunk of one head (chunk t % NC8) and the
+  // pieces q = t / NC8 (mod PG) of each pass.
+  const int NC8 = E / 8;                // chunks of 8 elements (D is a multiple of 8)
+  const int PG = NT / NC8;              // piece groups (1 at g = 8, D = 128)
+  const int c8 = tid % NC8, pg = tid / NC8;
+  const int hi8 = c8 / (D / 8), d8 = (c8 % (D / 8)) * 8;
 
   // round 1: descriptors, the steal records of this range and the next
-  // few (a cut unit rarely reaches further), item count
+  // few (a cut unit rarely reaches further), item count; and, speculatively,
+  // the partials of the usual shape of the own part's last cut unit: cut
+  // only where the next static ranges begin, its pieces are slots
+  // 2 w0 + 1, 2 (w0 + 1), 2 (w0 + 2) (piece group 0 holds them).
+  if (pg == 0) {
+#pragma unroll
+    for (int u = 0; u < kSpec; ++u) {
+      const int slot = u == 0 ? 2 * w0 + 1 : 2 * (w0 + u);
+      float2 ml = make_float2(-INFINITY, 0.f);
+      float4 o0 = make_float4(0.f, 0.f, 0.f, 0.f), o1 = o0;
+      if (slot < 2 * p.nwt) {
+        const long long base = static_cast<long long>(slot) * g + hi8;
+        ml = make_float2(p.part_ml[base * 2], p.part_ml[base * 2 + 1]);
+        const float4* op = reinterpret_cast<const float4*>(p.part_o + base * D + d8);
+        o0 = op[0];
+        o1 = op[1];
+      }
+      s_sp_ml[u][c8] = ml;
+      s_sp_o[u][c8][0] = o0;
+      s_sp_o[u][c8][1] = o1;
+    }
+  }
   if (tid < ND) s_desc[tid] = p.desc[w0 * ND + tid];
   else if (tid >= 32 && tid < 32 + kMergeAhead * kMaxSteals) {
     const int j = tid - 32, v = w0 + j / kMaxSteals;
@@ -1063,14 +1101,9 @@ __global__ void __launch_bounds__(128, 8) decode_merge_kernel(const __grid_const
     const int pos0 = (k == 0) ? 0 : m_own - (k - 1);
     const int first = ((k == 0) ? 2 * w0 : s_own_slot[k - 1]) + 1;  // the unit's first piece
 
-    // Thread t owns an 8-element chunk of one head (chunk t % NC8) and the
-    // pieces q = t / NC8 (mod PG) of each pass; it loads four pieces at a
-    // time (m, l and two float4 of O each) before folding them with an
-    // online max / rescale, then the piece groups are combined.
-    const int NC8 = E / 8;                // chunks of 8 elements (D is a multiple of 8)
-    const int PG = NT / NC8;              // piece groups (1 at g = 8, D = 128)
-    const int c8 = tid % NC8, pg = tid / NC8;
-    const int hi8 = c8 / (D / 8), d8 = (c8 % (D / 8)) * 8;
+    // Each thread loads four of its pieces at a time (m, l and two float4
+    // of O each) before folding them with an online max / rescale, then the
+    // piece groups are combined.
     float rm = -INFINITY, rl = 0.f, ra[8];
 #pragma unroll
     for (int x = 0; x < 8; ++x) ra[x] = 0.f;
@@ -1108,8 +1141,33 @@ __global__ void __launch_bounds__(128, 8) decode_merge_kernel(const __grid_const
         if (next >= p.nwt || range_lo(next, W, p.nwt) >= U1) break;
       }
       const int n = min(run - wlo, kCap);
+      // the speculatively loaded pieces are this unit's, in this order
+      bool spec = k == 0 && pass == 0 && run <= kSpec;
+      for (int u = 1; u < kSpec && spec; ++u)
+        spec = u >= run || s_slot[u] == 2 * (w0 + u);
       // rounds 3 and 4: fold this pass's pieces in
-      if (pg < PG) {
+      if (spec) {
+        if (pg == 0) {
+#pragma unroll
+          for (int u = 0; u < kSpec; ++u) {
+            const float2 ml = s_sp_ml[u][c8];
+            if (u >= n || ml.x == -INFINITY) continue;
+            const float4 o0 = s_sp_o[u][c8][0], o1 = s_sp_o[u][c8][1];
+            const float mn = fmaxf(rm, ml.x);
+            const float sa = (rm == -INFINITY) ? 0.f : exp2f(rm - mn), sb = exp2f(ml.x - mn);
+            rl = rl * sa + ml.y * sb;
+            ra[0] = ra[0] * sa + o0.x * sb;
+            ra[1] = ra[1] * sa + o0.y * sb;
+            ra[2] = ra[2] * sa + o0.z * sb;
+            ra[3] = ra[3] * sa + o0.w * sb;
+            ra[4] = ra[4] * sa + o1.x * sb;
+            ra[5] = ra[5] * sa + o1.y * sb;
+            ra[6] = ra[6] * sa + o1.z * sb;
+            ra[7] = ra[7] * sa + o1.w * sb;
+            rm = mn;
+          }
+        }
+      } else if (pg < PG) {
         for (int q0 = pg; q0 < n; q0 += 4 * PG) {
           float mv[4], lv[4];
           float4 o0[4], o1[4];
