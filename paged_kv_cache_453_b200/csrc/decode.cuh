@@ -83,6 +83,7 @@ struct DecodeParams {
   unsigned* pool;             // steal-slot pool counter; 0 between calls
   int4* steal_info;           // [nwt][kMaxSteals] (start lo, slot base, tag, start hi)
   int4* desc;                 // [nwt][1 + kMaxSteals] last-piece descriptor per sub-range
+  long long* rlo;             // [nwt + 1] first item of each static warp range (the last: W)
   float* part_o;              // [2 nwt + pool_slots][g][D]
   float* part_ml;             // [2 nwt + pool_slots][g][2]
   // Prefix-aware decode (null otherwise): the first skip[s] table entries of
@@ -301,7 +302,11 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
     return;
   }
 
-  if (lane == 0) p.desc[gw * (1 + kMaxSteals)] = make_int4(-1, 0, 0, 0);
+  if (lane == 0) {
+    p.desc[gw * (1 + kMaxSteals)] = make_int4(-1, 0, 0, 0);
+    p.rlo[gw] = my_lo;  // the merge reads the range boundaries instead of dividing
+    if (gw == p.nwt - 1) p.rlo[p.nwt] = W;
+  }
 
   // Position of global item x: chunk by binary search, then a warp-wide walk.
   auto locate = [&](long long x, Cursor<BS, TOK>& out) -> bool {
@@ -977,6 +982,7 @@ __global__ void __launch_bounds__(128, 8) decode_merge_kernel(const __grid_const
   __shared__ int s_own_slot[kMaxSteals];
   __shared__ long long s_W;
   __shared__ int s_m_own;
+  __shared__ long long s_rlo[NT + 1];  // first items of ranges w0 .. w0 + NT
   constexpr int kSpec = 3;  // pieces loaded speculatively in the first round
   __shared__ float2 s_sp_ml[kSpec][NT];
   __shared__ float4 s_sp_o[kSpec][NT][2];
@@ -1016,6 +1022,8 @@ __global__ void __launch_bounds__(128, 8) decode_merge_kernel(const __grid_const
       s_sp_o[u][c8][1] = o1;
     }
   }
+  if (w0 + tid <= p.nwt) s_rlo[tid] = p.rlo[w0 + tid];
+  if (tid == 0 && w0 + NT <= p.nwt) s_rlo[NT] = p.rlo[w0 + NT];
   if (tid < ND) s_desc[tid] = p.desc[w0 * ND + tid];
   else if (tid >= 32 && tid < 32 + kMergeAhead * kMaxSteals) {
     const int j = tid - 32, v = w0 + j / kMaxSteals;
@@ -1028,11 +1036,13 @@ __global__ void __launch_bounds__(128, 8) decode_merge_kernel(const __grid_const
   }
   __syncthreads();
   const long long W = s_W;
+  // first item of static range v (v <= nwt)
+  auto rlo = [&](int v) -> long long { return v - w0 <= NT ? s_rlo[v - w0] : p.rlo[v]; };
 
   // Steal records j = 0, 1, ... of warp v's range that carry this call's tag,
   // each starting inside v's range with its slots in the pool.
   auto valid_steals = [&](int v, const int4* rec, long long* starts, int* slots) -> int {
-    const long long vlo = range_lo(v, W, p.nwt), vhi = range_lo(v + 1, W, p.nwt);
+    const long long vlo = rlo(v), vhi = rlo(v + 1);
     int m = 0;
     for (int j = 0; j < kMaxSteals; ++j) {
       if (rec[j].z != p.tag) break;
@@ -1075,7 +1085,7 @@ __global__ void __launch_bounds__(128, 8) decode_merge_kernel(const __grid_const
       for (int j = 0; j < kMaxSteals; ++j) rec[j] = p.steal_info[v * kMaxSteals + j];
       m = valid_steals(v, rec, st_v, sl_v);
     }
-    const long long vlo = range_lo(v, W, p.nwt), vhi = range_lo(v + 1, W, p.nwt);
+    const long long vlo = rlo(v), vhi = rlo(v + 1);
     int cnt = 0;
     for (int pos = from; pos <= m; ++pos) {
       const long long st = pos == 0 ? vlo : st_v[m - pos];
@@ -1117,7 +1127,7 @@ __global__ void __launch_bounds__(128, 8) decode_merge_kernel(const __grid_const
         const int v = w0 + chunk * NT + tid;
         int sl[ND];
         int cnt = 0;
-        if (v < p.nwt && range_lo(v, W, p.nwt) < U1) cnt = list_range(v, v == w0 ? pos0 + 1 : 0, U1, sl);
+        if (v < p.nwt && rlo(v) < U1) cnt = list_range(v, v == w0 ? pos0 + 1 : 0, U1, sl);
         int incl = cnt;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -1138,7 +1148,7 @@ __global__ void __launch_bounds__(128, 8) decode_merge_kernel(const __grid_const
         run += tot;
         __syncthreads();
         const long long next = w0 + static_cast<long long>(chunk + 1) * NT;
-        if (next >= p.nwt || range_lo(next, W, p.nwt) >= U1) break;
+        if (next >= p.nwt || rlo(static_cast<int>(next)) >= U1) break;
       }
       const int n = min(run - wlo, kCap);
       // the speculatively loaded pieces are this unit's, in this order

@@ -258,7 +258,7 @@ int launch_dependent(void (*kern)(P, int*), dim3 grid, dim3 block, cudaStream_t 
 constexpr int kWordsPerSM = 16;
 
 struct WsLayout {
-  size_t hdr, pool, words, steal, desc, part_o, part_ml, total;
+  size_t hdr, pool, words, steal, desc, rlo, part_o, part_ml, total;
   int pool_slots;
 };
 
@@ -273,7 +273,8 @@ WsLayout ws_layout(int sms, int nwt, int g, int D, int pool_slots) {
   if (cap < static_cast<size_t>(nwt)) cap = nwt;
   l.steal = round_up(l.words + cap * 8, 256);
   l.desc = round_up(l.steal + cap * kMaxSteals * 16, 256);
-  l.part_o = round_up(l.desc + cap * (1 + kMaxSteals) * 16, 256);
+  l.rlo = round_up(l.desc + cap * (1 + kMaxSteals) * 16, 256);
+  l.part_o = round_up(l.rlo + (cap + 1) * 8, 256);
   const size_t slots = 2 * static_cast<size_t>(nwt) + pool_slots;
   l.part_ml = round_up(l.part_o + slots * g * D * 4, 256);
   l.total = round_up(l.part_ml + slots * g * 2 * 4, 256);
@@ -440,6 +441,7 @@ int launch_decode(const DecodeArgs& a, bool fp8, void* ws, size_t ws_bytes, bool
   p.pool = reinterpret_cast<unsigned*>(w + L.pool);
   p.steal_info = reinterpret_cast<int4*>(w + L.steal);
   p.desc = reinterpret_cast<int4*>(w + L.desc);
+  p.rlo = reinterpret_cast<long long*>(w + L.rlo);
   p.part_o = reinterpret_cast<float*>(w + L.part_o);
   p.part_ml = reinterpret_cast<float*>(w + L.part_ml);
   if (tail) {
