@@ -54,6 +54,7 @@ enum CacheKind : int { kCacheF16 = 0, kCacheBF16 = 1, kCacheE4M3 = 2 };
 
 constexpr int kMaxSteals = 6;     // steals from one warp's range per call
 constexpr int kMinStealable = 4;  // a remainder worth splitting (items)
+constexpr int kStealMax = 8;      // items one steal takes at most
 constexpr int kStealTries = 8;
 constexpr int kScanBatch = 4;     // range words each lane loads when choosing a victim (a window of 128)
 constexpr int kMergeAhead = 8;    // ranges whose steal records the merge reads in its first round
@@ -364,6 +365,34 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
   long long issued = 0;  // items issued into the ring
 
   uint32_t qb[C::KS][2];
+  // q words of the next unit, loaded when its first item is issued (NS - 1
+  // items before it is consumed) so the load's latency hides under them;
+  // one unit at a time (qn_unit = s * Hk + h, or -1 when free).
+  uint32_t qn[C::KS][2];
+  int qn_unit = -1;
+  // The q words this thread holds of unit (s, h): head r = lane / 4 of the
+  // group (zero past g); 16-bit q: two element pairs per 16-dim step, fp8
+  // path: four consecutive elements per 16-dim step.
+  auto load_q_raw = [&](int s, int h, uint32_t (&raw)[C::KS][2]) {
+    const bool row_ok = r < p.g;
+    const long long qoff = s * p.q_s + (static_cast<long long>(h) * p.g + r) * p.q_h;
+    if constexpr (!FP8) {
+      const uint32_t* qp = reinterpret_cast<const uint32_t*>(static_cast<const uint16_t*>(p.q) + qoff);
+#pragma unroll
+      for (int ks = 0; ks < C::KS; ++ks) {
+        raw[ks][0] = row_ok ? __ldg(qp + (ks * 16 + 2 * c) / 2) : 0u;
+        raw[ks][1] = row_ok ? __ldg(qp + (ks * 16 + 8 + 2 * c) / 2) : 0u;
+      }
+    } else {
+      const uint2* qp = reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(p.q) + qoff);
+#pragma unroll
+      for (int ks = 0; ks < C::KS; ++ks) {
+        const uint2 v = row_ok ? __ldg(qp + (ks * 16 + 4 * c) / 4) : make_uint2(0u, 0u);
+        raw[ks][0] = v.x;
+        raw[ks][1] = v.y;
+      }
+    }
+  };
   float acc[C::MT][4];
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
   float sl0 = p.scale_log2, sl1 = p.scale_log2;  // logit scales of head columns 2c and 2c + 1
@@ -395,6 +424,10 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
     int pend_off = 0, pend_n = NS;
 
     auto issue = [&](int stage) {
+      if ((pc.b == 0 || pc.k == lo) && qn_unit < 0) {  // the first item of a unit: its q
+        load_q_raw(pc.s, pc.h, qn);
+        qn_unit = pc.s * p.Hk + pc.h;
+      }
       const uint32_t bar = my_bars + stage * 8;
       if (pc.L == 0) {
         if (lane == 0) mbar_arrive(bar);
@@ -473,26 +506,31 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
       float sl = p.scale_log2;
       if constexpr (FP8) sl *= __ldg(p.k_scale + cur.h);
       sl0 = sl1 = sl;
-      const bool row_ok = r < p.g;
-      const long long qoff = cur.s * p.q_s + (static_cast<long long>(cur.h) * p.g + r) * p.q_h;
-      if constexpr (!FP8) {
-        const uint32_t* qp =
-            reinterpret_cast<const uint32_t*>(static_cast<const uint16_t*>(p.q) + qoff);
+      uint32_t raw[C::KS][2];
+      if (qn_unit == cur.s * p.Hk + cur.h) {  // prefetched at issue
 #pragma unroll
         for (int ks = 0; ks < C::KS; ++ks) {
-          qb[ks][0] = row_ok ? __ldg(qp + (ks * 16 + 2 * c) / 2) : 0u;
-          qb[ks][1] = row_ok ? __ldg(qp + (ks * 16 + 8 + 2 * c) / 2) : 0u;
+          raw[ks][0] = qn[ks][0];
+          raw[ks][1] = qn[ks][1];
+        }
+        qn_unit = -1;
+      } else {
+        load_q_raw(cur.s, cur.h, raw);
+      }
+      if constexpr (!FP8) {
+#pragma unroll
+        for (int ks = 0; ks < C::KS; ++ks) {
+          qb[ks][0] = raw[ks][0];
+          qb[ks][1] = raw[ks][1];
         }
       } else {
         // k-slot order of the widened fp8 tile: slots 2c, 2c+1 <- dims 4c, 4c+1
         // and slots 2c+8, 2c+9 <- dims 4c+2, 4c+3 of each 16-dim step.
-        const uint2* qp =
-            reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(p.q) + qoff);
         float f[C::KS][4];
         float amax = 0.f;
 #pragma unroll
         for (int ks = 0; ks < C::KS; ++ks) {
-          uint2 v = row_ok ? __ldg(qp + (ks * 16 + 4 * c) / 4) : make_uint2(0u, 0u);
+          uint2 v = make_uint2(raw[ks][0], raw[ks][1]);
           if constexpr (QBF) {
             f[ks][0] = __uint_as_float(v.x << 16);
             f[ks][1] = __uint_as_float(v.x & 0xffff0000u);
@@ -923,7 +961,9 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
           const unsigned f = rw_front(cur), b = rw_back(cur), ns = rw_steals(cur);
           const long long rem = vlen - static_cast<long long>(f) - b;
           if (rem < kMinStealable || ns >= kMaxSteals) break;
-          const unsigned take = static_cast<unsigned>(rem / 2);
+          // half the remainder, at most kStealMax items: a stolen range is
+          // not stolen from again, so a large late steal becomes the tail
+          const unsigned take = static_cast<unsigned>(rem / 2 < kStealMax ? rem / 2 : kStealMax);
           const unsigned long long want = rw_make(f, b + take, ns + 1);
           const unsigned long long prev = atomicCAS(p.words + bv, cur, want);
           if (prev == cur) {
