@@ -85,6 +85,20 @@ struct DecodeParams {
   int4* steal_info;           // [nwt][kMaxSteals] (start lo, slot base, tag, start hi)
   int4* desc;                 // [nwt][1 + kMaxSteals] last-piece descriptor per sub-range
   long long* rlo;             // [nwt + 1] first item of each static warp range (the last: W)
+  // Adaptive partition (adapt = 1, with work stealing): when *part_nwt ==
+  // nwt, static range v starts at item floor(W * part[v] / 2^32) (part[0] =
+  // 0, range nwt ends at W); part was computed by the previous call's merge
+  // from the running weights wgt[gw] and each warp's predicted time for its
+  // whole range, rtime[gw] (us: from its start to the end of its own part,
+  // scaled by the items assigned over the items it processed itself).
+  // Otherwise the ranges are equal.
+  int adapt;
+  const int* part_nwt;
+  const unsigned* part;       // [nwt]
+  float* rtime;               // [nwt]
+  float* wgt;                 // [nwt]
+  int* part_nwt_w;            // the same word, written by the merge
+  unsigned* part_w;
   float* part_o;              // [2 nwt + pool_slots][g][D]
   float* part_ml;             // [2 nwt + pool_slots][g][2]
   // Prefix-aware decode (null otherwise): the first skip[s] table entries of
@@ -260,6 +274,7 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
   // The owner's first claim on its range word (NS items, see run_range) goes
   // out now so its round trip overlaps the length scan below.
   const int gw = blockIdx.x * NC + warp;
+  const uint64_t t_start = global_ns();
   unsigned long long first_claim = 0;
   if (p.steal && lane == 0) first_claim = atomicAdd(p.words + gw, static_cast<unsigned long long>(NS));
 
@@ -296,8 +311,16 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
   const long long W = *total;
   if (blockIdx.x == 0 && tid == 0) p.hdr[0] = W;
 
-  const long long my_lo = range_lo(gw, W, p.nwt);
-  const long long my_len = range_lo(gw + 1, W, p.nwt) - my_lo;
+  // first item of static range v (0 <= v <= nwt)
+  const bool adapt = p.adapt && p.steal && __ldcg(p.part_nwt) == p.nwt;
+  auto rlo_of = [&](int v) -> long long {
+    if (!adapt) return range_lo(v, W, p.nwt);
+    if (v >= p.nwt) return W;
+    return static_cast<long long>(__umul64hi(static_cast<unsigned long long>(W),
+                                             static_cast<unsigned long long>(__ldcg(p.part + v)) << 32));
+  };
+  const long long my_lo = rlo_of(gw);
+  const long long my_len = rlo_of(gw + 1) - my_lo;
   if (my_len >= (1ll << 23)) {  // range words hold 24-bit counts
     if (lane == 0) atomicOr(p.err, kErrBadLen);
     return;
@@ -690,6 +713,7 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
         return false;
       }
 
+
       bool refilled = false;
       if (cur.L > 0) {
         const uint32_t tk = my_stages + stage * C::STAGE;
@@ -872,8 +896,11 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
   // ---- own range, then steal until no remainder is worth splitting ----
   if (my_len > 0 && !run_range(my_lo, my_lo + my_len, p.steal != 0, gw, 0, 2ll * gw)) return;
   if (!p.steal) return;  // static split: every unit is cut at the same places in every call
+  if (p.adapt && lane == 0) {  // the predicted time of this warp's whole range, for the next call's partition
+    const float dt = static_cast<float>(global_ns() - t_start) * 1e-3f;
+    p.rtime[gw] = (it > 0 && my_len > 0) ? dt * static_cast<float>(my_len) / static_cast<float>(it) : 0.f;
+  }
 
-  const long long nominal = W / p.nwt;  // every static range is nominal or nominal + 1 long
   // Two partial slots from the pool per steal, reserved only once a victim
   // is in sight and kept across failed attempts (a reservation made for
   // nothing would use up the pool: every warp ends with a failed search).
@@ -898,10 +925,13 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
       // so a warp with nothing to steal leaves after one round trip.
       {
         unsigned long long wb[kScanBatch];
+        long long vl[kScanBatch];  // the sampled ranges' lengths
 #pragma unroll
         for (int j = 0; j < kScanBatch; ++j) {
           const int off = lane + 32 * j;
-          wb[j] = off < p.nwt ? ld_relaxed(p.words + (win0 + off) % p.nwt) : 0ull;
+          const int v = (win0 + off) % p.nwt;
+          wb[j] = off < p.nwt ? ld_relaxed(p.words + v) : 0ull;
+          vl[j] = rlo_of(v + 1) - rlo_of(v);
         }
 #pragma unroll
         for (int j = 0; j < kScanBatch; ++j) {
@@ -910,7 +940,7 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
           const int v = (win0 + off) % p.nwt;
           long long rem = (off >= p.nwt || rw_steals(w) >= kMaxSteals)
                               ? 0
-                              : nominal - static_cast<long long>(rw_front(w)) - rw_back(w);
+                              : vl[j] - static_cast<long long>(rw_front(w)) - rw_back(w);
           // Thieves that finish together would all pick the same largest
           // remainder and collide on one word: each scores a victim at its
           // remainder plus up to a quarter of it, by a hash of (thief,
@@ -954,8 +984,8 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
         // The owner claims an item every microsecond or so, so the word read
         // by the scan is usually stale by now: a failed CAS returns the
         // current word, which the next attempt takes as its expectation.
-        const long long vlo = range_lo(bv, W, p.nwt);
-        const long long vlen = range_lo(bv + 1, W, p.nwt) - vlo;
+        const long long vlo = rlo_of(bv);
+        const long long vlen = rlo_of(bv + 1) - vlo;
         unsigned long long cur = bw;
         for (int c = 0; c < kStealTries; ++c) {
           const unsigned f = rw_front(cur), b = rw_back(cur), ns = rw_steals(cur);
@@ -1315,6 +1345,77 @@ __global__ void __launch_bounds__(128, 8) decode_merge_kernel(const __grid_const
       }
     }
     __syncthreads();  // s_red is reused by the next cut unit
+  }
+
+  // CTA 0: the next call's partition from this call's predicted range times
+  // T_v. The weight of range v (1 at first) is multiplied by
+  // 1 + (mean T / T_v - 1) / 2 (half-way to equal times: one call's times
+  // are noisy), the weights are scaled to mean 1 and clamped to [0.5, 2],
+  // and range v gets a share of the items proportional to its weight. A
+  // range without a time keeps its weight.
+  if (blockIdx.x == 0 && p.adapt && p.steal) {
+    const int n = p.nwt;
+    const int per = (n + NT - 1) / NT;
+    const int va = min(n, tid * per), vb = min(n, va + per);
+    const bool have = __ldcg(p.part_nwt) == n;
+    double* sd = reinterpret_cast<double*>(s_red);  // [NT / 32] per-warp sums
+    // block-wide sum (and the exclusive prefix of this thread) of x
+    auto block_scan = [&](double x, double& before, double& all) {
+      double incl = x;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const double y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      __syncthreads();
+      if (lane == 31) sd[tid >> 5] = incl;
+      __syncthreads();
+      before = incl - x;
+      all = 0.0;
+#pragma unroll
+      for (int w = 0; w < NT / 32; ++w) {
+        if (w < (tid >> 5)) before += sd[w];
+        all += sd[w];
+      }
+    };
+    auto valid_time = [](float v) { return v > 0.f && v < 1e9f; };
+    double ssum = 0.0, scnt = 0.0, dummy, st, ct;
+    for (int v = va; v < vb; ++v) {
+      const float sp = p.rtime[v];
+      if (valid_time(sp)) {
+        ssum += sp;
+        scnt += 1.0;
+      }
+    }
+    block_scan(ssum, dummy, st);
+    block_scan(scnt, dummy, ct);
+    const float mean = ct > 0.0 ? static_cast<float>(st / ct) : 0.f;
+    double wsum = 0.0;
+    for (int v = va; v < vb; ++v) {
+      float wo = have ? p.wgt[v] : 1.f;
+      if (!(wo >= 0.5f && wo <= 2.f)) wo = 1.f;
+      const float sp = p.rtime[v];
+      const float w = (mean > 0.f && valid_time(sp)) ? wo * (0.5f + 0.5f * (mean / sp)) : wo;
+      p.wgt[v] = w;
+      wsum += w;
+    }
+    double wtot;
+    block_scan(wsum, dummy, wtot);
+    const float wscale = wtot > 0.0 ? static_cast<float>(n / wtot) : 1.f;
+    wsum = 0.0;
+    for (int v = va; v < vb; ++v) {
+      const float w = fminf(fmaxf(p.wgt[v] * wscale, 0.5f), 2.f);
+      p.wgt[v] = w;
+      wsum += w;
+    }
+    double run, total;
+    block_scan(wsum, run, total);
+    for (int v = va; v < vb; ++v) {
+      const double f = run / total * 4294967296.0;
+      p.part_w[v] = f >= 4294967295.0 ? 4294967295u : static_cast<unsigned>(f);
+      run += p.wgt[v];
+    }
+    if (tid == 0) *p.part_nwt_w = n;
   }
 }
 

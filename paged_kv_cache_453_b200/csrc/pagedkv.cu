@@ -261,7 +261,8 @@ int launch_dependent(void (*kern)(P, int*), dim3 grid, dim3 block, cudaStream_t 
 constexpr int kWordsPerSM = 16;
 
 struct WsLayout {
-  size_t hdr, pool, words, steal, desc, rlo, part_o, part_ml, total;
+  size_t hdr, pool, words, steal, desc, rlo, adapt, part_o, part_ml, total;
+  size_t cap;  // warps the fixed regions are sized for
   int pool_slots;
 };
 
@@ -277,7 +278,10 @@ WsLayout ws_layout(int sms, int nwt, int g, int D, int pool_slots) {
   l.steal = round_up(l.words + cap * 8, 256);
   l.desc = round_up(l.steal + cap * kMaxSteals * 16, 256);
   l.rlo = round_up(l.desc + cap * (1 + kMaxSteals) * 16, 256);
-  l.part_o = round_up(l.rlo + (cap + 1) * 8, 256);
+  // adaptive partition: its nwt word, then part, speed and wgt [cap] each
+  l.adapt = round_up(l.rlo + (cap + 1) * 8, 256);
+  l.cap = cap;
+  l.part_o = round_up(l.adapt + 16 + cap * 12, 256);
   const size_t slots = 2 * static_cast<size_t>(nwt) + pool_slots;
   l.part_ml = round_up(l.part_o + slots * g * D * 4, 256);
   l.total = round_up(l.part_ml + slots * g * 2 * 4, 256);
@@ -436,6 +440,13 @@ int launch_decode(const DecodeArgs& a, bool fp8, void* ws, size_t ws_bytes, bool
   p.nwt = nwt;
   p.tag = next_tag();
   p.steal = fixed_split ? 0 : 1;
+  // The adaptive partition pays off where the per-warp speed differences
+  // repeat from call to call: the fp8 kernel is issue-bound and a range of
+  // many short sequences is slower than one of few long ones. The 16-bit
+  // kernels are HBM-bound; their speed differences follow the SMs the CTAs
+  // land on, which change between calls, and equal ranges plus stealing do
+  // better there.
+  p.adapt = fp8 && !fixed_split ? 1 : 0;
   p.pool_slots = L.pool_slots;
   uint8_t* w = static_cast<uint8_t*>(ws);
   p.hdr = reinterpret_cast<long long*>(w + L.hdr);
@@ -445,6 +456,17 @@ int launch_decode(const DecodeArgs& a, bool fp8, void* ws, size_t ws_bytes, bool
   p.steal_info = reinterpret_cast<int4*>(w + L.steal);
   p.desc = reinterpret_cast<int4*>(w + L.desc);
   p.rlo = reinterpret_cast<long long*>(w + L.rlo);
+  {
+    int* an = reinterpret_cast<int*>(w + L.adapt);
+    const size_t cap = L.cap;
+    unsigned* part = reinterpret_cast<unsigned*>(w + L.adapt + 16);
+    p.part_nwt = an;
+    p.part_nwt_w = an;
+    p.part = part;
+    p.part_w = part;
+    p.rtime = reinterpret_cast<float*>(part + cap);
+    p.wgt = p.rtime + cap;
+  }
   p.part_o = reinterpret_cast<float*>(w + L.part_o);
   p.part_ml = reinterpret_cast<float*>(w + L.part_ml);
   if (tail) {

@@ -247,3 +247,38 @@ def test_deterministic_flag_gives_identical_bits(name):
         P.paged_attn_decode_ex(t.q, t.k_cache, t.v_cache, tables, lens, s.num_kv_heads, s.scale, s.block_size,
                                outs[0], ws, t.k_scale, t.v_scale, flags=2)
     assert e.value.status == P.PKV_ERR_INVALID_ARG
+
+
+def test_fp8_adaptive_partition_across_shapes():
+    # The fp8 decode cuts its static ranges by weights the previous call
+    # learned (kept in the workspace). Alternate two batches of one kernel
+    # configuration on one workspace, so that most calls run on a partition
+    # learned from the other batch: every call must still match the oracle,
+    # and a PKV_DECODE_DETERMINISTIC call (equal ranges, no stealing) must
+    # give the same bits whatever the learned state.
+    a = decode_case(W.scaled_down(W.spec("long_skewed"), 48, 3000, cache_dtype="fp8_e4m3"), seed=71)
+    b = decode_case(W.scaled_down(W.spec("llama3_8b"), 24, 2500, cache_dtype="fp8_e4m3"), seed=72)
+    s0 = a[0]
+    nbytes = P.workspace_bytes(s0.num_q_heads, s0.num_kv_heads, s0.head_dim, s0.block_size,
+                               P.PKV_FP8_E4M3, torch.cuda.current_device())
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    refs = [oracle_decode(*c) for c in (a, b)]
+    dev_args = [(lay.tables.cuda(), lay.lens.cuda()) for _, lay, _ in (a, b)]
+
+    def call(i, flags=0):
+        s, lay, t = (a, b)[i]
+        out = torch.full_like(t.q, float("nan"))
+        P.paged_attn_decode_ex(t.q, t.k_cache, t.v_cache, *dev_args[i], s.num_kv_heads, s.scale,
+                               s.block_size, out, ws, t.k_scale, t.v_scale, flags=flags)
+        return out
+
+    det0 = call(0, P.PKV_DECODE_DETERMINISTIC)
+    for r in range(6):
+        for i in (0, 1):
+            out = call(i)
+            torch.cuda.synchronize()
+            assert max_err(out, refs[i]) <= TOL["fp8_e4m3"], (r, i)
+    det1 = call(0, P.PKV_DECODE_DETERMINISTIC)
+    torch.cuda.synchronize()
+    check_no_device_error()
+    assert torch.equal(det0.view(torch.int16), det1.view(torch.int16))
