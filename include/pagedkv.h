@@ -205,7 +205,8 @@ int paged_attn_decode_ex(const pkv_tensor* q, const pkv_tensor* k_cache,
  *
  *   q             device [T, Hq, D] f16 | bf16, rows grouped by sequence
  *   k_cache, v_cache, block_tables, context_lens, num_kv_heads, scale,
- *   block_size    as paged_attn_decode (16-bit caches)
+ *   block_size    as paged_attn_decode (16-bit caches; fp8 caches:
+ *                 paged_attn_prefill_fp8)
  *   q_start       device int32 [S + 1], non-decreasing, q_start[S] <= T
  *   max_q_tokens  host int >= every n_s (sizes the launch)
  *   out           device [T, Hq, D] like q; rows of tokens in no sequence
@@ -227,6 +228,25 @@ int paged_attn_prefill(const pkv_tensor* q, const pkv_tensor* k_cache, const pkv
                        const pkv_tensor* block_tables, const pkv_tensor* context_lens,
                        const pkv_tensor* q_start, int max_q_tokens, int num_kv_heads, float scale,
                        int block_size, pkv_tensor* out, void* stream);
+
+/*
+ * paged_attn_prefill_fp8 - paged_attn_prefill over an fp8-e4m3 cache:
+ * k_cache / v_cache PKV_FP8_E4M3 codes [NB, Hk, B, 128], k_scale / v_scale
+ * f32 device [Hk] (element value = decode(code) * scale[h]); q / out f16 |
+ * bf16, q rounded to f16 for the dot products as in paged_attn_decode_fp8
+ * (a bf16 row of one head reaching 2^16 first scaled by a power of two that
+ * its logit scale takes back). Every row count runs on the warp-MMA kernel
+ * (codes widened to f16 in registers; a tcgen05 f16 product takes both
+ * operands in one 16-bit type); one new token per sequence is the fp8
+ * decode step. head_dim 128, block_size 16 or 32, else PKV_ERR_UNSUPPORTED;
+ * other arguments and errors as paged_attn_prefill.
+ */
+int paged_attn_prefill_fp8(const pkv_tensor* q, const pkv_tensor* k_cache,
+                           const pkv_tensor* v_cache, const pkv_tensor* k_scale,
+                           const pkv_tensor* v_scale, const pkv_tensor* block_tables,
+                           const pkv_tensor* context_lens, const pkv_tensor* q_start,
+                           int max_q_tokens, int num_kv_heads, float scale, int block_size,
+                           pkv_tensor* out, void* stream);
 
 /*
  * swap_out_blocks / swap_in_blocks - the device half of preemption by
@@ -266,7 +286,7 @@ int swap_in_blocks(const void* host_src, size_t host_bytes, const pkv_tensor* bl
  * softmax over a sequence's tokens is split into its prefix and the rest and
  * recombined with the log-sum-exp rule), equal to it up to rounding order.
  *
- * Same q, caches (16-bit only), block_tables, context_lens, num_kv_heads,
+ * Same q, caches (16-bit), block_tables, context_lens, num_kv_heads,
  * scale, block_size, out and stream as paged_attn_decode, plus a grouping of
  * the batch (pkv_prefix_groups computes one from the tables on the host):
  *   prefix_blocks  device int32 [S]: the leading table entries sequence s
@@ -289,7 +309,7 @@ int swap_in_blocks(const void* host_src, size_t host_bytes, const pkv_tensor* bl
  * in which every query head of every member attends the shared blocks, and a
  * final merge writing out. Uses a library-owned device buffer (grown with
  * cudaMalloc when a larger batch needs it; fp32 partials of S * Hq rows plus
- * the prefix chunks). PKV_ERR_UNSUPPORTED for fp8 caches.
+ * the prefix chunks). fp8 caches: paged_attn_decode_cascade_fp8.
  */
 int paged_attn_decode_cascade(const pkv_tensor* q, const pkv_tensor* k_cache,
                               const pkv_tensor* v_cache, const pkv_tensor* block_tables,
@@ -298,6 +318,27 @@ int paged_attn_decode_cascade(const pkv_tensor* q, const pkv_tensor* k_cache,
                               int num_groups, int max_group_size, int max_prefix_blocks,
                               int num_kv_heads, float scale, int block_size, pkv_tensor* out,
                               void* stream);
+
+/*
+ * paged_attn_decode_cascade_fp8 - paged_attn_decode_cascade over an
+ * fp8-e4m3 cache: k_cache / v_cache PKV_FP8_E4M3 codes [NB, Hk, B, 128],
+ * k_scale / v_scale f32 device [Hk] (element value = decode(code) *
+ * scale[h]), q / out f16 | bf16 with the rounding of paged_attn_decode_fp8
+ * (q to f16 for the dot products, a bf16 row of one head reaching 2^16
+ * first scaled by a power of two that its logit scale takes back). The
+ * shared prefix is still read once per group; the prefix pass widens the
+ * codes in registers as the decode does. head_dim 128, block_size 16 or 32,
+ * else PKV_ERR_UNSUPPORTED; other arguments and errors as
+ * paged_attn_decode_cascade.
+ */
+int paged_attn_decode_cascade_fp8(const pkv_tensor* q, const pkv_tensor* k_cache,
+                                  const pkv_tensor* v_cache, const pkv_tensor* k_scale,
+                                  const pkv_tensor* v_scale, const pkv_tensor* block_tables,
+                                  const pkv_tensor* context_lens, const pkv_tensor* prefix_blocks,
+                                  const pkv_tensor* group_start, const pkv_tensor* group_members,
+                                  int num_groups, int max_group_size, int max_prefix_blocks,
+                                  int num_kv_heads, float scale, int block_size, pkv_tensor* out,
+                                  void* stream);
 
 /*
  * paged_attn_decode_noalloc - paged_attn_decode / paged_attn_decode_fp8 for

@@ -47,7 +47,8 @@ PKV_DECODE_DETERMINISTIC = 1  # paged_attn_decode_ex flag: static split, identic
 EXPORTED = (
     "pkv_status_string", "pkv_version",
     "paged_attn_decode", "paged_attn_decode_fp8", "paged_attn_decode_workspace_bytes",
-    "paged_attn_decode_ex", "paged_attn_decode_noalloc", "paged_attn_decode_cascade", "reshape_and_cache", "reshape_and_cache_fp8", "copy_blocks",
+    "paged_attn_decode_ex", "paged_attn_decode_noalloc", "paged_attn_decode_cascade",
+    "paged_attn_decode_cascade_fp8", "paged_attn_prefill_fp8", "reshape_and_cache", "reshape_and_cache_fp8", "copy_blocks",
     "pkv_device_error",
     "pkv_alloc_create", "pkv_alloc_destroy", "pkv_seq_allocate", "pkv_seq_append_slot",
     "pkv_seq_fork", "pkv_seq_free", "pkv_seq_num_tokens", "pkv_seq_block_table",
@@ -114,8 +115,13 @@ def lib() -> ctypes.CDLL:
             "pkv_block_refcount": (ctypes.c_int, [vp, i32]),
             "paged_attn_decode_cascade": (ctypes.c_int, [P, P, P, P, P, P, P, P, ctypes.c_int, ctypes.c_int,
                                                          ctypes.c_int, ctypes.c_int, f32, ctypes.c_int, P, vp]),
+            "paged_attn_decode_cascade_fp8": (ctypes.c_int, [P, P, P, P, P, P, P, P, P, P, ctypes.c_int,
+                                                             ctypes.c_int, ctypes.c_int, ctypes.c_int, f32,
+                                                             ctypes.c_int, P, vp]),
             "paged_attn_prefill": (ctypes.c_int, [P, P, P, P, P, P, ctypes.c_int, ctypes.c_int, f32, ctypes.c_int,
                                                   P, vp]),
+            "paged_attn_prefill_fp8": (ctypes.c_int, [P, P, P, P, P, P, P, P, ctypes.c_int, ctypes.c_int, f32,
+                                                      ctypes.c_int, P, vp]),
             "pkv_alloc_utilisation": (ctypes.c_int, [vp, ctypes.POINTER(i64), ctypes.POINTER(i32)]),
             "pkv_seq_allocate_prefix": (ctypes.c_int, [vp, i64, ctypes.POINTER(i32), i32, i32]),
             "pkv_cache_create": (ctypes.c_int, [vp, ctypes.POINTER(vp)]),
@@ -232,41 +238,72 @@ class PrefixGroups:
         return g
 
 
+def _cascade_descs(q, k_cache, v_cache, block_tables, context_lens, groups, out, k_scale, v_scale):
+    """Descriptors in the argument order of paged_attn_decode_cascade(_fp8)."""
+    fp8 = k_scale is not None
+    head = [_desc(q), _desc(k_cache, fp8), _desc(v_cache, fp8)]
+    if fp8:
+        head += [_desc(k_scale), _desc(v_scale)]
+    tail = [_desc(x) for x in (block_tables, context_lens, groups.prefix_blocks, groups.group_start,
+                               groups.members)]
+    return fp8, head + tail, _desc(out)
+
+
 def paged_attn_decode_cascade(q, k_cache, v_cache, block_tables, context_lens, groups: PrefixGroups,
-                              num_kv_heads: int, scale: float, block_size: int, out, stream=None) -> None:
-    ds = [_desc(x) for x in (q, k_cache, v_cache, block_tables, context_lens, groups.prefix_blocks,
-                             groups.group_start, groups.members, out)]
-    _check(lib().paged_attn_decode_cascade(*[_ref(d) for d in ds[:8]], groups.num_groups,
-                                           groups.max_group_size, groups.max_prefix_blocks,
-                                           int(num_kv_heads), float(scale), int(block_size), _ref(ds[8]),
-                                           _stream(stream)), "paged_attn_decode_cascade")
+                              num_kv_heads: int, scale: float, block_size: int, out, stream=None,
+                              k_scale=None, v_scale=None) -> None:
+    """Prefix-aware decode; with k_scale / v_scale the caches are fp8-e4m3
+    (paged_attn_decode_cascade_fp8)."""
+    fp8, ds, do = _cascade_descs(q, k_cache, v_cache, block_tables, context_lens, groups, out,
+                                 k_scale, v_scale)
+    name = "paged_attn_decode_cascade_fp8" if fp8 else "paged_attn_decode_cascade"
+    _check(getattr(lib(), name)(*[_ref(d) for d in ds], groups.num_groups, groups.max_group_size,
+                                groups.max_prefix_blocks, int(num_kv_heads), float(scale),
+                                int(block_size), _ref(do), _stream(stream)), name)
 
 
 def prepare_decode_cascade(q, k_cache, v_cache, block_tables, context_lens, groups: PrefixGroups,
-                           num_kv_heads: int, scale: float, block_size: int, out, stream=None) -> "Prepared":
-    ds = [_desc(x) for x in (q, k_cache, v_cache, block_tables, context_lens, groups.prefix_blocks,
-                             groups.group_start, groups.members, out)]
-    args = tuple(ctypes.byref(d) for d in ds[:8]) + (
+                           num_kv_heads: int, scale: float, block_size: int, out, stream=None,
+                           k_scale=None, v_scale=None) -> "Prepared":
+    fp8, ds, do = _cascade_descs(q, k_cache, v_cache, block_tables, context_lens, groups, out,
+                                 k_scale, v_scale)
+    name = "paged_attn_decode_cascade_fp8" if fp8 else "paged_attn_decode_cascade"
+    args = tuple(ctypes.byref(d) for d in ds) + (
         groups.num_groups, groups.max_group_size, groups.max_prefix_blocks, int(num_kv_heads),
-        float(scale), int(block_size), ctypes.byref(ds[8]))
-    return Prepared("paged_attn_decode_cascade", lib().paged_attn_decode_cascade, args, (ds, groups), stream)
+        float(scale), int(block_size), ctypes.byref(do))
+    return Prepared(name, getattr(lib(), name), args, (ds, do, groups), stream)
+
+
+def _prefill_descs(q, k_cache, v_cache, block_tables, context_lens, q_start, out, k_scale, v_scale):
+    """Descriptors in the argument order of paged_attn_prefill(_fp8)."""
+    fp8 = k_scale is not None
+    ds = [_desc(q), _desc(k_cache, fp8), _desc(v_cache, fp8)]
+    if fp8:
+        ds += [_desc(k_scale), _desc(v_scale)]
+    ds += [_desc(block_tables), _desc(context_lens), _desc(q_start)]
+    return ("paged_attn_prefill_fp8" if fp8 else "paged_attn_prefill"), ds, _desc(out)
 
 
 def paged_attn_prefill(q, k_cache, v_cache, block_tables, context_lens, q_start, max_q_tokens: int,
-                       num_kv_heads: int, scale: float, block_size: int, out, stream=None) -> None:
+                       num_kv_heads: int, scale: float, block_size: int, out, stream=None,
+                       k_scale=None, v_scale=None) -> None:
     """Causal attention of several new tokens per sequence (q rows of sequence
-    s: q_start[s] .. q_start[s + 1], its last tokens; lens include them)."""
-    ds = [_desc(x) for x in (q, k_cache, v_cache, block_tables, context_lens, q_start, out)]
-    _check(lib().paged_attn_prefill(*[_ref(d) for d in ds[:6]], int(max_q_tokens), int(num_kv_heads), float(scale),
-                                    int(block_size), _ref(ds[6]), _stream(stream)), "paged_attn_prefill")
+    s: q_start[s] .. q_start[s + 1], its last tokens; lens include them); with
+    k_scale / v_scale the caches are fp8-e4m3 (paged_attn_prefill_fp8)."""
+    name, ds, do = _prefill_descs(q, k_cache, v_cache, block_tables, context_lens, q_start, out,
+                                  k_scale, v_scale)
+    _check(getattr(lib(), name)(*[_ref(d) for d in ds], int(max_q_tokens), int(num_kv_heads), float(scale),
+                                int(block_size), _ref(do), _stream(stream)), name)
 
 
 def prepare_prefill(q, k_cache, v_cache, block_tables, context_lens, q_start, max_q_tokens: int,
-                    num_kv_heads: int, scale: float, block_size: int, out, stream=None) -> "Prepared":
-    ds = [_desc(x) for x in (q, k_cache, v_cache, block_tables, context_lens, q_start, out)]
-    args = tuple(ctypes.byref(d) for d in ds[:6]) + (int(max_q_tokens), int(num_kv_heads), float(scale),
-                                                    int(block_size), ctypes.byref(ds[6]))
-    return Prepared("paged_attn_prefill", lib().paged_attn_prefill, args, ds, stream)
+                    num_kv_heads: int, scale: float, block_size: int, out, stream=None,
+                    k_scale=None, v_scale=None) -> "Prepared":
+    name, ds, do = _prefill_descs(q, k_cache, v_cache, block_tables, context_lens, q_start, out,
+                                  k_scale, v_scale)
+    args = tuple(ctypes.byref(d) for d in ds) + (int(max_q_tokens), int(num_kv_heads), float(scale),
+                                                 int(block_size), ctypes.byref(do))
+    return Prepared(name, getattr(lib(), name), args, (ds, do), stream)
 
 
 def swap_record_bytes(k_cache) -> int:

@@ -26,6 +26,10 @@
 //   3. cascade_merge_kernel: one warp per (member, query head) folds the
 //      prefix chunks' partials and the step-1 partial, normalises and writes
 //      the output row.
+// With an fp8-e4m3 cache the prefix pass widens the codes to f16 in
+// registers as the decode does (q rounded to f16, a bf16 row past the f16
+// range scaled by a power of two that its logit scale takes back; the K
+// scale folded into the logit scale, the V scale into the partials).
 #pragma once
 
 #include "decode.cuh"
@@ -67,13 +71,16 @@ struct CascadeParams {
   float* pre_ml;        // [G * Hk * ncc * nkc][kCasCols][2]
   const float* suf_o;   // [S * Hq][D] step-1 partials
   const float* suf_ml;  // [S * Hq][2]
+  const float* k_scale;  // [Hk], fp8 caches only
+  const float* v_scale;
 };
 
-template <bool QBF, int D, int BS, int NS>
+template <bool QBF, int D, int BS, int NS, bool FP8 = false>
 struct PrefixCfg {
-  static constexpr int EPR = 64;           // 16-bit elements per 128-byte row
-  static constexpr int NH = (D * 2) / 128;  // 128-byte column groups per token row
-  static constexpr int TILE = BS * D * 2;
+  static constexpr int EB = FP8 ? 1 : 2;     // cache element bytes
+  static constexpr int EPR = 128 / EB;       // elements per 128-byte row
+  static constexpr int NH = (D * EB) / 128;  // 128-byte column groups per token row
+  static constexpr int TILE = BS * D * EB;
   static constexpr int STAGE = 2 * TILE;
   static constexpr int KS = D / 16;
   static constexpr int MT = D / 16;
@@ -81,11 +88,12 @@ struct PrefixCfg {
   static constexpr int SMEM = 1024 + NS * STAGE + 2 * NS * 8 + kCasMaxChunk * 4;
   static_assert(D % 64 == 0, "head_dim must be a multiple of 64");
   static_assert(BS % 16 == 0, "block_size must be a multiple of 16");
+  static_assert(!FP8 || D == 128, "fp8 caches: head_dim 128");
 };
 
-template <bool QBF, int D, int BS, int NS>
+template <bool QBF, int D, int BS, int NS, bool FP8 = false>
 __global__ void __launch_bounds__(128, 1) cascade_prefix_kernel(const __grid_constant__ CascadeParams p) {
-  using C = PrefixCfg<QBF, D, BS, NS>;
+  using C = PrefixCfg<QBF, D, BS, NS, FP8>;
   constexpr uint64_t kWaitNs = 2000000000ull;
 
   extern __shared__ uint8_t smem_raw[];
@@ -166,8 +174,15 @@ __global__ void __launch_bounds__(128, 1) cascade_prefix_kernel(const __grid_con
 
   // Q^T fragments of this warp's 16 columns: n-tile jt holds columns
   // cc * 64 + warp * 16 + jt * 8 + (0..7); lane r carries column 8 jt + r.
+  // fp8: the k-slot order of the widened tile puts dims 4c, 4c + 1 in slots
+  // 2c, 2c + 1 and dims 4c + 2, 4c + 3 in slots 2c + 8, 2c + 9 of each
+  // 16-dim step; q is rounded to f16 (a bf16 row of 2^16 and up first
+  // scaled by 2^-e) and slj holds the logit scales of this lane's two
+  // accumulator columns (K scale and 2^e included).
   uint32_t qb[2][C::KS][2];
   bool col_ok[2][2];
+  float slj[2][2];
+  const float sl_base = FP8 ? p.scale_log2 * __ldg(p.k_scale + h) : p.scale_log2;
 #pragma unroll
   for (int jt = 0; jt < 2; ++jt) {
     const int col = cc * kCasCols + warp * 16 + jt * 8 + r;
@@ -175,12 +190,54 @@ __global__ void __launch_bounds__(128, 1) cascade_prefix_kernel(const __grid_con
     const int mi = ok ? col / p.g : 0;
     const int s = ok ? __ldg(p.members + m0 + mi) : 0;
     const bool s_ok = ok && s >= 0 && s < p.S;
-    const uint32_t* qp = reinterpret_cast<const uint32_t*>(
-        static_cast<const uint16_t*>(p.q) + s * p.q_s + (static_cast<long long>(h) * p.g + col % p.g) * p.q_h);
+    const long long qoff = s * p.q_s + (static_cast<long long>(h) * p.g + col % p.g) * p.q_h;
+    slj[jt][0] = slj[jt][1] = sl_base;
+    if constexpr (!FP8) {
+      const uint32_t* qp = reinterpret_cast<const uint32_t*>(static_cast<const uint16_t*>(p.q) + qoff);
 #pragma unroll
-    for (int ks = 0; ks < C::KS; ++ks) {
-      qb[jt][ks][0] = s_ok ? __ldg(qp + (ks * 16 + 2 * c) / 2) : 0u;
-      qb[jt][ks][1] = s_ok ? __ldg(qp + (ks * 16 + 8 + 2 * c) / 2) : 0u;
+      for (int ks = 0; ks < C::KS; ++ks) {
+        qb[jt][ks][0] = s_ok ? __ldg(qp + (ks * 16 + 2 * c) / 2) : 0u;
+        qb[jt][ks][1] = s_ok ? __ldg(qp + (ks * 16 + 8 + 2 * c) / 2) : 0u;
+      }
+    } else {
+      const uint2* qp = reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(p.q) + qoff);
+      float f[C::KS][4];
+      float amax = 0.f;
+#pragma unroll
+      for (int ks = 0; ks < C::KS; ++ks) {
+        const uint2 v = s_ok ? __ldg(qp + (ks * 16 + 4 * c) / 4) : make_uint2(0u, 0u);
+        if constexpr (QBF) {
+          f[ks][0] = __uint_as_float(v.x << 16);
+          f[ks][1] = __uint_as_float(v.x & 0xffff0000u);
+          f[ks][2] = __uint_as_float(v.y << 16);
+          f[ks][3] = __uint_as_float(v.y & 0xffff0000u);
+          amax = fmaxf(amax, fmaxf(fmaxf(fabsf(f[ks][0]), fabsf(f[ks][1])),
+                                   fmaxf(fabsf(f[ks][2]), fabsf(f[ks][3]))));
+        } else {
+          const __half2 a2 = *reinterpret_cast<const __half2*>(&v.x);
+          const __half2 b2 = *reinterpret_cast<const __half2*>(&v.y);
+          f[ks][0] = __low2float(a2);
+          f[ks][1] = __high2float(a2);
+          f[ks][2] = __low2float(b2);
+          f[ks][3] = __high2float(b2);
+        }
+      }
+      float qs = 1.f;
+      if constexpr (QBF) {  // the row of column 8 jt + r is held by lanes 4r .. 4r + 3
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        const int ex = static_cast<int>((__float_as_uint(amax) >> 23) & 0xffu) - 127;
+        const int e = ex >= 16 ? ex - 15 : 0;
+        qs = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+        const int e0 = __shfl_sync(0xffffffffu, e, 8 * c), e1 = __shfl_sync(0xffffffffu, e, 8 * c + 4);
+        slj[jt][0] = sl_base * __uint_as_float(static_cast<uint32_t>(127 + e0) << 23);
+        slj[jt][1] = sl_base * __uint_as_float(static_cast<uint32_t>(127 + e1) << 23);
+      }
+#pragma unroll
+      for (int ks = 0; ks < C::KS; ++ks) {
+        qb[jt][ks][0] = pack2<false>(f[ks][0] * qs, f[ks][1] * qs);
+        qb[jt][ks][1] = pack2<false>(f[ks][2] * qs, f[ks][3] * qs);
+      }
     }
     // the two accumulator columns of this lane: 8 jt + 2c and + 1
     const int cb0 = cc * kCasCols + warp * 16 + jt * 8 + 2 * c;
@@ -197,7 +254,6 @@ __global__ void __launch_bounds__(128, 1) cascade_prefix_kernel(const __grid_con
     mrun[jt][0] = mrun[jt][1] = -INFINITY;
     lrun[jt][0] = lrun[jt][1] = 0.f;
   }
-  const float sl = p.scale_log2;
   bool failed = false;
   int issued = min(NS, n);  // thread 0's count of blocks issued
   int jfail = n;            // first block this warp gave up on
@@ -219,18 +275,37 @@ __global__ void __launch_bounds__(128, 1) cascade_prefix_kernel(const __grid_con
 #pragma unroll
       for (int jt = 0; jt < 2; ++jt) sacc[jt][0] = sacc[jt][1] = sacc[jt][2] = sacc[jt][3] = 0.f;
       const int trow = tt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+      if constexpr (!FP8) {
 #pragma unroll
-      for (int ks = 0; ks < C::KS; ++ks) {
-        uint32_t a0, a1, a2, a3;
-        ldsm_x4(tk + swz<BS>(trow, ks * 32 + (lane >> 4) * 16), a0, a1, a2, a3);
+        for (int ks = 0; ks < C::KS; ++ks) {
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(tk + swz<BS>(trow, ks * 32 + (lane >> 4) * 16), a0, a1, a2, a3);
 #pragma unroll
-        for (int jt = 0; jt < 2; ++jt) mma16816<QBF>(sacc[jt], a0, a1, a2, a3, qb[jt][ks][0], qb[jt][ks][1]);
+          for (int jt = 0; jt < 2; ++jt) mma16816<QBF>(sacc[jt], a0, a1, a2, a3, qb[jt][ks][0], qb[jt][ks][1]);
+        }
+      } else {
+#pragma unroll
+        for (int kp = 0; kp < C::KS / 2; ++kp) {
+          uint32_t x0, x1, x2, x3;
+          ldsm_x4(tk + swz<BS>(trow, kp * 32 + (lane >> 4) * 16), x0, x1, x2, x3);
+          uint32_t a0, a2, a1, a3, b0, b2, b1, b3;
+          e4m3x4_to_f16x2x2(x0, a0, a2);
+          e4m3x4_to_f16x2x2(x1, a1, a3);
+          e4m3x4_to_f16x2x2(x2, b0, b2);
+          e4m3x4_to_f16x2x2(x3, b1, b3);
+#pragma unroll
+          for (int jt = 0; jt < 2; ++jt) {
+            mma16816<false>(sacc[jt], a0, a1, a2, a3, qb[jt][2 * kp][0], qb[jt][2 * kp][1]);
+            mma16816<false>(sacc[jt], b0, b1, b2, b3, qb[jt][2 * kp + 1][0], qb[jt][2 * kp + 1][1]);
+          }
+        }
       }
       // online softmax per column (every prefix token is valid)
       uint32_t pb[2][2];
 #pragma unroll
       for (int jt = 0; jt < 2; ++jt) {
-        float x0 = sacc[jt][0] * sl, x1 = sacc[jt][1] * sl, x2 = sacc[jt][2] * sl, x3 = sacc[jt][3] * sl;
+        const float x0 = sacc[jt][0] * slj[jt][0], x1 = sacc[jt][1] * slj[jt][1];
+        const float x2 = sacc[jt][2] * slj[jt][0], x3 = sacc[jt][3] * slj[jt][1];
         float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
 #pragma unroll
         for (int o = 4; o < 32; o <<= 1) {
@@ -254,17 +329,38 @@ __global__ void __launch_bounds__(128, 1) cascade_prefix_kernel(const __grid_con
         const float p2 = exp2f(x2 - mn0), p3 = exp2f(x3 - mn1);
         lrun[jt][0] += p0 + p2;
         lrun[jt][1] += p1 + p3;
-        pb[jt][0] = movmatrix_t(pack2<QBF>(p0, p1));
-        pb[jt][1] = movmatrix_t(pack2<QBF>(p2, p3));
+        pb[jt][0] = movmatrix_t(pack2<QBF && !FP8>(p0, p1));
+        pb[jt][1] = movmatrix_t(pack2<QBF && !FP8>(p2, p3));
       }
-      // O^T += V^T P^T (V fragments shared by both n-tiles)
+      // O^T += V^T P^T (V fragments shared by both n-tiles; fp8: one
+      // transposed load covers two m-tiles, widened to f16)
+      if constexpr (!FP8) {
 #pragma unroll
-      for (int i = 0; i < C::MT; ++i) {
-        const int vrow = tt * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
-        uint32_t f0, f1, f2, f3;
-        ldsm_x4_t(tv + swz<BS>(vrow, i * 32 + ((lane >> 3) & 1) * 16), f0, f1, f2, f3);
+        for (int i = 0; i < C::MT; ++i) {
+          const int vrow = tt * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
+          uint32_t f0, f1, f2, f3;
+          ldsm_x4_t(tv + swz<BS>(vrow, i * 32 + ((lane >> 3) & 1) * 16), f0, f1, f2, f3);
 #pragma unroll
-        for (int jt = 0; jt < 2; ++jt) mma16816<QBF>(acc[jt][i], f0, f1, f2, f3, pb[jt][0], pb[jt][1]);
+          for (int jt = 0; jt < 2; ++jt) mma16816<QBF>(acc[jt][i], f0, f1, f2, f3, pb[jt][0], pb[jt][1]);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < C::MT / 2; ++i) {
+          const int vrow = tt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+          uint32_t x0, x1, x2, x3, f[8];
+          ldsm_x4_t(tv + swz<BS>(vrow, i * 32 + (lane >> 4) * 16), x0, x1, x2, x3);
+          // bytes (d, t), (d + 1, t), (d, t + 1), (d + 1, t + 1) -> token
+          // pairs (d, t | t + 1) and (d + 1, t | t + 1)
+          e4m3x4_to_f16x2x2(prmt(x0, 0, 0x3120), f[0], f[1]);
+          e4m3x4_to_f16x2x2(prmt(x1, 0, 0x3120), f[2], f[3]);
+          e4m3x4_to_f16x2x2(prmt(x2, 0, 0x3120), f[4], f[5]);
+          e4m3x4_to_f16x2x2(prmt(x3, 0, 0x3120), f[6], f[7]);
+#pragma unroll
+          for (int jt = 0; jt < 2; ++jt) {
+            mma16816<false>(acc[jt][2 * i], f[0], f[1], f[2], f[3], pb[jt][0], pb[jt][1]);
+            mma16816<false>(acc[jt][2 * i + 1], f[4], f[5], f[6], f[7], pb[jt][0], pb[jt][1]);
+          }
+        }
       }
     }
     __syncwarp();
@@ -288,7 +384,9 @@ __global__ void __launch_bounds__(128, 1) cascade_prefix_kernel(const __grid_con
     return;
   }
 
-  // partials of this chunk: one row of D floats (and m, l) per column
+  // partials of this chunk: one row of D floats (and m, l) per column, O
+  // scaled by the V scale (fp8)
+  const float vs = FP8 ? __ldg(p.v_scale + h) : 1.f;
   const long long item = ((static_cast<long long>(blockIdx.z) * p.ncc + cc) * p.nkc + kc);
   float* po = p.pre_o + item * kCasCols * D;
   float* pm = p.pre_ml + item * kCasCols * 2;
@@ -303,14 +401,15 @@ __global__ void __launch_bounds__(128, 1) cascade_prefix_kernel(const __grid_con
     const int cl = warp * 16 + jt * 8 + 2 * c;  // column within the chunk
 #pragma unroll
     for (int mt = 0; mt < C::MT; ++mt) {
-      const int da = 16 * mt + r, db = da + 8;
+      const int da = FP8 ? 16 * mt + 2 * r : 16 * mt + r;
+      const int db = FP8 ? da + 1 : da + 8;
       if (col_ok[jt][0]) {
-        po[cl * D + da] = acc[jt][mt][0];
-        po[cl * D + db] = acc[jt][mt][2];
+        po[cl * D + da] = acc[jt][mt][0] * vs;
+        po[cl * D + db] = acc[jt][mt][2] * vs;
       }
       if (col_ok[jt][1]) {
-        po[(cl + 1) * D + da] = acc[jt][mt][1];
-        po[(cl + 1) * D + db] = acc[jt][mt][3];
+        po[(cl + 1) * D + da] = acc[jt][mt][1] * vs;
+        po[(cl + 1) * D + db] = acc[jt][mt][3] * vs;
       }
     }
     if (r == 0) {

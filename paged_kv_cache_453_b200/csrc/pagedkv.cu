@@ -507,15 +507,20 @@ struct CascadeLaunch {
   bool attr_set[kMaxDevices];
 };
 
-template <bool QBF, int D, int BS>
+template <bool QBF, int D, int BS, bool FP8 = false>
 CascadeLaunch* cascade_entry() {
   constexpr int NS = 4;
-  static CascadeLaunch e = {&cascade_prefix_kernel<QBF, D, BS, NS>, &cascade_merge_kernel<QBF, D>,
-                            PrefixCfg<QBF, D, BS, NS>::SMEM, {false}};
+  static CascadeLaunch e = {&cascade_prefix_kernel<QBF, D, BS, NS, FP8>, &cascade_merge_kernel<QBF, D>,
+                            PrefixCfg<QBF, D, BS, NS, FP8>::SMEM, {false}};
   return &e;
 }
 
-CascadeLaunch* pick_cascade(bool qbf, int D, int BS) {
+CascadeLaunch* pick_cascade(bool qbf, int D, int BS, bool fp8) {
+  if (fp8) {  // e4m3 pools, D = 128
+    if (D != 128) return nullptr;
+    if (qbf) return BS == 16 ? cascade_entry<true, 128, 16, true>() : cascade_entry<true, 128, 32, true>();
+    return BS == 16 ? cascade_entry<false, 128, 16, true>() : cascade_entry<false, 128, 32, true>();
+  }
   if (qbf) {
     if (D == 128 && BS == 16) return cascade_entry<true, 128, 16>();
     if (D == 128 && BS == 32) return cascade_entry<true, 128, 32>();
@@ -530,12 +535,12 @@ CascadeLaunch* pick_cascade(bool qbf, int D, int BS) {
   return nullptr;
 }
 
-int launch_cascade(const DecodeArgs& a, const pkv_tensor* pblk, const pkv_tensor* gstart,
+int launch_cascade(const DecodeArgs& a, bool fp8, const pkv_tensor* pblk, const pkv_tensor* gstart,
                    const pkv_tensor* gmem, int G, int max_members, int max_prefix,
                    cudaStream_t stream) {
   int ck = 0;
   DecodeLaunch* e = nullptr;
-  int st = check_decode(a, false, &ck, &e);
+  int st = check_decode(a, fp8, &ck, &e);
   if (st != PKV_OK) return st;
   if (!pblk || !gstart || !gmem || G < 0 || max_members < 0 || max_prefix < 0)
     return PKV_ERR_INVALID_ARG;
@@ -553,7 +558,7 @@ int launch_cascade(const DecodeArgs& a, const pkv_tensor* pblk, const pkv_tensor
     return PKV_ERR_INVALID_ARG;
   const int D = static_cast<int>(a.q->shape[2]);
   const int g = static_cast<int>(a.q->shape[1] / a.Hk);
-  CascadeLaunch* ce = pick_cascade(a.q->dtype == PKV_BF16, D, a.BS);
+  CascadeLaunch* ce = pick_cascade(a.q->dtype == PKV_BF16, D, a.BS, fp8);
   if (!ce) return PKV_ERR_UNSUPPORTED;
   int dev;
   if ((st = current_device(&dev)) != PKV_OK) return st;
@@ -595,14 +600,15 @@ int launch_cascade(const DecodeArgs& a, const pkv_tensor* pblk, const pkv_tensor
   }
   CascadeTail tail{static_cast<const int*>(pblk->data), reinterpret_cast<float*>(cw + suf_o),
                    reinterpret_cast<float*>(cw + suf_ml)};
-  if ((st = launch_decode(a, false, nullptr, 0, true, stream, false, false, &tail)) != PKV_OK)
+  if ((st = launch_decode(a, fp8, nullptr, 0, true, stream, false, false, &tail)) != PKV_OK)
     return st;
   if (G == 0 || M == 0) return PKV_OK;
 
   CascadeParams p;
   std::memset(&p, 0, sizeof(p));
-  if ((st = encode_pool_map(&p.tmk, a.kc, a.q->dtype)) != PKV_OK) return st;
-  if ((st = encode_pool_map(&p.tmv, a.vc, a.q->dtype)) != PKV_OK) return st;
+  const int cdt = fp8 ? PKV_FP8_E4M3 : a.q->dtype;
+  if ((st = encode_pool_map(&p.tmk, a.kc, cdt)) != PKV_OK) return st;
+  if ((st = encode_pool_map(&p.tmv, a.vc, cdt)) != PKV_OK) return st;
   p.q = a.q->data;
   p.q_s = a.q->stride[0];
   p.q_h = a.q->stride[1];
@@ -611,6 +617,8 @@ int launch_cascade(const DecodeArgs& a, const pkv_tensor* pblk, const pkv_tensor
   p.o_h = a.out->stride[1];
   p.tables = static_cast<const int*>(a.bt->data);
   p.t_s = a.bt->stride[0];
+  p.k_scale = fp8 ? static_cast<const float*>(a.ks->data) : nullptr;
+  p.v_scale = fp8 ? static_cast<const float*>(a.vs->data) : nullptr;
   p.prefix_blocks = static_cast<const int*>(pblk->data);
   p.group_start = static_cast<const int*>(gstart->data);
   p.members = static_cast<const int*>(gmem->data);
@@ -662,22 +670,27 @@ struct PrefillLaunch {
   bool attr_set[kMaxDevices];
 };
 
-template <bool QBF, int D, int BS, int NW>
+template <bool QBF, int D, int BS, int NW, bool FP8 = false>
 PrefillLaunch* prefill_entry() {
   constexpr int NS = 4;
-  static PrefillLaunch e = {&prefill_kernel<QBF, D, BS, NS, NW>, &prefill_merge_kernel<QBF, D>, NW * 32,
-                            PrefillCfg<QBF, D, BS, NS, NW>::SMEM, NW * 16, {false}};
+  static PrefillLaunch e = {&prefill_kernel<QBF, D, BS, NS, NW, FP8>, &prefill_merge_kernel<QBF, D>, NW * 32,
+                            PrefillCfg<QBF, D, BS, NS, NW, FP8>::SMEM, NW * 16, {false}};
   return &e;
 }
 
-template <bool QBF, int D, int BS>
+template <bool QBF, int D, int BS, bool FP8 = false>
 PrefillLaunch* prefill_by_cols(int cols) {
-  if (cols <= 16) return prefill_entry<QBF, D, BS, 1>();
-  if (cols <= 32) return prefill_entry<QBF, D, BS, 2>();
-  return prefill_entry<QBF, D, BS, 4>();
+  if (cols <= 16) return prefill_entry<QBF, D, BS, 1, FP8>();
+  if (cols <= 32) return prefill_entry<QBF, D, BS, 2, FP8>();
+  return prefill_entry<QBF, D, BS, 4, FP8>();
 }
 
-PrefillLaunch* pick_prefill(bool qbf, int D, int BS, int cols) {
+PrefillLaunch* pick_prefill(bool qbf, int D, int BS, int cols, bool fp8) {
+  if (fp8) {  // e4m3 pools, D = 128
+    if (D != 128) return nullptr;
+    if (qbf) return BS == 16 ? prefill_by_cols<true, 128, 16, true>(cols) : prefill_by_cols<true, 128, 32, true>(cols);
+    return BS == 16 ? prefill_by_cols<false, 128, 16, true>(cols) : prefill_by_cols<false, 128, 32, true>(cols);
+  }
   if (qbf) {
     if (D == 128 && BS == 16) return prefill_by_cols<true, 128, 16>(cols);
     if (D == 128 && BS == 32) return prefill_by_cols<true, 128, 32>(cols);
@@ -726,6 +739,7 @@ PrefillTcLaunch* pick_prefill_tc(bool qbf, int BS, int cols) {
 }
 
 int launch_prefill(const pkv_tensor* q, const pkv_tensor* kc, const pkv_tensor* vc,
+                   const pkv_tensor* ks, const pkv_tensor* vs, bool fp8,
                    const pkv_tensor* bt, const pkv_tensor* cl, const pkv_tensor* qs, int max_q,
                    int Hk, float scale, int BS, pkv_tensor* out, cudaStream_t stream) {
   if (!q || !kc || !vc || !bt || !cl || !qs || !out) return PKV_ERR_INVALID_ARG;
@@ -733,7 +747,11 @@ int launch_prefill(const pkv_tensor* q, const pkv_tensor* kc, const pkv_tensor* 
   if (qdt != PKV_F16 && qdt != PKV_BF16) return PKV_ERR_INVALID_ARG;
   if (!well_formed(q, 3, qdt) || !well_formed(out, 3, qdt) || !same_shape(q, out))
     return PKV_ERR_INVALID_ARG;
-  if (!pool_ok(kc, qdt) || !pool_ok(vc, qdt) || !same_shape(kc, vc)) return PKV_ERR_INVALID_ARG;
+  const int cdt = fp8 ? PKV_FP8_E4M3 : qdt;
+  if (!pool_ok(kc, cdt) || !pool_ok(vc, cdt) || !same_shape(kc, vc)) return PKV_ERR_INVALID_ARG;
+  if (fp8 && (!ks || !vs || !well_formed(ks, 1, PKV_F32) || !well_formed(vs, 1, PKV_F32) ||
+              ks->shape[0] != Hk || vs->shape[0] != Hk || ks->stride[0] != 1 || vs->stride[0] != 1))
+    return PKV_ERR_INVALID_ARG;
   const int64_t T = q->shape[0], Hq = q->shape[1], D = q->shape[2];
   const int64_t NB = kc->shape[0];
   if (kc->shape[1] != Hk || kc->shape[2] != BS || kc->shape[3] != D || Hk <= 0 || Hq % Hk != 0)
@@ -744,17 +762,19 @@ int launch_prefill(const pkv_tensor* q, const pkv_tensor* kc, const pkv_tensor* 
   if (!well_formed(qs, 1, PKV_I32) || qs->shape[0] != S + 1 || qs->stride[0] != 1)
     return PKV_ERR_INVALID_ARG;
   if (!std::isfinite(scale) || max_q < 0) return PKV_ERR_INVALID_ARG;
-  if (T > 0 && (q->stride[0] % 2 || q->stride[1] % 2 || !aligned(q->data, 4)))
+  // q rows are read as 4- (16-bit cache) or 8-byte (fp8 cache) words
+  const int qa = fp8 ? 4 : 2;
+  if (T > 0 && (q->stride[0] % qa || q->stride[1] % qa || !aligned(q->data, 2 * qa)))
     return PKV_ERR_INVALID_ARG;
   const int64_t g = Hq / Hk;
-  if ((D != 64 && D != 128) || (BS != 16 && BS != 32)) return PKV_ERR_UNSUPPORTED;
+  if ((D != 64 && D != 128) || (BS != 16 && BS != 32) || (fp8 && D != 128)) return PKV_ERR_UNSUPPORTED;
   if (NB > INT32_MAX || T > INT32_MAX || S * Hk > 65535LL || S > 65535LL ||
       static_cast<int64_t>(max_q) * g > INT32_MAX / 2)
     return PKV_ERR_UNSUPPORTED;
   if (S == 0 || T == 0 || max_q == 0) return PKV_OK;
   if (bt->shape[1] < 1 || NB < 1) return PKV_ERR_INVALID_ARG;
   const int cols = static_cast<int>(max_q * g);
-  PrefillLaunch* e = pick_prefill(qdt == PKV_BF16, static_cast<int>(D), BS, cols);
+  PrefillLaunch* e = pick_prefill(qdt == PKV_BF16, static_cast<int>(D), BS, cols, fp8);
   if (!e) return PKV_ERR_UNSUPPORTED;
   int dev, st;
   if ((st = current_device(&dev)) != PKV_OK) return st;
@@ -767,7 +787,9 @@ int launch_prefill(const pkv_tensor* q, const pkv_tensor* kc, const pkv_tensor* 
   // the scale is positive (that kernel takes row maxima of unscaled scores)
   const bool rows16 = q->stride[0] % 8 == 0 && q->stride[1] % 8 == 0 && aligned(q->data, 16) &&
                       out->stride[0] % 8 == 0 && out->stride[1] % 8 == 0 && aligned(out->data, 16);
-  const bool use_tc = D == 128 && cols >= 64 && rows16 && scale > 0.f;
+  // (fp8 caches stay on the warp MMAs: a tcgen05 f16 product takes both
+  // operands in one 16-bit type, and these kernels stage K and V as stored)
+  const bool use_tc = !fp8 && D == 128 && cols >= 64 && rows16 && scale > 0.f;
   {
     std::lock_guard<std::mutex> lk(g_mu);
     if (!e->attr_set[dev]) {
@@ -779,8 +801,10 @@ int launch_prefill(const pkv_tensor* q, const pkv_tensor* kc, const pkv_tensor* 
   }
   PrefillParams p;
   std::memset(&p, 0, sizeof(p));
-  if ((st = encode_pool_map(&p.tmk, kc, qdt)) != PKV_OK) return st;
-  if ((st = encode_pool_map(&p.tmv, vc, qdt)) != PKV_OK) return st;
+  if ((st = encode_pool_map(&p.tmk, kc, cdt)) != PKV_OK) return st;
+  if ((st = encode_pool_map(&p.tmv, vc, cdt)) != PKV_OK) return st;
+  p.k_scale = fp8 ? static_cast<const float*>(ks->data) : nullptr;
+  p.v_scale = fp8 ? static_cast<const float*>(vs->data) : nullptr;
   p.q = q->data;
   p.q_t = q->stride[0];
   p.q_h = q->stride[1];
@@ -1047,6 +1071,27 @@ int noalloc_scratch(int dev, void** out) {
 
 using namespace pkv;
 
+// One new token per sequence (max_q_tokens 1 and as many query rows as
+// sequences) is the decode step: the decode kernel serves it (q_start can
+// then only be 0, 1, ..., S and is not read). Shapes the decode does not take
+// go to the multi-token kernels.
+static int prefill_or_decode(const pkv_tensor* q, const pkv_tensor* k_cache, const pkv_tensor* v_cache,
+                      const pkv_tensor* k_scale, const pkv_tensor* v_scale, bool fp8,
+                      const pkv_tensor* block_tables, const pkv_tensor* context_lens,
+                      const pkv_tensor* q_start, int max_q_tokens, int num_kv_heads, float scale,
+                      int block_size, pkv_tensor* out, void* stream) {
+  if (q && block_tables && max_q_tokens == 1 && q->ndim == 3 && block_tables->ndim == 2 &&
+      q->shape[0] == block_tables->shape[0]) {
+    DecodeArgs a{q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
+                 num_kv_heads, scale, block_size, out};
+    const int st = launch_decode(a, fp8, nullptr, 0, true, static_cast<cudaStream_t>(stream));
+    if (st != PKV_ERR_UNSUPPORTED) return st;
+  }
+  return launch_prefill(q, k_cache, v_cache, k_scale, v_scale, fp8, block_tables, context_lens,
+                        q_start, max_q_tokens, num_kv_heads, scale, block_size, out,
+                        static_cast<cudaStream_t>(stream));
+}
+
 extern "C" {
 
 const char* pkv_status_string(int s) {
@@ -1096,8 +1141,22 @@ int paged_attn_decode_cascade(const pkv_tensor* q, const pkv_tensor* k_cache,
                               void* stream) {
   DecodeArgs a{q, k_cache, v_cache, nullptr, nullptr, block_tables, context_lens,
                num_kv_heads, scale, block_size, out};
-  return launch_cascade(a, prefix_blocks, group_start, group_members, num_groups, max_group_size,
-                        max_prefix_blocks, static_cast<cudaStream_t>(stream));
+  return launch_cascade(a, false, prefix_blocks, group_start, group_members, num_groups,
+                        max_group_size, max_prefix_blocks, static_cast<cudaStream_t>(stream));
+}
+
+int paged_attn_decode_cascade_fp8(const pkv_tensor* q, const pkv_tensor* k_cache,
+                                  const pkv_tensor* v_cache, const pkv_tensor* k_scale,
+                                  const pkv_tensor* v_scale, const pkv_tensor* block_tables,
+                                  const pkv_tensor* context_lens, const pkv_tensor* prefix_blocks,
+                                  const pkv_tensor* group_start, const pkv_tensor* group_members,
+                                  int num_groups, int max_group_size, int max_prefix_blocks,
+                                  int num_kv_heads, float scale, int block_size, pkv_tensor* out,
+                                  void* stream) {
+  DecodeArgs a{q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
+               num_kv_heads, scale, block_size, out};
+  return launch_cascade(a, true, prefix_blocks, group_start, group_members, num_groups,
+                        max_group_size, max_prefix_blocks, static_cast<cudaStream_t>(stream));
 }
 
 size_t paged_attn_decode_workspace_bytes(int num_q_heads, int num_kv_heads, int head_dim,
@@ -1210,23 +1269,23 @@ int copy_blocks(pkv_tensor* k_cache, pkv_tensor* v_cache, const pkv_tensor* pair
   return launch_dependent(copy_blocks_kernel, grid, dim3(tpb), static_cast<cudaStream_t>(stream), p, ds->err);
 }
 
+
 int paged_attn_prefill(const pkv_tensor* q, const pkv_tensor* k_cache, const pkv_tensor* v_cache,
                        const pkv_tensor* block_tables, const pkv_tensor* context_lens,
                        const pkv_tensor* q_start, int max_q_tokens, int num_kv_heads, float scale,
                        int block_size, pkv_tensor* out, void* stream) {
-  // One new token per sequence (max_q_tokens 1 and as many query rows as
-  // sequences) is the decode step: the decode kernel serves it (q_start can
-  // then only be 0, 1, ..., S and is not read). Shapes the decode does not
-  // take go to the multi-token kernels.
-  if (q && block_tables && max_q_tokens == 1 && q->ndim == 3 && block_tables->ndim == 2 &&
-      q->shape[0] == block_tables->shape[0]) {
-    DecodeArgs a{q, k_cache, v_cache, nullptr, nullptr, block_tables, context_lens,
-                 num_kv_heads, scale, block_size, out};
-    const int st = launch_decode(a, false, nullptr, 0, true, static_cast<cudaStream_t>(stream));
-    if (st != PKV_ERR_UNSUPPORTED) return st;
-  }
-  return launch_prefill(q, k_cache, v_cache, block_tables, context_lens, q_start, max_q_tokens,
-                        num_kv_heads, scale, block_size, out, static_cast<cudaStream_t>(stream));
+  return prefill_or_decode(q, k_cache, v_cache, nullptr, nullptr, false, block_tables, context_lens,
+                           q_start, max_q_tokens, num_kv_heads, scale, block_size, out, stream);
+}
+
+int paged_attn_prefill_fp8(const pkv_tensor* q, const pkv_tensor* k_cache,
+                           const pkv_tensor* v_cache, const pkv_tensor* k_scale,
+                           const pkv_tensor* v_scale, const pkv_tensor* block_tables,
+                           const pkv_tensor* context_lens, const pkv_tensor* q_start,
+                           int max_q_tokens, int num_kv_heads, float scale, int block_size,
+                           pkv_tensor* out, void* stream) {
+  return prefill_or_decode(q, k_cache, v_cache, k_scale, v_scale, true, block_tables, context_lens,
+                           q_start, max_q_tokens, num_kv_heads, scale, block_size, out, stream);
 }
 
 int swap_out_blocks(const pkv_tensor* k_cache, const pkv_tensor* v_cache, const pkv_tensor* blocks,

@@ -22,6 +22,11 @@
 // cut into chunks of kv_chunk blocks, one CTA each, which leave fp32
 // partials (m, l, unnormalised O) per column, and prefill_merge_kernel folds
 // a row's chunks with the log-sum-exp rule.
+//
+// An fp8-e4m3 cache is read as the decode reads it: codes widened to f16 in
+// registers, q rounded to f16 (a bf16 row reaching 2^16 first scaled by a
+// power of two that its logit scale takes back), the K scale folded into the
+// logit scale and the V scale into the output (or the partials).
 #pragma once
 
 #include "cascade.cuh"
@@ -49,6 +54,8 @@ struct PrefillParams {
   float* part_o;    // [T * Hq * nkv][D] (split only)
   float* part_ml;   // [T * Hq * nkv][2]
   const int* order;  // [S] sequences by decreasing context length, or null (tensor-core kernels)
+  const float* k_scale;  // [Hk], fp8 caches only
+  const float* v_scale;
 };
 
 // order[r] = the sequence with the r-th longest context (ties: lower index
@@ -74,11 +81,12 @@ __global__ void __launch_bounds__(kOrderMaxSeqs) order_by_len_kernel(const int* 
   }
 }
 
-template <bool QBF, int D, int BS, int NS, int NW>
+template <bool QBF, int D, int BS, int NS, int NW, bool FP8 = false>
 struct PrefillCfg {
-  static constexpr int EPR = 64;
-  static constexpr int NH = (D * 2) / 128;
-  static constexpr int TILE = BS * D * 2;
+  static constexpr int EB = FP8 ? 1 : 2;     // cache element bytes
+  static constexpr int EPR = 128 / EB;       // elements per 128-byte row
+  static constexpr int NH = (D * EB) / 128;  // 128-byte column groups per token row
+  static constexpr int TILE = BS * D * EB;
   static constexpr int STAGE = 2 * TILE;
   static constexpr int KS = D / 16;
   static constexpr int MT = D / 16;
@@ -86,11 +94,12 @@ struct PrefillCfg {
   static constexpr int COLS = NW * 16;
   static constexpr int SMEM = 1024 + NS * STAGE + 2 * NS * 8;
   static_assert(D % 64 == 0 && BS % 16 == 0, "head_dim multiple of 64, block_size of 16");
+  static_assert(!FP8 || D == 128, "fp8 caches: head_dim 128");
 };
 
-template <bool QBF, int D, int BS, int NS, int NW>
+template <bool QBF, int D, int BS, int NS, int NW, bool FP8 = false>
 __global__ void __launch_bounds__(NW * 32, 1) prefill_kernel(const __grid_constant__ PrefillParams p) {
-  using C = PrefillCfg<QBF, D, BS, NS, NW>;
+  using C = PrefillCfg<QBF, D, BS, NS, NW, FP8>;
   constexpr uint64_t kWaitNs = 2000000000ull;
 
   extern __shared__ uint8_t smem_raw[];
@@ -181,22 +190,68 @@ __global__ void __launch_bounds__(NW * 32, 1) prefill_kernel(const __grid_consta
   }
 
   // Q^T fragments of this warp's columns; lane r carries column 8 jt + r.
+  // fp8: the widened tile's k-slots 2c, 2c + 1 hold dims 4c, 4c + 1 and
+  // slots 2c + 8, 2c + 9 dims 4c + 2, 4c + 3 of each 16-dim step; slj are
+  // the logit scales of this lane's two accumulator columns.
   const bool active = col0 + warp * 16 < cols;
   uint32_t qb[2][C::KS][2];
   int lim[2][2];  // positions of this lane's two accumulator columns per n-tile
   bool col_ok[2][2];
+  float slj[2][2];
+  const float sl_base = FP8 ? p.scale_log2 * __ldg(p.k_scale + h) : p.scale_log2;
 #pragma unroll
   for (int jt = 0; jt < 2; ++jt) {
     const int col = col0 + warp * 16 + jt * 8 + r;
     const bool ok = col < cols;
     const int tok = ok ? col / p.g : 0;
-    const uint32_t* qp = reinterpret_cast<const uint32_t*>(
-        static_cast<const uint16_t*>(p.q) + (q0 + tok) * p.q_t +
-        (static_cast<long long>(h) * p.g + (ok ? col % p.g : 0)) * p.q_h);
+    const long long qoff = (q0 + tok) * p.q_t + (static_cast<long long>(h) * p.g + (ok ? col % p.g : 0)) * p.q_h;
+    slj[jt][0] = slj[jt][1] = sl_base;
+    if constexpr (!FP8) {
+      const uint32_t* qp = reinterpret_cast<const uint32_t*>(static_cast<const uint16_t*>(p.q) + qoff);
 #pragma unroll
-    for (int ks = 0; ks < C::KS; ++ks) {
-      qb[jt][ks][0] = ok ? __ldg(qp + (ks * 16 + 2 * c) / 2) : 0u;
-      qb[jt][ks][1] = ok ? __ldg(qp + (ks * 16 + 8 + 2 * c) / 2) : 0u;
+      for (int ks = 0; ks < C::KS; ++ks) {
+        qb[jt][ks][0] = ok ? __ldg(qp + (ks * 16 + 2 * c) / 2) : 0u;
+        qb[jt][ks][1] = ok ? __ldg(qp + (ks * 16 + 8 + 2 * c) / 2) : 0u;
+      }
+    } else {
+      const uint2* qp = reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(p.q) + qoff);
+      float f[C::KS][4];
+      float amax = 0.f;
+#pragma unroll
+      for (int ks = 0; ks < C::KS; ++ks) {
+        const uint2 v = ok ? __ldg(qp + (ks * 16 + 4 * c) / 4) : make_uint2(0u, 0u);
+        if constexpr (QBF) {
+          f[ks][0] = __uint_as_float(v.x << 16);
+          f[ks][1] = __uint_as_float(v.x & 0xffff0000u);
+          f[ks][2] = __uint_as_float(v.y << 16);
+          f[ks][3] = __uint_as_float(v.y & 0xffff0000u);
+          amax = fmaxf(amax, fmaxf(fmaxf(fabsf(f[ks][0]), fabsf(f[ks][1])),
+                                   fmaxf(fabsf(f[ks][2]), fabsf(f[ks][3]))));
+        } else {
+          const __half2 a2 = *reinterpret_cast<const __half2*>(&v.x);
+          const __half2 b2 = *reinterpret_cast<const __half2*>(&v.y);
+          f[ks][0] = __low2float(a2);
+          f[ks][1] = __high2float(a2);
+          f[ks][2] = __low2float(b2);
+          f[ks][3] = __high2float(b2);
+        }
+      }
+      float qs = 1.f;
+      if constexpr (QBF) {  // the row of column 8 jt + r is held by lanes 4r .. 4r + 3
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        const int ex = static_cast<int>((__float_as_uint(amax) >> 23) & 0xffu) - 127;
+        const int e = ex >= 16 ? ex - 15 : 0;
+        qs = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+        const int e0 = __shfl_sync(0xffffffffu, e, 8 * c), e1 = __shfl_sync(0xffffffffu, e, 8 * c + 4);
+        slj[jt][0] = sl_base * __uint_as_float(static_cast<uint32_t>(127 + e0) << 23);
+        slj[jt][1] = sl_base * __uint_as_float(static_cast<uint32_t>(127 + e1) << 23);
+      }
+#pragma unroll
+      for (int ks = 0; ks < C::KS; ++ks) {
+        qb[jt][ks][0] = pack2<false>(f[ks][0] * qs, f[ks][1] * qs);
+        qb[jt][ks][1] = pack2<false>(f[ks][2] * qs, f[ks][3] * qs);
+      }
     }
     const int cb0 = col0 + warp * 16 + jt * 8 + 2 * c;
 #pragma unroll
@@ -216,7 +271,6 @@ __global__ void __launch_bounds__(NW * 32, 1) prefill_kernel(const __grid_consta
     mrun[jt][0] = mrun[jt][1] = -INFINITY;
     lrun[jt][0] = lrun[jt][1] = 0.f;
   }
-  const float sl = p.scale_log2;
   int jfail = nblk;
 
   for (int j = 0; j < nblk; ++j) {
@@ -238,18 +292,37 @@ __global__ void __launch_bounds__(NW * 32, 1) prefill_kernel(const __grid_consta
 #pragma unroll
         for (int jt = 0; jt < 2; ++jt) sacc[jt][0] = sacc[jt][1] = sacc[jt][2] = sacc[jt][3] = 0.f;
         const int trow = tt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+        if constexpr (!FP8) {
 #pragma unroll
-        for (int ks = 0; ks < C::KS; ++ks) {
-          uint32_t a0, a1, a2, a3;
-          ldsm_x4(tk + swz<BS>(trow, ks * 32 + (lane >> 4) * 16), a0, a1, a2, a3);
+          for (int ks = 0; ks < C::KS; ++ks) {
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(tk + swz<BS>(trow, ks * 32 + (lane >> 4) * 16), a0, a1, a2, a3);
 #pragma unroll
-          for (int jt = 0; jt < 2; ++jt) mma16816<QBF>(sacc[jt], a0, a1, a2, a3, qb[jt][ks][0], qb[jt][ks][1]);
+            for (int jt = 0; jt < 2; ++jt) mma16816<QBF>(sacc[jt], a0, a1, a2, a3, qb[jt][ks][0], qb[jt][ks][1]);
+          }
+        } else {
+#pragma unroll
+          for (int kp = 0; kp < C::KS / 2; ++kp) {
+            uint32_t x0, x1, x2, x3;
+            ldsm_x4(tk + swz<BS>(trow, kp * 32 + (lane >> 4) * 16), x0, x1, x2, x3);
+            uint32_t a0, a2, a1, a3, b0, b2, b1, b3;
+            e4m3x4_to_f16x2x2(x0, a0, a2);
+            e4m3x4_to_f16x2x2(x1, a1, a3);
+            e4m3x4_to_f16x2x2(x2, b0, b2);
+            e4m3x4_to_f16x2x2(x3, b1, b3);
+#pragma unroll
+            for (int jt = 0; jt < 2; ++jt) {
+              mma16816<false>(sacc[jt], a0, a1, a2, a3, qb[jt][2 * kp][0], qb[jt][2 * kp][1]);
+              mma16816<false>(sacc[jt], b0, b1, b2, b3, qb[jt][2 * kp + 1][0], qb[jt][2 * kp + 1][1]);
+            }
+          }
         }
         const int k0 = b * BS + tt * 16 + r, k1 = k0 + 8;  // keys of this lane's rows
         uint32_t pb[2][2];
 #pragma unroll
         for (int jt = 0; jt < 2; ++jt) {
-          float x0 = sacc[jt][0] * sl, x1 = sacc[jt][1] * sl, x2 = sacc[jt][2] * sl, x3 = sacc[jt][3] * sl;
+          float x0 = sacc[jt][0] * slj[jt][0], x1 = sacc[jt][1] * slj[jt][1];
+          float x2 = sacc[jt][2] * slj[jt][0], x3 = sacc[jt][3] * slj[jt][1];
           if (masked) {
             x0 = k0 <= lim[jt][0] ? x0 : -INFINITY;
             x1 = k0 <= lim[jt][1] ? x1 : -INFINITY;
@@ -283,25 +356,53 @@ __global__ void __launch_bounds__(NW * 32, 1) prefill_kernel(const __grid_consta
           const float p2 = exp2f(x2 - b0), p3 = exp2f(x3 - b1);
           lrun[jt][0] += p0 + p2;
           lrun[jt][1] += p1 + p3;
-          pb[jt][0] = movmatrix_t(pack2<QBF>(p0, p1));
-          pb[jt][1] = movmatrix_t(pack2<QBF>(p2, p3));
+          pb[jt][0] = movmatrix_t(pack2<QBF && !FP8>(p0, p1));
+          pb[jt][1] = movmatrix_t(pack2<QBF && !FP8>(p2, p3));
         }
         // V rows past the sequence's tokens zeroed (their P is 0, a NaN
         // there would still poison the sum)
         const int tb = tt * 16 + 2 * c;
         const uint32_t keep01 = (tb < nvalid ? 0x0000ffffu : 0u) | (tb + 1 < nvalid ? 0xffff0000u : 0u);
         const uint32_t keep23 = (tb + 8 < nvalid ? 0x0000ffffu : 0u) | (tb + 9 < nvalid ? 0xffff0000u : 0u);
+        if constexpr (!FP8) {
 #pragma unroll
-        for (int i = 0; i < C::MT; ++i) {
-          const int vrow = tt * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
-          uint32_t f0, f1, f2, f3;
-          ldsm_x4_t(tv + swz<BS>(vrow, i * 32 + ((lane >> 3) & 1) * 16), f0, f1, f2, f3);
-          f0 &= keep01;
-          f1 &= keep01;
-          f2 &= keep23;
-          f3 &= keep23;
+          for (int i = 0; i < C::MT; ++i) {
+            const int vrow = tt * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
+            uint32_t f0, f1, f2, f3;
+            ldsm_x4_t(tv + swz<BS>(vrow, i * 32 + ((lane >> 3) & 1) * 16), f0, f1, f2, f3);
+            f0 &= keep01;
+            f1 &= keep01;
+            f2 &= keep23;
+            f3 &= keep23;
 #pragma unroll
-          for (int jt = 0; jt < 2; ++jt) mma16816<QBF>(acc[jt][i], f0, f1, f2, f3, pb[jt][0], pb[jt][1]);
+            for (int jt = 0; jt < 2; ++jt) mma16816<QBF>(acc[jt][i], f0, f1, f2, f3, pb[jt][0], pb[jt][1]);
+          }
+        } else {  // one transposed load covers two m-tiles, widened to f16
+#pragma unroll
+          for (int i = 0; i < C::MT / 2; ++i) {
+            const int vrow = tt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+            uint32_t x0, x1, x2, x3, f[8];
+            ldsm_x4_t(tv + swz<BS>(vrow, i * 32 + (lane >> 4) * 16), x0, x1, x2, x3);
+            // bytes (d, t), (d + 1, t), (d, t + 1), (d + 1, t + 1) -> token
+            // pairs (d, t | t + 1) and (d + 1, t | t + 1)
+            e4m3x4_to_f16x2x2(prmt(x0, 0, 0x3120), f[0], f[1]);
+            e4m3x4_to_f16x2x2(prmt(x1, 0, 0x3120), f[2], f[3]);
+            e4m3x4_to_f16x2x2(prmt(x2, 0, 0x3120), f[4], f[5]);
+            e4m3x4_to_f16x2x2(prmt(x3, 0, 0x3120), f[6], f[7]);
+            f[0] &= keep01;
+            f[1] &= keep01;
+            f[2] &= keep23;
+            f[3] &= keep23;
+            f[4] &= keep01;
+            f[5] &= keep01;
+            f[6] &= keep23;
+            f[7] &= keep23;
+#pragma unroll
+            for (int jt = 0; jt < 2; ++jt) {
+              mma16816<false>(acc[jt][2 * i], f[0], f[1], f[2], f[3], pb[jt][0], pb[jt][1]);
+              mma16816<false>(acc[jt][2 * i + 1], f[4], f[5], f[6], f[7], pb[jt][0], pb[jt][1]);
+            }
+          }
         }
       }
     }
@@ -338,7 +439,8 @@ __global__ void __launch_bounds__(NW * 32, 1) prefill_kernel(const __grid_consta
       l0 += __shfl_xor_sync(0xffffffffu, l0, o);
       l1 += __shfl_xor_sync(0xffffffffu, l1, o);
     }
-    const float i0 = l0 > 0.f ? 1.f / l0 : 0.f, i1 = l1 > 0.f ? 1.f / l1 : 0.f;
+    const float vs = FP8 ? __ldg(p.v_scale + h) : 1.f;  // O carries the V scale
+    const float i0 = l0 > 0.f ? vs / l0 : 0.f, i1 = l1 > 0.f ? vs / l1 : 0.f;
     const int cb0 = col0 + warp * 16 + jt * 8 + 2 * c;
     if (p.nkv > 1) {  // partials of this KV chunk
 #pragma unroll
@@ -350,8 +452,10 @@ __global__ void __launch_bounds__(NW * 32, 1) prefill_kernel(const __grid_consta
         float* po = p.part_o + row * D;
 #pragma unroll
         for (int mt = 0; mt < C::MT; ++mt) {
-          po[16 * mt + r] = acc[jt][mt][u];
-          po[16 * mt + r + 8] = acc[jt][mt][u + 2];
+          const int da = FP8 ? 16 * mt + 2 * r : 16 * mt + r;
+          const int db = FP8 ? da + 1 : da + 8;
+          po[da] = acc[jt][mt][u] * vs;
+          po[db] = acc[jt][mt][u + 2] * vs;
         }
         if (r == 0) {
           p.part_ml[row * 2] = mrun[jt][u];
@@ -370,7 +474,8 @@ __global__ void __launch_bounds__(NW * 32, 1) prefill_kernel(const __grid_consta
 #pragma unroll
       for (int mt = 0; mt < C::MT; ++mt) {
         const float x = acc[jt][mt][u] * inv, y = acc[jt][mt][u + 2] * inv;
-        const int da = 16 * mt + r, db = da + 8;
+        const int da = FP8 ? 16 * mt + 2 * r : 16 * mt + r;
+        const int db = FP8 ? da + 1 : da + 8;
         if constexpr (QBF) {
           o[da] = __bfloat16_as_ushort(__float2bfloat16_rn(x));
           o[db] = __bfloat16_as_ushort(__float2bfloat16_rn(y));

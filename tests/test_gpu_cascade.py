@@ -6,6 +6,8 @@ a grouping, chunking or merge mistake shows up as an error against it.
 Layouts come from allocator runs (shared prompt, forks, private suffixes,
 copy-on-write of a partly filled shared block).
 """
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -63,7 +65,8 @@ def _run_cascade(s, lay, t, min_members=2):
     groups = P.PrefixGroups(lay.tables, lay.lens, s.block_size, min_members)
     out = torch.full_like(t.q, float("nan"))
     P.paged_attn_decode_cascade(t.q, t.k_cache, t.v_cache, lay.tables.cuda(), lay.lens.cuda(), groups,
-                                s.num_kv_heads, s.scale, s.block_size, out)
+                                s.num_kv_heads, s.scale, s.block_size, out,
+                                k_scale=t.k_scale, v_scale=t.v_scale)
     return out, groups
 
 
@@ -149,3 +152,53 @@ def test_cascade_bad_prefix_is_flagged():
                                 s.num_kv_heads, s.scale, s.block_size, out)
     assert P.device_error(torch.cuda.current_device()) == P.PKV_ERR_DEVICE_CHECK
     check_no_device_error()
+
+
+# fp8-e4m3 caches (paged_attn_decode_cascade_fp8): q dtype, Hq, Hk, B, groups, solo; D = 128
+FP8_CASES = {
+    "fp8_gqa_bf16q_b16": ("bf16", 32, 8, 16, [(300, [10, 20, 0, 64])], [500, 1]),
+    "fp8_g8_f16q_b32": ("f16", 64, 8, 32, [(257, [3, 40, 96]), (64, [0, 0, 33])], [90]),
+    "fp8_mha_many_members": ("bf16", 2, 2, 16, [(64, list(range(0, 140, 2)))], []),  # 3 column chunks
+    "fp8_long_prefix": ("bf16", 16, 4, 16, [(3000, [9, 100, 250])], [1000]),
+}
+
+
+def _fp8_spec(qd, Hq, Hk, B):
+    return W.spec("llama3_8b").replace(num_q_heads=Hq, num_kv_heads=Hk, head_dim=128, block_size=B,
+                                       cache_dtype="fp8_e4m3", q_dtype=qd, table_width=None)
+
+
+@pytest.mark.parametrize("name", list(FP8_CASES))
+def test_cascade_fp8_matches_oracle(name):
+    qd, Hq, Hk, B, groups, solo = FP8_CASES[name]
+    s, lay = _layout(_fp8_spec(qd, Hq, Hk, B), groups, solo, seed=sum(map(ord, name)))
+    t = W.make_tensors(s, lay.num_blocks, lay.fill_tables, lay.fill_lens, device="cuda", seed=9)
+    out, gr = _run_cascade(s, lay, t)
+    torch.cuda.synchronize()
+    check_no_device_error()
+    assert gr.num_groups == len(groups)
+    ref = oracle_decode(s, lay, t)
+    assert max_err(out, ref) <= TOL["fp8_e4m3"], name
+    plain = run_decode(s, lay, t)
+    torch.cuda.synchronize()
+    assert max_err(plain, ref) <= TOL["fp8_e4m3"]
+
+
+def test_cascade_fp8_bf16_q_rows_beyond_f16_range():
+    # Members' bf16 q rows of 2^17 and more: the prefix pass scales such a row
+    # by a power of two before rounding it to f16 and takes it back in the
+    # logit scale, as the decode does.
+    qd, Hq, Hk, B, groups, solo = FP8_CASES["fp8_gqa_bf16q_b16"]
+    s, lay = _layout(_fp8_spec(qd, Hq, Hk, B), groups, solo, seed=21)
+    t = W.make_tensors(s, lay.num_blocks, lay.fill_tables, lay.fill_lens, device="cuda", seed=23)
+    gr = P.PrefixGroups(lay.tables, lay.lens, s.block_size)
+    big = [int(x) for x in gr.members[:2]]
+    q = t.q.clone()
+    q[big[0]] *= 2.0 ** 17
+    q[big[1], :Hq // 2] *= 3.0e5
+    t = dataclasses.replace(t, q=q)
+    out, _ = _run_cascade(s, lay, t)
+    torch.cuda.synchronize()
+    check_no_device_error()
+    assert torch.isfinite(out.float()).all()
+    assert max_err(out, oracle_decode(s, lay, t)) <= TOL["fp8_e4m3"]

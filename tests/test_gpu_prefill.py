@@ -38,14 +38,17 @@ def _case(spec, nq, seed=5):
 def _run(s, lay, t, q, q_start, max_q):
     out = torch.full_like(q, float("nan"))
     P.paged_attn_prefill(q, t.k_cache, t.v_cache, lay.tables.cuda(), lay.lens.cuda(), q_start.cuda(), max_q,
-                         s.num_kv_heads, s.scale, s.block_size, out)
+                         s.num_kv_heads, s.scale, s.block_size, out, k_scale=t.k_scale, v_scale=t.v_scale)
     torch.cuda.synchronize()
     return out
 
 
 def _oracle(s, lay, t, q, q_start, seqs=None):
+    ks = None if t.k_scale is None else t.k_scale.cpu().numpy()
+    vs = None if t.v_scale is None else t.v_scale.cpu().numpy()
     return paged_prefill(raw(q), raw(t.k_cache), raw(t.v_cache), lay.tables.numpy(), lay.lens.numpy(),
-                         q_start.numpy(), s.scale, s.block_size, s.q_dtype, s.cache_dtype, seqs=seqs)
+                         q_start.numpy(), s.scale, s.block_size, s.q_dtype, s.cache_dtype,
+                         k_scale=ks, v_scale=vs, seqs=seqs)
 
 
 CASES = {
@@ -73,6 +76,15 @@ CASES = {
     "tc_half_tile": (W.spec("llama3_8b").replace(num_seqs=4, lens=("fixed", [200, 16, 77, 1000]),
                                                  table_width=None),
                      [16, 9, 1, 16]),
+    # fp8-e4m3 caches (paged_attn_prefill_fp8): the warp-MMA kernel at every
+    # row count, with and without the KV split
+    "fp8_verify_gqa": (W.scaled_down(W.spec("llama3_8b"), 8, 900, cache_dtype="fp8_e4m3"), [4] * 8),
+    "fp8_chunk_g8_b32": (W.spec("llama3_70b").replace(num_seqs=2, block_size=32, cache_dtype="fp8_e4m3",
+                                                      lens=("fixed", [900, 601]), table_width=None),
+                         [300, 129]),
+    "fp8_mixed_f16q": (W.spec("llama3_8b").replace(num_seqs=6, cache_dtype="fp8_e4m3", q_dtype="f16",
+                                                   lens=("fixed", [16, 17, 1, 500, 48, 2]), table_width=None),
+                       [16, 0, 1, 40, 33, 2]),
 }
 
 
@@ -148,3 +160,34 @@ def test_inconsistent_rows_are_flagged():
                          s.num_kv_heads, s.scale, s.block_size, out)
     assert P.device_error(torch.cuda.current_device()) == P.PKV_ERR_DEVICE_CHECK
     check_no_device_error()
+
+
+def test_fp8_one_token_per_sequence_is_the_fp8_decode_step():
+    spec = W.scaled_down(W.spec("long_skewed"), 8, 1500, cache_dtype="fp8_e4m3")
+    s, lay, t, q, q_start, max_q = _case(spec, [1] * 8)
+    out = _run(s, lay, t, q, q_start, max_q)
+    dec = torch.full_like(q, float("nan"))
+    P.paged_attn_decode_fp8(q, t.k_cache, t.v_cache, t.k_scale, t.v_scale, lay.tables.cuda(), lay.lens.cuda(),
+                            s.num_kv_heads, s.scale, s.block_size, dec)
+    torch.cuda.synchronize()
+    check_no_device_error()
+    assert (out.float() - dec.float()).abs().max().item() <= TOL["fp8_e4m3"]
+    assert max_err(out, _oracle(s, lay, t, q, q_start)) <= TOL["fp8_e4m3"]
+
+
+def test_fp8_bf16_q_rows_beyond_f16_range():
+    # bf16 query rows past the f16 maximum on an fp8 cache: each such row is
+    # scaled by a power of two before its f16 rounding (its logit scale takes
+    # it back), so the outputs stay finite and within tolerance
+    spec = W.scaled_down(W.spec("llama3_8b"), 4, 600, cache_dtype="fp8_e4m3")
+    s, lay, t, q, q_start, max_q = _case(spec, [5, 3, 8, 2])
+    q = q.float()
+    q[::2] *= 2.5e4
+    q[1, 3] = 0.0
+    q[1, 3, 5] = -1.2e5
+    q = q.to(torch.bfloat16)
+    assert q.float().abs().max() > 65504
+    out = _run(s, lay, t, q, q_start, max_q)
+    check_no_device_error()
+    assert torch.isfinite(out.float()).all()
+    assert max_err(out, _oracle(s, lay, t, q, q_start)) <= TOL["fp8_e4m3"]
