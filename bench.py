@@ -503,7 +503,8 @@ def run_prefill(a, s: W.Spec):
     q = torch.randn((T, s.num_q_heads, s.head_dim), generator=g, device="cuda:0").to(t.q.dtype)
     out = torch.empty_like(q)
     call = P.prepare_prefill(q, t.k_cache, t.v_cache, lay.tables.cuda(), lay.lens.cuda(), q_start.cuda(),
-                             max(nq), s.num_kv_heads, s.scale, s.block_size, out)
+                             max(nq), s.num_kv_heads, s.scale, s.block_size, out,
+                             k_scale=t.k_scale, v_scale=t.v_scale)
     kv = kv_bytes_of(s, lens)
     alg = kv + 2 * T * s.num_q_heads * s.head_dim * 2 + sum(-(-L // s.block_size) for L in lens) * 4 + 8 * s.num_seqs
     keys = sum(sum(L - n + j + 1 for j in range(n)) for L, n in zip(lens, nq))
@@ -530,7 +531,7 @@ def run_prefill(a, s: W.Spec):
     # that launch is bound by the MMAs, the others by the KV bytes
     g = s.num_q_heads // s.num_kv_heads
     cols = max(nq) * g
-    tc = s.head_dim == 128 and cols >= 64 and s.scale > 0
+    tc = s.cache_dtype != "fp8_e4m3" and s.head_dim == 128 and cols >= 64 and s.scale > 0
     # kernels one call launches: the tensor-core kernel (after the one-CTA
     # longest-first ordering pass when 1 < S <= 1024 and the grid is more
     # than one wave), or the warp-MMA
@@ -636,7 +637,8 @@ def main():
             g = P.PrefixGroups.on_device(b.d("prefix_blocks"), b.d("group_start"), b.d("members"),
                                          groups.num_groups, groups.max_group_size, groups.max_prefix_blocks)
             decode = P.prepare_decode_cascade(b.d("q"), t.k_cache, t.v_cache, b.d("tables"), b.d("lens"), g,
-                                              s.num_kv_heads, s.scale, s.block_size, out)
+                                              s.num_kv_heads, s.scale, s.block_size, out,
+                                              k_scale=t.k_scale, v_scale=t.v_scale)
         else:
             decode = P.prepare_decode(b.d("q"), t.k_cache, t.v_cache, b.d("tables"), b.d("lens"), s.num_kv_heads,
                                       s.scale, s.block_size, out, t.k_scale, t.v_scale)
