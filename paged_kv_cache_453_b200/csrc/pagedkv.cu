@@ -278,7 +278,7 @@ WsLayout ws_layout(int sms, int nwt, int g, int D, int pool_slots) {
   l.steal = round_up(l.words + cap * 8, 256);
   l.desc = round_up(l.steal + cap * kMaxSteals * 16, 256);
   l.rlo = round_up(l.desc + cap * (1 + kMaxSteals) * 16, 256);
-  // adaptive partition: its nwt word, then part, speed and wgt [cap] each
+  // adaptive partition: its nwt word, then part, rtime and wgt [cap] each
   l.adapt = round_up(l.rlo + (cap + 1) * 8, 256);
   l.cap = cap;
   l.part_o = round_up(l.adapt + 16 + cap * 12, 256);
@@ -1075,11 +1075,12 @@ using namespace pkv;
 // sequences) is the decode step: the decode kernel serves it (q_start can
 // then only be 0, 1, ..., S and is not read). Shapes the decode does not take
 // go to the multi-token kernels.
-static int prefill_or_decode(const pkv_tensor* q, const pkv_tensor* k_cache, const pkv_tensor* v_cache,
-                      const pkv_tensor* k_scale, const pkv_tensor* v_scale, bool fp8,
-                      const pkv_tensor* block_tables, const pkv_tensor* context_lens,
-                      const pkv_tensor* q_start, int max_q_tokens, int num_kv_heads, float scale,
-                      int block_size, pkv_tensor* out, void* stream) {
+static int prefill_or_decode(const pkv_tensor* q, const pkv_tensor* k_cache,
+                             const pkv_tensor* v_cache, const pkv_tensor* k_scale,
+                             const pkv_tensor* v_scale, bool fp8, const pkv_tensor* block_tables,
+                             const pkv_tensor* context_lens, const pkv_tensor* q_start,
+                             int max_q_tokens, int num_kv_heads, float scale, int block_size,
+                             pkv_tensor* out, void* stream) {
   if (q && block_tables && max_q_tokens == 1 && q->ndim == 3 && block_tables->ndim == 2 &&
       q->shape[0] == block_tables->shape[0]) {
     DecodeArgs a{q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
