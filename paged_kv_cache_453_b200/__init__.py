@@ -271,7 +271,9 @@ def prepare_decode_cascade(q, k_cache, v_cache, block_tables, context_lens, grou
     args = tuple(ctypes.byref(d) for d in ds) + (
         groups.num_groups, groups.max_group_size, groups.max_prefix_blocks, int(num_kv_heads),
         float(scale), int(block_size), ctypes.byref(do))
-    return Prepared(name, getattr(lib(), name), args, (ds, do, groups), stream)
+    return Prepared(name, getattr(lib(), name), args,
+                    (ds, do, groups, (q, k_cache, v_cache, block_tables, context_lens, out, k_scale, v_scale)),
+                    stream)
 
 
 def _prefill_descs(q, k_cache, v_cache, block_tables, context_lens, q_start, out, k_scale, v_scale):
@@ -303,7 +305,9 @@ def prepare_prefill(q, k_cache, v_cache, block_tables, context_lens, q_start, ma
                                   k_scale, v_scale)
     args = tuple(ctypes.byref(d) for d in ds) + (int(max_q_tokens), int(num_kv_heads), float(scale),
                                                  int(block_size), ctypes.byref(do))
-    return Prepared(name, getattr(lib(), name), args, (ds, do), stream)
+    return Prepared(name, getattr(lib(), name), args,
+                    (ds, do, (q, k_cache, v_cache, block_tables, context_lens, q_start, out, k_scale, v_scale)),
+                    stream)
 
 
 def swap_record_bytes(k_cache) -> int:
@@ -615,7 +619,8 @@ class BlockAllocator:
 class Prepared:
     """A device call with its descriptors built once (argument marshalling
     only); calling it enqueues the kernels on `stream` (default: torch's
-    current stream at preparation time)."""
+    current stream at preparation time). It keeps the tensors it was built
+    from alive, so their device memory cannot be reused under it."""
 
     def __init__(self, name: str, fn, args, keep, stream=None):
         self._name, self._fn, self._args, self._keep = name, fn, args, keep
@@ -633,6 +638,7 @@ def prepare_decode(q, k_cache, v_cache, block_tables, context_lens, num_kv_heads
     fp8 = k_scale is not None
     ds = [_desc(q), _desc(k_cache, fp8), _desc(v_cache, fp8), _desc(block_tables), _desc(context_lens),
           _desc(out)]
+    tensors = (q, k_cache, v_cache, block_tables, context_lens, out, k_scale, v_scale)
     L = lib()
     if workspace is not None or fp8:
         ks = _desc(k_scale) if fp8 else None
@@ -641,17 +647,17 @@ def prepare_decode(q, k_cache, v_cache, block_tables, context_lens, num_kv_heads
             args = (ctypes.byref(ds[0]), ctypes.byref(ds[1]), ctypes.byref(ds[2]), ctypes.byref(ks),
                     ctypes.byref(vs), ctypes.byref(ds[3]), ctypes.byref(ds[4]), int(num_kv_heads),
                     float(scale), int(block_size), ctypes.byref(ds[5]))
-            return Prepared("paged_attn_decode_fp8", L.paged_attn_decode_fp8, args, (ds, ks, vs), stream)
+            return Prepared("paged_attn_decode_fp8", L.paged_attn_decode_fp8, args, (ds, ks, vs, tensors), stream)
         args = (ctypes.byref(ds[0]), ctypes.byref(ds[1]), ctypes.byref(ds[2]),
                 ctypes.byref(ks) if fp8 else None, ctypes.byref(vs) if fp8 else None,
                 ctypes.byref(ds[3]), ctypes.byref(ds[4]), int(num_kv_heads), float(scale),
                 int(block_size), ctypes.byref(ds[5]), ctypes.c_void_p(workspace.data_ptr()),
                 workspace.numel() * workspace.element_size(), int(flags))
-        return Prepared("paged_attn_decode_ex", L.paged_attn_decode_ex, args, (ds, ks, vs, workspace),
+        return Prepared("paged_attn_decode_ex", L.paged_attn_decode_ex, args, (ds, ks, vs, workspace, tensors),
                         stream)
     args = (ctypes.byref(ds[0]), ctypes.byref(ds[1]), ctypes.byref(ds[2]), ctypes.byref(ds[3]),
             ctypes.byref(ds[4]), int(num_kv_heads), float(scale), int(block_size), ctypes.byref(ds[5]))
-    return Prepared("paged_attn_decode", L.paged_attn_decode, args, ds, stream)
+    return Prepared("paged_attn_decode", L.paged_attn_decode, args, (ds, tensors), stream)
 
 
 def prepare_reshape(k, v, k_cache, v_cache, slot_mapping, k_scale=None, v_scale=None,
@@ -662,13 +668,15 @@ def prepare_reshape(k, v, k_cache, v_cache, slot_mapping, k_scale=None, v_scale=
     if fp8:
         ds += [_desc(k_scale), _desc(v_scale)]
         return Prepared("reshape_and_cache_fp8", L.reshape_and_cache_fp8,
-                        tuple(ctypes.byref(d) for d in ds), ds, stream)
-    return Prepared("reshape_and_cache", L.reshape_and_cache, tuple(ctypes.byref(d) for d in ds), ds,
-                    stream)
+                        tuple(ctypes.byref(d) for d in ds),
+                        (ds, (k, v, k_cache, v_cache, slot_mapping, k_scale, v_scale)), stream)
+    return Prepared("reshape_and_cache", L.reshape_and_cache, tuple(ctypes.byref(d) for d in ds),
+                    (ds, (k, v, k_cache, v_cache, slot_mapping)), stream)
 
 
 def prepare_copy_blocks(k_cache, v_cache, pairs, stream=None) -> Prepared:
     import torch
     fp8 = k_cache.dtype in (torch.uint8, torch.float8_e4m3fn)
     ds = [_desc(k_cache, fp8), _desc(v_cache, fp8), _desc(pairs)]
-    return Prepared("copy_blocks", lib().copy_blocks, tuple(ctypes.byref(d) for d in ds), ds, stream)
+    return Prepared("copy_blocks", lib().copy_blocks, tuple(ctypes.byref(d) for d in ds),
+                    (ds, (k_cache, v_cache, pairs)), stream)

@@ -28,3 +28,27 @@ def test_step_buffers_round_trip_and_alignment():
         assert v.dtype == x.dtype and tuple(v.shape) == tuple(x.shape)
         assert torch.equal(v, x), k
         assert (v.data_ptr() - b.dev.data_ptr()) % bench.StepBuffers.ALIGN == 0, k
+
+
+def test_prepared_calls_keep_their_tensors_alive():
+    # A prepared call holds raw device pointers; it must also hold the tensors
+    # (a temporary such as tables.cuda() passed inline would otherwise be freed
+    # and its memory reused under the call). Checked on CPU with the
+    # constructor's bookkeeping only: no device call is made.
+    import gc
+    import weakref
+    import torch
+    import paged_kv_cache_453_b200 as P
+
+    class T(torch.Tensor):  # a tensor subclass can be weakly referenced
+        pass
+
+    x = torch.zeros(4).as_subclass(T)
+    ref = weakref.ref(x)
+    call = P.Prepared("noop", lambda *a: 0, (), (None, (x,)), stream=0)  # stream 0: no CUDA query
+    del x
+    gc.collect()
+    assert ref() is not None, "Prepared dropped a tensor it was built from"
+    del call
+    gc.collect()
+    assert ref() is None
