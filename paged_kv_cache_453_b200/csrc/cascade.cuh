@@ -313,7 +313,7 @@ __global__ void __launch_bounds__(128, 1) cascade_prefix_kernel(const __grid_con
           mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
         }
         const float mn0 = fmaxf(mrun[jt][0], mx0), mn1 = fmaxf(mrun[jt][1], mx1);
-        const float al0 = exp2f(mrun[jt][0] - mn0), al1 = exp2f(mrun[jt][1] - mn1);
+        const float al0 = ex2_fast(mrun[jt][0] - mn0), al1 = ex2_fast(mrun[jt][1] - mn1);
         lrun[jt][0] *= al0;
         lrun[jt][1] *= al1;
 #pragma unroll
@@ -325,8 +325,8 @@ __global__ void __launch_bounds__(128, 1) cascade_prefix_kernel(const __grid_con
         }
         mrun[jt][0] = mn0;
         mrun[jt][1] = mn1;
-        const float p0 = exp2f(x0 - mn0), p1 = exp2f(x1 - mn1);
-        const float p2 = exp2f(x2 - mn0), p3 = exp2f(x3 - mn1);
+        const float p0 = ex2_fast(x0 - mn0), p1 = ex2_fast(x1 - mn1);
+        const float p2 = ex2_fast(x2 - mn0), p3 = ex2_fast(x3 - mn1);
         lrun[jt][0] += p0 + p2;
         lrun[jt][1] += p1 + p3;
         pb[jt][0] = movmatrix_t(pack2<QBF && !FP8>(p0, p1));

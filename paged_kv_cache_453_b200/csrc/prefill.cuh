@@ -340,7 +340,7 @@ __global__ void __launch_bounds__(NW * 32, 1) prefill_kernel(const __grid_consta
           // base is then 0 instead of -inf.
           const float mn0 = fmaxf(mrun[jt][0], mx0), mn1 = fmaxf(mrun[jt][1], mx1);
           const float b0 = mn0 == -INFINITY ? 0.f : mn0, b1 = mn1 == -INFINITY ? 0.f : mn1;
-          const float al0 = exp2f(mrun[jt][0] - b0), al1 = exp2f(mrun[jt][1] - b1);
+          const float al0 = ex2_fast(mrun[jt][0] - b0), al1 = ex2_fast(mrun[jt][1] - b1);
           lrun[jt][0] *= al0;
           lrun[jt][1] *= al1;
 #pragma unroll
@@ -352,8 +352,8 @@ __global__ void __launch_bounds__(NW * 32, 1) prefill_kernel(const __grid_consta
           }
           mrun[jt][0] = mn0;
           mrun[jt][1] = mn1;
-          const float p0 = exp2f(x0 - b0), p1 = exp2f(x1 - b1);
-          const float p2 = exp2f(x2 - b0), p3 = exp2f(x3 - b1);
+          const float p0 = ex2_fast(x0 - b0), p1 = ex2_fast(x1 - b1);
+          const float p2 = ex2_fast(x2 - b0), p3 = ex2_fast(x3 - b1);
           lrun[jt][0] += p0 + p2;
           lrun[jt][1] += p1 + p3;
           pb[jt][0] = movmatrix_t(pack2<QBF && !FP8>(p0, p1));

@@ -142,14 +142,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
-// 2^x by the hardware approximation (ex2.approx.ftz): 2^-inf = +0; P is
-// rounded to 16 bits right after, far coarser than its error
-__device__ __forceinline__ float ex2_fast(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
 template <int BS>
 struct PrefillTcCfg {
   static constexpr int D = 128;

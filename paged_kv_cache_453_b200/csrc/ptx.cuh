@@ -122,6 +122,22 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
 // Four e4m3 codes (bytes 0..3) to two f16x2 (exact: every e4m3 value is an
 // f16 value): lo = (byte 0, byte 1), hi = (byte 2, byte 3), the lower byte
 // the first element; the register's halves feed the conversions directly.
+// 2^x by the hardware approximation (ex2.approx.ftz), one instruction:
+// 2^-inf = +0, results below 2^-126 flush to +0. The softmax weights it
+// makes are rounded to 16 bits before their products, far coarser than its
+// error, and a weight below 2^-126 of the running maximum's is nothing
+// against the sum that holds that maximum's weight.
+__device__ __forceinline__ float ex2_fast(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// 2^x by ex2_fast where FAST, else by exp2f
+template <bool FAST>
+__device__ __forceinline__ float ex2(float x) {
+  if constexpr (FAST) return ex2_fast(x);
+  else return exp2f(x);
+}
 __device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t v, uint32_t& lo, uint32_t& hi) {
   asm("{\n\t.reg .b16 l, h;\n\t"
       "mov.b32 {l, h}, %2;\n\t"

@@ -282,3 +282,46 @@ def test_fp8_adaptive_partition_across_shapes():
     torch.cuda.synchronize()
     check_no_device_error()
     assert torch.equal(det0.view(torch.int16), det1.view(torch.int16))
+
+
+@pytest.mark.parametrize("block_size", [16, 32])
+def test_fp8_logits_climbing_and_jumping_along_the_context(block_size):
+    # The fp8 decode moves a column's exponent base only when a score passes
+    # it by more than 8, so its softmax weights reach 2^8 between moves. Keys
+    # whose logits climb along the context (about 60 in the exp2 domain from
+    # first to last token: many moves, weights up to 2^8 in between) and, on
+    # every other sequence, a jump of about 30 over the last tenth of the
+    # context (O rescaled late) must still match the oracle.
+    from oracle.numerics import encode_e4m3
+    s, lay, t = decode_case(W.scaled_down(W.spec("long_skewed"), 6, 3000, cache_dtype="fp8_e4m3",
+                                          block_size=block_size), seed=91)
+    g, Hk, B = s.num_q_heads // s.num_kv_heads, s.num_kv_heads, s.block_size
+    ks = t.k_scale.cpu().numpy().astype(np.float64)
+    log2e = 1.0 / np.log(2.0)
+    # q = (A_h, 0, ..., 0): the exp2-domain logit of a key is A_h * scale *
+    # k_scale[h] * log2(e) * K[0], and K[0] = 448 (the e4m3 maximum) maps to 60
+    amp = 60.0 / (448.0 * s.scale * ks * log2e)
+    q = torch.zeros(t.q.shape, dtype=torch.float32)
+    for hq in range(s.num_q_heads):
+        q[:, hq, 0] = float(amp[hq // g])
+    t.q.copy_(q.to(t.q.dtype))
+    kc = t.k_cache.cpu().numpy()
+    tables, lens = lay.tables.numpy(), lay.lens.numpy()
+    for si in range(s.num_seqs):
+        L = int(lens[si])
+        if L == 0:
+            continue
+        j = np.arange(L)
+        if si % 2 == 0:
+            val = 448.0 * j / max(L - 1, 1)
+        else:
+            val = np.where(j >= int(0.9 * L), 448.0, 224.0 * j / max(L - 1, 1))
+        codes = encode_e4m3(val)
+        phys = tables[si, j // B]
+        for h in range(Hk):
+            kc[phys, h, j % B, 0] = codes
+    t.k_cache.copy_(torch.from_numpy(kc))
+    out = run_decode(s, lay, t)
+    torch.cuda.synchronize()
+    check_no_device_error()
+    assert max_err(out, oracle_decode(s, lay, t)) <= TOL["fp8_e4m3"]
