@@ -55,6 +55,10 @@ enum CacheKind : int { kCacheF16 = 0, kCacheBF16 = 1, kCacheE4M3 = 2 };
 constexpr int kMaxSteals = 6;     // steals from one warp's range per call
 constexpr int kMinStealable = 4;  // a remainder worth splitting (items)
 constexpr int kStealMax = 8;      // items one steal takes at most
+// The merge's CTA 0 keeps each of its threads' ranges of the adaptive
+// partition in registers: at most this many per thread (grids of up to
+// 128 x kAdaptPer warps).
+constexpr int kAdaptPer = 16;
 constexpr int kStealTries = 8;
 constexpr int kScanBatch = 4;     // range words each lane loads when choosing a victim (a window of 128)
 constexpr int kMergeAhead = 8;    // ranges whose steal records the merge reads in its first round
@@ -1407,7 +1411,8 @@ __global__ void __launch_bounds__(128, 8) decode_merge_kernel(const __grid_const
   // range without a time keeps its weight.
   if (blockIdx.x == 0 && p.adapt && p.steal) {
     const int n = p.nwt;
-    const int per = (n + NT - 1) / NT;
+    const int per = (n + NT - 1) / NT;  // at most kAdaptPer: the host enables adapt only then
+    if (per > kAdaptPer) return;
     const int va = min(n, tid * per), vb = min(n, va + per);
     const bool have = __ldcg(p.part_nwt) == n;
     double* sd = reinterpret_cast<double*>(s_red);  // [NT / 32] per-warp sums
@@ -1431,11 +1436,19 @@ __global__ void __launch_bounds__(128, 8) decode_merge_kernel(const __grid_const
       }
     };
     auto valid_time = [](float v) { return v > 0.f && v < 1e9f; };
+    // this thread's ranges in registers, every load in flight at once
+    float sp[kAdaptPer], w[kAdaptPer];
+#pragma unroll
+    for (int k = 0; k < kAdaptPer; ++k) {
+      const bool in = va + k < vb;
+      sp[k] = in ? __ldcg(p.rtime + va + k) : 0.f;
+      w[k] = in && have ? __ldcg(p.wgt + va + k) : 1.f;
+    }
     double ssum = 0.0, scnt = 0.0, dummy, st, ct;
-    for (int v = va; v < vb; ++v) {
-      const float sp = p.rtime[v];
-      if (valid_time(sp)) {
-        ssum += sp;
+#pragma unroll
+    for (int k = 0; k < kAdaptPer; ++k) {
+      if (va + k < vb && valid_time(sp[k])) {
+        ssum += sp[k];
         scnt += 1.0;
       }
     }
@@ -1443,29 +1456,36 @@ __global__ void __launch_bounds__(128, 8) decode_merge_kernel(const __grid_const
     block_scan(scnt, dummy, ct);
     const float mean = ct > 0.0 ? static_cast<float>(st / ct) : 0.f;
     double wsum = 0.0;
-    for (int v = va; v < vb; ++v) {
-      float wo = have ? p.wgt[v] : 1.f;
-      if (!(wo >= 0.5f && wo <= 2.f)) wo = 1.f;
-      const float sp = p.rtime[v];
-      const float w = (mean > 0.f && valid_time(sp)) ? wo * (0.5f + 0.5f * (mean / sp)) : wo;
-      p.wgt[v] = w;
-      wsum += w;
+#pragma unroll
+    for (int k = 0; k < kAdaptPer; ++k) {
+      if (va + k < vb) {
+        float wo = w[k];
+        if (!(wo >= 0.5f && wo <= 2.f)) wo = 1.f;
+        w[k] = (mean > 0.f && valid_time(sp[k])) ? wo * (0.5f + 0.5f * (mean / sp[k])) : wo;
+        wsum += w[k];
+      }
     }
     double wtot;
     block_scan(wsum, dummy, wtot);
     const float wscale = wtot > 0.0 ? static_cast<float>(n / wtot) : 1.f;
     wsum = 0.0;
-    for (int v = va; v < vb; ++v) {
-      const float w = fminf(fmaxf(p.wgt[v] * wscale, 0.5f), 2.f);
-      p.wgt[v] = w;
-      wsum += w;
+#pragma unroll
+    for (int k = 0; k < kAdaptPer; ++k) {
+      if (va + k < vb) {
+        w[k] = fminf(fmaxf(w[k] * wscale, 0.5f), 2.f);
+        wsum += w[k];
+      }
     }
     double run, total;
     block_scan(wsum, run, total);
-    for (int v = va; v < vb; ++v) {
-      const double f = run / total * 4294967296.0;
-      p.part_w[v] = f >= 4294967295.0 ? 4294967295u : static_cast<unsigned>(f);
-      run += p.wgt[v];
+#pragma unroll
+    for (int k = 0; k < kAdaptPer; ++k) {
+      if (va + k < vb) {
+        const double f = run / total * 4294967296.0;
+        p.part_w[va + k] = f >= 4294967295.0 ? 4294967295u : static_cast<unsigned>(f);
+        p.wgt[va + k] = w[k];
+        run += w[k];
+      }
     }
     if (tid == 0) *p.part_nwt_w = n;
   }

@@ -446,7 +446,7 @@ int launch_decode(const DecodeArgs& a, bool fp8, void* ws, size_t ws_bytes, bool
   // kernels are HBM-bound; their speed differences follow the SMs the CTAs
   // land on, which change between calls, and equal ranges plus stealing do
   // better there.
-  p.adapt = fp8 && !fixed_split ? 1 : 0;
+  p.adapt = fp8 && !fixed_split && nwt <= 128 * kAdaptPer ? 1 : 0;
   p.pool_slots = L.pool_slots;
   uint8_t* w = static_cast<uint8_t*>(ws);
   p.hdr = reinterpret_cast<long long*>(w + L.hdr);
