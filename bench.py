@@ -485,6 +485,23 @@ def run_swap(a, s: W.Spec):
     }))
 
 
+def prefill_roofline(flops: float, alg_bytes: float, sec: float, tensor_peak, hbm_peak) -> dict:
+    """Roofline of a tensor-core multi-token launch: bound by whichever of
+    its FLOPs at the tensor peak and its algorithmic bytes at the HBM peak
+    takes longer (few new tokens per sequence: HBM; many: the MMAs). The
+    other side's fraction is reported beside it."""
+    (tp, tsrc), (hp, hsrc) = tensor_peak, hbm_peak
+    t_tensor = flops / (tp * 1e12)
+    t_hbm = alg_bytes / (hp * 1e9)
+    f_tensor = flops / sec / 1e12 / tp
+    f_hbm = alg_bytes / sec / 1e9 / hp
+    if t_hbm >= t_tensor:
+        return {"bound": "hbm", "achieved": alg_bytes / sec / 1e9, "peak": hp, "unit": "GB/s", "frac": f_hbm,
+                "peak_source": hsrc, "tensor_frac": f_tensor, "tensor_peak": tp}
+    return {"bound": "tensor", "achieved": flops / sec / 1e12, "peak": tp, "unit": "TFLOP/s", "frac": f_tensor,
+            "peak_source": tsrc + " (bf16 burst)", "hbm_frac": f_hbm, "hbm_peak": hp}
+
+
 def run_prefill(a, s: W.Spec):
     """Causal attention of --q-tokens new tokens per sequence (the last ones of
     each context) over the workload's paged cache, inputs resident."""
@@ -550,12 +567,10 @@ def run_prefill(a, s: W.Spec):
         sms = torch.cuda.get_device_properties(0).multi_processor_count
         per_call = 1 + (1 if s.num_seqs * s.num_kv_heads * ncc < 4 * sms and lay.tables.shape[1] > 32 else 0)
     if tc and not decode_step:
-        peak, src = measured_peak_bf16()
         kern = "prefill_tc2_kernel" if cols > 128 else "prefill_tc_kernel"
-        roof = {"kernel": kern, "bound": "tensor", "achieved": flops / sec / 1e12, "peak": peak,
-                "unit": "TFLOP/s", "frac": flops / sec / 1e12 / peak, "peak_source": src + " (bf16 burst)",
-                "traffic": prefill_traffic(s, a.q_tokens, kern), "alg_bytes_per_launch": alg,
-                "flops_per_launch": flops}
+        roof = prefill_roofline(flops, alg, sec, measured_peak_bf16(), measured_peak_hbm())
+        roof.update({"kernel": kern, "traffic": prefill_traffic(s, a.q_tokens, kern),
+                     "alg_bytes_per_launch": alg, "flops_per_launch": flops})
     else:
         peak, src = measured_peak_hbm()
         roof = {"kernel": "decode_kernel + decode_merge_kernel" if decode_step else "prefill_kernel",

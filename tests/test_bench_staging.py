@@ -52,3 +52,18 @@ def test_prepared_calls_keep_their_tensors_alive():
     del call
     gc.collect()
     assert ref() is None
+
+
+def test_prefill_roofline_takes_the_binding_bound():
+    # 16 new tokens x 4 heads on the llama3_8b batch: ~40 GFLOP against
+    # ~648 MB, so the bytes at the HBM peak take longer than the FLOPs at the
+    # tensor peak; at 512 new tokens the MMAs bind.
+    hbm, tensor = (6650.0, "fallback"), (1590.0, "fallback")
+    r = bench.prefill_roofline(40.3e9, 648e6, 132e-6, tensor, hbm)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert abs(r["frac"] - 648e6 / 132e-6 / 1e9 / 6650.0) < 1e-12
+    assert abs(r["tensor_frac"] - 40.3e9 / 132e-6 / 1e12 / 1590.0) < 1e-12
+    r = bench.prefill_roofline(1.29e12, 1.1e9, 1.45e-3, tensor, hbm)
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert abs(r["frac"] - 1.29e12 / 1.45e-3 / 1e12 / 1590.0) < 1e-12
+    assert r["hbm_frac"] < r["frac"]
