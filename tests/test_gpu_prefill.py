@@ -85,6 +85,13 @@ CASES = {
     "fp8_mixed_f16q": (W.spec("llama3_8b").replace(num_seqs=6, cache_dtype="fp8_e4m3", q_dtype="f16",
                                                    lens=("fixed", [16, 17, 1, 500, 48, 2]), table_width=None),
                        [16, 0, 1, 40, 33, 2]),
+    # fp8 with several warps per CTA: 16 tokens x 4 heads over long contexts
+    # (4 warps, KV split), and 2 warps on 32-token blocks with partly filled
+    # last blocks
+    "fp8_q16_split": (W.scaled_down(W.spec("llama3_8b"), 6, 2500, cache_dtype="fp8_e4m3"), [16] * 6),
+    "fp8_q8_b32": (W.spec("llama3_8b").replace(num_seqs=3, block_size=32, cache_dtype="fp8_e4m3",
+                                               lens=("fixed", [70, 33, 300]), table_width=None),
+                   [8, 5, 8]),
 }
 
 
