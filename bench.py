@@ -417,7 +417,8 @@ def run_reference(a, s: W.Spec, ws: int, rank: int):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws,
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * tot_t / max(1, a.steps),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": config_of(s, lay, kv_bytes_of(s, lay.lens.tolist())),
+        "data": "synthetic",
+        "config": config_of(s, lay, kv_bytes_of(s, lay.lens.tolist())) | {"parallelism": f"replicas x{ws}"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": _blas_threads(), "host_cores": _host_cores(),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
