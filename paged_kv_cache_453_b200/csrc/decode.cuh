@@ -830,12 +830,11 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
         float mx0 = -INFINITY, mx1 = -INFINITY;
         if constexpr (FP8) {
 #pragma unroll
+          const uint64_t sl2 = f2_pack(sl0, sl1);  // (columns 2c, 2c + 1) pairs: packed f32x2
           for (int tt = 0; tt < C::TT; ++tt) {
             if (full) {
-              sacc[tt][0] *= sl0;
-              sacc[tt][1] *= sl1;
-              sacc[tt][2] *= sl0;
-              sacc[tt][3] *= sl1;
+              f2_unpack(f2_mul(f2_pack(sacc[tt][0], sacc[tt][1]), sl2), sacc[tt][0], sacc[tt][1]);
+              f2_unpack(f2_mul(f2_pack(sacc[tt][2], sacc[tt][3]), sl2), sacc[tt][2], sacc[tt][3]);
             } else {
               const int t0 = tt * 16 + r, t1 = t0 + 8;
               sacc[tt][0] = t0 < nvalid ? sacc[tt][0] * sl0 : -INFINITY;
@@ -907,10 +906,25 @@ __global__ void __launch_bounds__(NC * 32, 1) decode_kernel(const __grid_constan
         uint32_t pb[C::TT][2];
 #pragma unroll
         for (int tt = 0; tt < C::TT; ++tt) {
-          const float p0 = ex2<FP8>(sacc[tt][0] - m0), p1 = ex2<FP8>(sacc[tt][1] - m1);
-          const float p2 = ex2<FP8>(sacc[tt][2] - m0), p3 = ex2<FP8>(sacc[tt][3] - m1);
-          l0 += p0 + p2;
-          l1 += p1 + p3;
+          float p0, p1, p2, p3;
+          if constexpr (FP8) {  // exponent arguments and row sums as packed pairs
+            const uint64_t nm2 = f2_pack(-m0, -m1);
+            float a0, a1, a2, a3;
+            f2_unpack(f2_add(f2_pack(sacc[tt][0], sacc[tt][1]), nm2), a0, a1);
+            f2_unpack(f2_add(f2_pack(sacc[tt][2], sacc[tt][3]), nm2), a2, a3);
+            p0 = ex2_fast(a0);
+            p1 = ex2_fast(a1);
+            p2 = ex2_fast(a2);
+            p3 = ex2_fast(a3);
+            f2_unpack(f2_add(f2_pack(l0, l1), f2_add(f2_pack(p0, p1), f2_pack(p2, p3))), l0, l1);
+          } else {
+            p0 = exp2f(sacc[tt][0] - m0);
+            p1 = exp2f(sacc[tt][1] - m1);
+            p2 = exp2f(sacc[tt][2] - m0);
+            p3 = exp2f(sacc[tt][3] - m1);
+            l0 += p0 + p2;
+            l1 += p1 + p3;
+          }
           pb[tt][0] = movmatrix_t(pack2<MBF>(p0, p1));
           pb[tt][1] = movmatrix_t(pack2<MBF>(p2, p3));
         }
