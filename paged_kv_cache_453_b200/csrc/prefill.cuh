@@ -330,28 +330,36 @@ __global__ void __launch_bounds__(NW * 32, 1) prefill_kernel(const __grid_consta
             x3 = k1 <= lim[jt][1] ? x3 : -INFINITY;
           }
           float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+          // The exponent base moves only when a score passes it by more than
+          // 8 (P stays at or below 2^8, rounded to 16 bits with the same
+          // relative error): until then neither the column maxima across the
+          // warp nor a rescale of O is needed. When it moves it becomes the
+          // column's running maximum. A column with no key yet (every key so
+          // far past its position, only in a later KV chunk) keeps m = -inf,
+          // l = 0, O = 0, and its exponent base is 0 instead of -inf.
+          if (__any_sync(0xffffffffu, mx0 > mrun[jt][0] + 8.f || mx1 > mrun[jt][1] + 8.f)) {
 #pragma unroll
-          for (int o = 4; o < 32; o <<= 1) {
-            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
-          }
-          // A column with no key yet (every key so far past its position, only
-          // in a later KV chunk) keeps m = -inf, l = 0, O = 0: the exponent
-          // base is then 0 instead of -inf.
-          const float mn0 = fmaxf(mrun[jt][0], mx0), mn1 = fmaxf(mrun[jt][1], mx1);
-          const float b0 = mn0 == -INFINITY ? 0.f : mn0, b1 = mn1 == -INFINITY ? 0.f : mn1;
-          const float al0 = ex2_fast(mrun[jt][0] - b0), al1 = ex2_fast(mrun[jt][1] - b1);
-          lrun[jt][0] *= al0;
-          lrun[jt][1] *= al1;
+            for (int o = 4; o < 32; o <<= 1) {
+              mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+              mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+            }
+            const float mn0 = fmaxf(mrun[jt][0], mx0), mn1 = fmaxf(mrun[jt][1], mx1);
+            const float n0 = mn0 == -INFINITY ? 0.f : mn0, n1 = mn1 == -INFINITY ? 0.f : mn1;
+            const float al0 = ex2_fast(mrun[jt][0] - n0), al1 = ex2_fast(mrun[jt][1] - n1);
+            lrun[jt][0] *= al0;
+            lrun[jt][1] *= al1;
 #pragma unroll
-          for (int mt = 0; mt < C::MT; ++mt) {
-            acc[jt][mt][0] *= al0;
-            acc[jt][mt][1] *= al1;
-            acc[jt][mt][2] *= al0;
-            acc[jt][mt][3] *= al1;
+            for (int mt = 0; mt < C::MT; ++mt) {
+              acc[jt][mt][0] *= al0;
+              acc[jt][mt][1] *= al1;
+              acc[jt][mt][2] *= al0;
+              acc[jt][mt][3] *= al1;
+            }
+            mrun[jt][0] = mn0;
+            mrun[jt][1] = mn1;
           }
-          mrun[jt][0] = mn0;
-          mrun[jt][1] = mn1;
+          const float b0 = mrun[jt][0] == -INFINITY ? 0.f : mrun[jt][0];
+          const float b1 = mrun[jt][1] == -INFINITY ? 0.f : mrun[jt][1];
           const float p0 = ex2_fast(x0 - b0), p1 = ex2_fast(x1 - b1);
           const float p2 = ex2_fast(x2 - b0), p3 = ex2_fast(x3 - b1);
           lrun[jt][0] += p0 + p2;
