@@ -442,11 +442,14 @@ int launch_decode(const DecodeArgs& a, bool fp8, void* ws, size_t ws_bytes, bool
   p.steal = fixed_split ? 0 : 1;
   // The adaptive partition pays off where the per-warp speed differences
   // repeat from call to call: the fp8 kernel is issue-bound and a range of
-  // many short sequences is slower than one of few long ones. The 16-bit
-  // kernels are HBM-bound; their speed differences follow the SMs the CTAs
-  // land on, which change between calls, and equal ranges plus stealing do
-  // better there.
-  p.adapt = fp8 && !fixed_split && nwt <= 128 * kAdaptPer ? 1 : 0;
+  // many short sequences is slower than one of few long ones. With fewer
+  // (sequence, kv head) units than warp ranges every range lies inside one
+  // or two long units, and the speed differences follow the SMs the CTAs
+  // land on, which change between calls; so do those of the HBM-bound
+  // 16-bit kernels. Equal ranges plus stealing do better there (fp8
+  // llama3_8b shape, 512 units for 1184 ranges: 65.7 against 68.8 us).
+  const long long units = static_cast<long long>(p.S) * a.Hk;
+  p.adapt = fp8 && !fixed_split && nwt <= 128 * kAdaptPer && units >= nwt ? 1 : 0;
   p.pool_slots = L.pool_slots;
   uint8_t* w = static_cast<uint8_t*>(ws);
   p.hdr = reinterpret_cast<long long*>(w + L.hdr);

@@ -251,13 +251,15 @@ def test_deterministic_flag_gives_identical_bits(name):
 
 def test_fp8_adaptive_partition_across_shapes():
     # The fp8 decode cuts its static ranges by weights the previous call
-    # learned (kept in the workspace). Alternate two batches of one kernel
-    # configuration on one workspace, so that most calls run on a partition
-    # learned from the other batch: every call must still match the oracle,
-    # and a PKV_DECODE_DETERMINISTIC call (equal ranges, no stealing) must
-    # give the same bits whatever the learned state.
-    a = decode_case(W.scaled_down(W.spec("long_skewed"), 48, 3000, cache_dtype="fp8_e4m3"), seed=71)
-    b = decode_case(W.scaled_down(W.spec("llama3_8b"), 24, 2500, cache_dtype="fp8_e4m3"), seed=72)
+    # learned (kept in the workspace) when the batch has at least as many
+    # (sequence, kv head) units as warp ranges (1184 on a B200). Alternate
+    # two such batches of one kernel configuration on one workspace, so that
+    # most calls run on a partition learned from the other batch: every call
+    # must still match the oracle, and a PKV_DECODE_DETERMINISTIC call (equal
+    # ranges, no stealing) must give the same bits whatever the learned state.
+    a = decode_case(W.scaled_down(W.spec("long_skewed"), 160, 3000, cache_dtype="fp8_e4m3"), seed=71)
+    b = decode_case(W.scaled_down(W.spec("llama3_8b"), 150, 900, cache_dtype="fp8_e4m3"), seed=72)
+    assert a[0].num_seqs * a[0].num_kv_heads >= 1184 and b[0].num_seqs * b[0].num_kv_heads >= 1184
     s0 = a[0]
     nbytes = P.workspace_bytes(s0.num_q_heads, s0.num_kv_heads, s0.head_dim, s0.block_size,
                                P.PKV_FP8_E4M3, torch.cuda.current_device())
