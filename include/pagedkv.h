@@ -171,7 +171,12 @@ size_t paged_attn_decode_workspace_bytes(int num_q_heads, int num_kv_heads, int 
  * (e.g. cudaMemset): it holds the split-KV work-claiming state, which every
  * call leaves zeroed again. The workspace must not be used by another call
  * until this one has finished on the GPU; after a PKV_ERR_DEVICE_CHECK from
- * a call that used it, zero it again.
+ * a call that used it, zero it again. With an fp8 cache, and a batch with at
+ * least as many (sequence, kv head) units as the call has warp ranges, the
+ * workspace also carries from call to call how the work was split: each
+ * call learns from its warps' times where the next call should cut the
+ * work (results do not depend on it; a workspace shared by very different
+ * batches only balances less well).
  *
  * flags: 0, or PKV_DECODE_DETERMINISTIC. By default a warp that runs out of
  * work takes over part of another warp's remaining blocks, so where a
