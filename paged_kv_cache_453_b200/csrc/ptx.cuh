@@ -1,5 +1,6 @@
 // Thin inline-PTX wrappers used by the sm_100a kernels: mbarriers, TMA
-// tensor loads, ldmatrix / movmatrix, warp-level MMA and fp8 conversion.
+// tensor loads, ldmatrix / movmatrix, warp-level MMA, fp8 conversion, the
+// one-instruction 2^x and packed f32x2 arithmetic.
 #pragma once
 
 #include <cuda.h>
@@ -155,12 +156,6 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
   uint64_t d;
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
-}
-// 2^x by ex2_fast where FAST, else by exp2f
-template <bool FAST>
-__device__ __forceinline__ float ex2(float x) {
-  if constexpr (FAST) return ex2_fast(x);
-  else return exp2f(x);
 }
 __device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t v, uint32_t& lo, uint32_t& hi) {
   asm("{\n\t.reg .b16 l, h;\n\t"
