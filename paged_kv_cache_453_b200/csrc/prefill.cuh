@@ -321,8 +321,11 @@ __global__ void __launch_bounds__(NW * 32, 1) prefill_kernel(const __grid_consta
         uint32_t pb[2][2];
 #pragma unroll
         for (int jt = 0; jt < 2; ++jt) {
-          float x0 = sacc[jt][0] * slj[jt][0], x1 = sacc[jt][1] * slj[jt][1];
-          float x2 = sacc[jt][2] * slj[jt][0], x3 = sacc[jt][3] * slj[jt][1];
+          // a lane's two columns as packed f32x2 pairs
+          const uint64_t sl2 = f2_pack(slj[jt][0], slj[jt][1]);
+          float x0, x1, x2, x3;
+          f2_unpack(f2_mul(f2_pack(sacc[jt][0], sacc[jt][1]), sl2), x0, x1);
+          f2_unpack(f2_mul(f2_pack(sacc[jt][2], sacc[jt][3]), sl2), x2, x3);
           if (masked) {
             x0 = k0 <= lim[jt][0] ? x0 : -INFINITY;
             x1 = k0 <= lim[jt][1] ? x1 : -INFINITY;
@@ -358,12 +361,15 @@ __global__ void __launch_bounds__(NW * 32, 1) prefill_kernel(const __grid_consta
             mrun[jt][0] = mn0;
             mrun[jt][1] = mn1;
           }
-          const float b0 = mrun[jt][0] == -INFINITY ? 0.f : mrun[jt][0];
-          const float b1 = mrun[jt][1] == -INFINITY ? 0.f : mrun[jt][1];
-          const float p0 = ex2_fast(x0 - b0), p1 = ex2_fast(x1 - b1);
-          const float p2 = ex2_fast(x2 - b0), p3 = ex2_fast(x3 - b1);
-          lrun[jt][0] += p0 + p2;
-          lrun[jt][1] += p1 + p3;
+          const uint64_t nb2 = f2_pack(mrun[jt][0] == -INFINITY ? 0.f : -mrun[jt][0],
+                                       mrun[jt][1] == -INFINITY ? 0.f : -mrun[jt][1]);
+          float a0, a1, a2, a3;
+          f2_unpack(f2_add(f2_pack(x0, x1), nb2), a0, a1);
+          f2_unpack(f2_add(f2_pack(x2, x3), nb2), a2, a3);
+          const float p0 = ex2_fast(a0), p1 = ex2_fast(a1);
+          const float p2 = ex2_fast(a2), p3 = ex2_fast(a3);
+          f2_unpack(f2_add(f2_pack(lrun[jt][0], lrun[jt][1]), f2_add(f2_pack(p0, p1), f2_pack(p2, p3))),
+                    lrun[jt][0], lrun[jt][1]);
           pb[jt][0] = movmatrix_t(pack2<QBF && !FP8>(p0, p1));
           pb[jt][1] = movmatrix_t(pack2<QBF && !FP8>(p2, p3));
         }
